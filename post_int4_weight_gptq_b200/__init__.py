@@ -1,0 +1,302 @@
+"""B200 (sm_100a) layer-wise INT4/INT3 weight quantization: GPTQ and AWQ.
+
+A thin binding over the C ABI of ``lib/libpiq.so`` (declared in
+``include/piq.h``).  The functions here only marshal arguments: PyTorch
+supplies device memory and the current CUDA stream, and every step of the
+quantization runs in the library's own CUDA kernels.  There is no CPU path:
+if the library is missing or the device is not a B200, calls raise.
+
+Methods (web pages on the subject, cited by title and section):
+* GPTQ - "GPTQ versus AWQ objectives", "A strong answer" (the column loop with
+  error feedback through the upper Cholesky factor of the inverse proxy
+  Hessian, group scales, block-batched updates) and "What interviewers probe
+  next" (act-order, damping).
+* AWQ  - same page, AWQ paragraph: per-channel scales mean|x_j|^alpha, one
+  alpha per layer by grid search on the calibration output error.
+"""
+from __future__ import annotations
+
+import collections
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libpiq.so")
+
+PIQ_OK = 0
+PIQ_ERR_INVALID_ARG = -1
+PIQ_ERR_WORKSPACE_TOO_SMALL = -2
+PIQ_ERR_NOT_PD = -3
+PIQ_ERR_CUDA = -4
+PIQ_ERR_TIMEOUT = -5
+PIQ_ERR_UNSUPPORTED_DEVICE = -6
+
+AWQ_DEFAULT_GRID = tuple(k / 20.0 for k in range(20))
+
+_c_i64 = ctypes.c_int64
+_c_int = ctypes.c_int
+_c_float = ctypes.c_float
+_c_size_p = ctypes.POINTER(ctypes.c_size_t)
+_vp = ctypes.c_void_p
+
+# name -> (restype, argtypes); kept in the order of include/piq.h
+SIGNATURES = {
+    "piq_status_string": (ctypes.c_char_p, [_c_int]),
+    "piq_hessian_bytes": (_c_int, [_c_i64, _c_size_p]),
+    "piq_hessian": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_int, _vp]),
+    "piq_upper_factor_workspace_bytes": (_c_int, [_c_i64, _c_size_p]),
+    "piq_upper_factor": (_c_int, [_vp, _c_i64, _c_float, _vp, _vp,
+                                  ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t, _vp]),
+    "piq_gptq_sweep_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_size_p]),
+    "piq_gptq_sweep": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_int, _c_int, _vp, _vp, _vp,
+                                ctypes.c_size_t, _vp]),
+    "piq_gptq_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_size_p]),
+    "gptq_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int, _c_float,
+                                     _c_int, _vp, _vp, _vp, _vp,
+                                     ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
+                                     _vp]),
+    "piq_awq_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_size_p]),
+    "awq_search_layer": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int,
+                                  ctypes.POINTER(ctypes.c_float), _c_int,
+                                  ctypes.POINTER(ctypes.c_float), _vp, _vp, _vp,
+                                  ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t, _vp]),
+    "piq_rtn_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_size_p]),
+    "piq_rtn_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp,
+                                        ctypes.c_size_t, _vp]),
+    "piq_output_error_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_size_p]),
+    "piq_layer_output_error": (_c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _c_int, _c_int,
+                                        _vp, _c_i64, ctypes.POINTER(ctypes.c_double), _vp,
+                                        ctypes.c_size_t, _vp]),
+    "piq_set_timing": (_c_int, [_c_int]),
+    "piq_last_phase_times": (_c_int, [ctypes.POINTER(ctypes.c_double), _c_int,
+                                      ctypes.POINTER(_c_int)]),
+    "piq_phase_name": (ctypes.c_char_p, [_c_int]),
+    "piq_kernel_launches": (ctypes.c_uint64, []),
+}
+
+_lib = None
+
+
+class PiqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libpiq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m post_int4_weight_gptq_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().piq_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != PIQ_OK:
+        raise PiqError(rc, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes: int, device, workspace=None):
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _query(fn, *args) -> int:
+    out = ctypes.c_size_t(0)
+    _check(fn(*args, ctypes.byref(out)), fn.__name__)
+    return int(out.value)
+
+
+# ------------------------------------------------------------------ entry points
+def hessian_bytes(inp: int) -> int:
+    return _query(load_library().piq_hessian_bytes, inp)
+
+
+def hessian(X, H=None, accumulate=False, stream=None):
+    """H = X^T X (upper triangle valid), fp32 [in, in]."""
+    lib = load_library()
+    _need(X, torch.bfloat16, "X")
+    n, inp = X.shape
+    if H is None:
+        H = torch.empty(inp, inp, dtype=torch.float32, device=X.device)
+    _need(H, torch.float32, "H")
+    _check(lib.piq_hessian(_ptr(X), n, inp, _ptr(H), int(bool(accumulate)), _stream(stream)),
+           "piq_hessian")
+    return H
+
+
+def upper_factor(H, damp=0.01, perm=None, stream=None, workspace=None):
+    """(U, lambda): U upper with inv(H[perm][:, perm] + lambda I) = U^T U."""
+    lib = load_library()
+    _need(H, torch.float32, "H")
+    inp = H.shape[0]
+    if perm is not None:
+        _need(perm, torch.int32, "perm")
+    U = torch.empty_like(H)
+    ws = _workspace(_query(lib.piq_upper_factor_workspace_bytes, inp), H.device, workspace)
+    lam = ctypes.c_double(0.0)
+    _check(lib.piq_upper_factor(_ptr(H), inp, float(damp), _ptr(perm), _ptr(U), ctypes.byref(lam),
+                                _ptr(ws), ws.numel(), _stream(stream)), "piq_upper_factor")
+    return U, lam.value
+
+
+def gptq_sweep(Wp, U, bits=4, g=128, stream=None, workspace=None):
+    """(codes int8 [out, in], qscale fp32 [out, ceil(in/g)]) in quantization order."""
+    lib = load_library()
+    _need(Wp, torch.float32, "Wp")
+    _need(U, torch.float32, "U")
+    out, inp = Wp.shape
+    codes = torch.empty(out, inp, dtype=torch.int8, device=Wp.device)
+    qscale = torch.empty(out, -(-inp // g), dtype=torch.float32, device=Wp.device)
+    ws = _workspace(_query(lib.piq_gptq_sweep_workspace_bytes, out, inp), Wp.device, workspace)
+    _check(lib.piq_gptq_sweep(_ptr(Wp), out, inp, _ptr(U), bits, g, _ptr(codes), _ptr(qscale),
+                              _ptr(ws), ws.numel(), _stream(stream)), "piq_gptq_sweep")
+    return codes, qscale
+
+
+GPTQOutput = collections.namedtuple("GPTQOutput", "qweight scales perm g_idx err")
+AWQOutput = collections.namedtuple("AWQOutput", "best_alpha s qweight scales err_per_alpha")
+
+
+def gptq_workspace_bytes(out, inp, n, act_order=False) -> int:
+    return _query(load_library().piq_gptq_workspace_bytes, out, inp, n, int(bool(act_order)))
+
+
+def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_error=True,
+                        stream=None, workspace=None, out=None):
+    """GPTQ of one layer W [out, in] (fp32) on calibration X [n, in] (bf16)."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    _need(X, torch.bfloat16, "X")
+    rows, inp = W.shape
+    n = X.shape[0]
+    if X.shape[1] != inp:
+        raise ValueError("W and X disagree on the input dimension")
+    dev = W.device
+    if out is None:
+        out = GPTQOutput(torch.empty(rows, inp // 8, dtype=torch.int32, device=dev),
+                         torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev), None)
+    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order), dev, workspace)
+    err = ctypes.c_double(0.0)
+    _check(lib.gptq_quantize_layer(_ptr(W), rows, inp, _ptr(X), n, bits, g, float(damp),
+                                   int(bool(act_order)), _ptr(out.qweight), _ptr(out.scales),
+                                   _ptr(out.perm), _ptr(out.g_idx),
+                                   ctypes.byref(err) if with_error else None, _ptr(ws),
+                                   ws.numel(), _stream(stream)), "gptq_quantize_layer")
+    return out._replace(err=err.value if with_error else None)
+
+
+def awq_workspace_bytes(out, inp, n, n_alpha) -> int:
+    return _query(load_library().piq_awq_workspace_bytes, out, inp, n, n_alpha)
+
+
+def awq_search_layer(W, X, bits=4, g=128, alpha_grid=AWQ_DEFAULT_GRID, stream=None,
+                     workspace=None):
+    """AWQ scale search of one layer; returns the chosen alpha, s, packed codes, scales, errors."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    _need(X, torch.bfloat16, "X")
+    rows, inp = W.shape
+    n = X.shape[0]
+    na = len(alpha_grid)
+    dev = W.device
+    grid = (ctypes.c_float * na)(*[float(a) for a in alpha_grid])
+    errs = (ctypes.c_double * na)()
+    best = ctypes.c_float(0.0)
+    s = torch.empty(inp, dtype=torch.float32, device=dev)
+    qweight = torch.empty(rows, inp // 8, dtype=torch.int32, device=dev)
+    scales = torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev)
+    ws = _workspace(awq_workspace_bytes(rows, inp, n, na), dev, workspace)
+    _check(lib.awq_search_layer(_ptr(W), rows, inp, _ptr(X), n, bits, g, grid, na,
+                                ctypes.byref(best), _ptr(s), _ptr(qweight), _ptr(scales), errs,
+                                _ptr(ws), ws.numel(), _stream(stream)), "awq_search_layer")
+    return AWQOutput(best.value, s, qweight, scales, list(errs))
+
+
+def rtn_quantize_layer(W, bits=4, g=128, stream=None, workspace=None):
+    """Plain group round-to-nearest: (qweight, scales)."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    rows, inp = W.shape
+    dev = W.device
+    qweight = torch.empty(rows, inp // 8, dtype=torch.int32, device=dev)
+    scales = torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev)
+    ws = _workspace(_query(lib.piq_rtn_workspace_bytes, rows, inp), dev, workspace)
+    _check(lib.piq_rtn_quantize_layer(_ptr(W), rows, inp, bits, g, _ptr(qweight), _ptr(scales),
+                                      _ptr(ws), ws.numel(), _stream(stream)),
+           "piq_rtn_quantize_layer")
+    return qweight, scales
+
+
+def output_error_workspace_bytes(out, inp, n) -> int:
+    return _query(load_library().piq_output_error_workspace_bytes, out, inp, n)
+
+
+def layer_output_error(W, qweight, scales, X, bits=4, g=128, g_idx=None, s=None, stream=None,
+                       workspace=None) -> float:
+    """||X W^T - X What^T||^2 of a packed layer on inputs X."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    _need(X, torch.bfloat16, "X")
+    rows, inp = W.shape
+    n = X.shape[0]
+    ws = _workspace(_query(lib.piq_output_error_workspace_bytes, rows, inp, n), W.device,
+                    workspace)
+    e = ctypes.c_double(0.0)
+    _check(lib.piq_layer_output_error(_ptr(W), rows, inp, _ptr(qweight), _ptr(scales),
+                                      _ptr(g_idx), _ptr(s), bits, g, _ptr(X), n, ctypes.byref(e),
+                                      _ptr(ws), ws.numel(), _stream(stream)),
+           "piq_layer_output_error")
+    return e.value
+
+
+def set_timing(enable: bool):
+    load_library().piq_set_timing(int(bool(enable)))
+
+
+def last_phase_times() -> dict:
+    lib = load_library()
+    buf = (ctypes.c_double * 8)()
+    n = ctypes.c_int(0)
+    lib.piq_last_phase_times(buf, 8, ctypes.byref(n))
+    return {lib.piq_phase_name(i).decode(): buf[i] for i in range(min(n.value, 8))}
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libpiq in this process so far."""
+    return int(load_library().piq_kernel_launches())

@@ -1,0 +1,569 @@
+// C-ABI entry points (include/piq.h): argument checks, workspace carving and
+// the order of the steps.  Every step of the path runs in this library's
+// kernels on the caller's stream; the host only launches and, at the end,
+// reads back the status word and the host scalars.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace piq {
+
+// ------------------------------------------------------------------ devices
+int device_info(DeviceInfo* out) {
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 64) return PIQ_ERR_CUDA;
+  if (!have[dev]) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return PIQ_ERR_CUDA;
+    cache[dev].sm_count = prop.multiProcessorCount;
+    cache[dev].major = prop.major;
+    cache[dev].minor = prop.minor;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  return cache[dev].major == 10 ? PIQ_OK : PIQ_ERR_UNSUPPORTED_DEVICE;
+}
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int count) { g_launches.fetch_add(static_cast<uint64_t>(count)); }
+
+namespace {
+
+// Bump allocator over the caller's workspace; with base == nullptr it only
+// measures, so the *_workspace_bytes queries and the carving share one layout.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(int64_t count) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += static_cast<size_t>(std::max<int64_t>(count, 1)) * sizeof(T);
+    return p;
+  }
+  size_t bytes() const { return (off + 255) & ~static_cast<size_t>(255); }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_layer(int64_t out, int64_t in, int bits, int g) {
+  if (out < 1 || in < 8 || in % 8 != 0) return PIQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4 || g < 1) return PIQ_ERR_INVALID_ARG;
+  if (in > (int64_t)1 << 20 || out > (int64_t)1 << 24) return PIQ_ERR_INVALID_ARG;
+  return PIQ_OK;
+}
+
+// ------------------------------------------------------------- phase timing
+constexpr int kMaxPhases = 8;
+const char* kPhaseNames[2][kMaxPhases] = {
+    {"hessian", "act_order", "factor", "sweep", "pack", "error", nullptr, nullptr},
+    {"colstats", "quant_delta", "error_gemm", "select_pack", nullptr, nullptr, nullptr, nullptr}};
+
+struct Timing {
+  bool enabled = false;
+  int kind = 0;  // 0 gptq, 1 awq
+  int n = 0;
+  cudaEvent_t ev[kMaxPhases + 1] = {};
+  bool created = false;
+  double last_ms[kMaxPhases] = {};
+  int last_n = 0;
+  int last_kind = 0;
+};
+Timing g_timing;
+std::mutex g_timing_mu;
+
+struct PhaseClock {
+  bool on;
+  cudaStream_t s;
+  int idx = 0;
+  PhaseClock(int kind, cudaStream_t stream) : on(false), s(stream) {
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    if (!g_timing.enabled) return;
+    if (!g_timing.created) {
+      for (auto& e : g_timing.ev)
+        if (cudaEventCreate(&e) != cudaSuccess) return;
+      g_timing.created = true;
+    }
+    g_timing.kind = kind;
+    on = true;
+    cudaEventRecord(g_timing.ev[0], s);
+  }
+  void mark() {  // end of the current phase
+    if (!on || idx >= kMaxPhases) return;
+    cudaEventRecord(g_timing.ev[++idx], s);
+  }
+  void finish() {  // after the stream synchronized
+    if (!on) return;
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    for (int i = 0; i < idx; ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, g_timing.ev[i], g_timing.ev[i + 1]);
+      g_timing.last_ms[i] = ms;
+    }
+    g_timing.last_n = idx;
+    g_timing.last_kind = g_timing.kind;
+  }
+};
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA; }
+
+// Read the status word (and optional extra device bytes) after synchronizing.
+int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st) {
+  DeviceStatus tmp;
+  if (cudaMemcpyAsync(&tmp, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, stream) !=
+      cudaSuccess)
+    return PIQ_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PIQ_ERR_CUDA;
+  if (host_st) *host_st = tmp;
+  return tmp.code;
+}
+
+#define PIQ_TRY(expr)             \
+  do {                            \
+    const int rc_ = (expr);       \
+    if (rc_ != PIQ_OK) return rc_; \
+  } while (0)
+
+// ------------------------------------------------------------ layouts
+struct FactorWs {
+  DeviceStatus* st;
+  float* work;
+};
+FactorWs carve_factor(Carver& c, int64_t in) {
+  FactorWs w;
+  w.st = c.take<DeviceStatus>(1);
+  w.work = c.take<float>(factor_workspace_floats(in));
+  return w;
+}
+
+struct SweepWs {
+  DeviceStatus* st;
+  float* Wq;
+  float* Err;
+};
+SweepWs carve_sweep(Carver& c, int64_t out, int64_t in) {
+  SweepWs w;
+  w.st = c.take<DeviceStatus>(1);
+  w.Wq = c.take<float>(out * in);
+  w.Err = c.take<float>(out * kSweepB);
+  return w;
+}
+
+struct GptqWs {
+  DeviceStatus* st;
+  float* H;  // becomes U
+  float* fwork;
+  float* Wq;
+  float* Err;
+  int8_t* codes;
+  float* qscale;
+  uint16_t* dW;
+  int32_t* perm;
+  int32_t* invperm;
+  double* colpart;
+  double* sumsq;
+  double* partials;
+  double* err;
+};
+GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int act_order) {
+  GptqWs w;
+  w.st = c.take<DeviceStatus>(1);
+  w.H = c.take<float>(in * in);
+  w.fwork = c.take<float>(factor_workspace_floats(in));
+  w.Wq = c.take<float>(out * in);
+  w.Err = c.take<float>(out * kSweepB);
+  w.codes = c.take<int8_t>(out * in);
+  w.qscale = c.take<float>(out * ceil_div(in, 1));  // sized for g >= 1
+  w.dW = c.take<uint16_t>(out * in);
+  w.perm = c.take<int32_t>(in);
+  w.invperm = c.take<int32_t>(in);
+  w.colpart = c.take<double>(act_order ? static_cast<int64_t>(colstats_splits(n, in)) * in * 2 : 1);
+  w.sumsq = c.take<double>(in);
+  w.partials = c.take<double>(sumsq_partials_count(n, out, 1));
+  w.err = c.take<double>(1);
+  return w;
+}
+
+struct AwqWs {
+  DeviceStatus* st;
+  double* colpart;
+  double* mean_abs;
+  float* alphas;
+  float* s_table;
+  uint16_t* dW;
+  double* partials;
+  double* err;
+  int* best;
+  float* best_alpha;
+  int8_t* codes;
+  float* qscale;
+};
+AwqWs carve_awq(Carver& c, int64_t out, int64_t in, int64_t n, int n_alpha) {
+  AwqWs w;
+  w.st = c.take<DeviceStatus>(1);
+  w.colpart = c.take<double>(static_cast<int64_t>(colstats_splits(n, in)) * in * 2);
+  w.mean_abs = c.take<double>(in);
+  w.alphas = c.take<float>(64);
+  w.s_table = c.take<float>(static_cast<int64_t>(n_alpha) * in);
+  w.dW = c.take<uint16_t>(static_cast<int64_t>(n_alpha) * out * in);
+  w.partials = c.take<double>(sumsq_partials_count(n, out, n_alpha));
+  w.err = c.take<double>(64);
+  w.best = c.take<int>(1);
+  w.best_alpha = c.take<float>(1);
+  w.codes = c.take<int8_t>(out * in);
+  w.qscale = c.take<float>(out * in);  // sized for g >= 1
+  return w;
+}
+
+struct RtnWs {
+  int8_t* codes;
+  float* qscale;
+};
+RtnWs carve_rtn(Carver& c, int64_t out, int64_t in) {
+  RtnWs w;
+  w.codes = c.take<int8_t>(out * in);
+  w.qscale = c.take<float>(out * in);  // sized for g >= 1
+  return w;
+}
+
+struct ErrWs {
+  DeviceStatus* st;
+  uint16_t* dW;
+  double* partials;
+  double* err;
+};
+ErrWs carve_err(Carver& c, int64_t out, int64_t in, int64_t n) {
+  ErrWs w;
+  w.st = c.take<DeviceStatus>(1);
+  w.dW = c.take<uint16_t>(out * in);
+  w.partials = c.take<double>(sumsq_partials_count(n, out, 1));
+  w.err = c.take<double>(1);
+  return w;
+}
+
+int check_ws(void* ws, size_t have, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PIQ_ERR_INVALID_ARG;
+  return have >= need ? PIQ_OK : PIQ_ERR_WORKSPACE_TOO_SMALL;
+}
+
+}  // namespace
+}  // namespace piq
+
+using namespace piq;
+
+extern "C" {
+
+const char* piq_status_string(int status) {
+  switch (status) {
+    case PIQ_OK: return "ok";
+    case PIQ_ERR_INVALID_ARG: return "invalid argument";
+    case PIQ_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case PIQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case PIQ_ERR_CUDA: return "CUDA error";
+    case PIQ_ERR_TIMEOUT: return "bounded device wait timed out";
+    case PIQ_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    default: return "unknown status";
+  }
+}
+
+int piq_hessian_bytes(int64_t in, size_t* bytes) {
+  if (bytes == nullptr || in < 1) return PIQ_ERR_INVALID_ARG;
+  *bytes = static_cast<size_t>(in) * static_cast<size_t>(in) * sizeof(float);
+  return PIQ_OK;
+}
+
+int piq_hessian(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
+                void* stream) {
+  if (X == nullptr || H == nullptr || !aligned16(X) || !aligned16(H)) return PIQ_ERR_INVALID_ARG;
+  if (n < 1 || in < 8 || in % 8 != 0) return PIQ_ERR_INVALID_ARG;
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  return launch_syrk_xtx(X, n, in, H, accumulate, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int piq_upper_factor_workspace_bytes(int64_t in, size_t* bytes) {
+  if (bytes == nullptr || in < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_factor(c, in);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int piq_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm, float* U,
+                     double* lambda_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (H == nullptr || U == nullptr || in < 1 || !(damp >= 0.f)) return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_upper_factor_workspace_bytes(in, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  FactorWs w = carve_factor(c, in);
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  PIQ_TRY(run_upper_factor(H, in, damp, perm, U, w.work, w.st, s));
+  DeviceStatus hs;
+  const int rc = finish_call(w.st, s, &hs);
+  if (lambda_out) *lambda_out = hs.lambda;
+  return rc;
+}
+
+int piq_gptq_sweep_workspace_bytes(int64_t out, int64_t in, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_sweep(c, out, in);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int bits, int g,
+                   int8_t* codes, float* qscale, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (Wp == nullptr || U == nullptr || codes == nullptr || qscale == nullptr)
+    return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_gptq_sweep_workspace_bytes(out, in, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  SweepWs w = carve_sweep(c, out, in);
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  PIQ_TRY(cuda_rc(cudaMemcpyAsync(w.Wq, Wp, sizeof(float) * out * in, cudaMemcpyDeviceToDevice, s)));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, codes, qscale, w.Err, w.st, s));
+  return finish_call(w.st, s, nullptr);
+}
+
+int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int act_order, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1 || n < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
+                        int bits, int g, float damp, int act_order, uint32_t* qweight,
+                        uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || X == nullptr || qweight == nullptr || scales == nullptr || n < 1 ||
+      !(damp >= 0.f) || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
+    return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_gptq_workspace_bytes(out, in, n, act_order, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  GptqWs w = carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  PhaseClock clk(0, s);
+
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  // 1. H = X^T X on the tensor cores
+  PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
+  clk.mark();
+  // 2. quantization order
+  const int32_t* qperm = nullptr;
+  const int32_t* qinv = nullptr;
+  if (act_order) {
+    PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), nullptr, w.sumsq, s));
+    PIQ_TRY(launch_act_order_perm(w.sumsq, in, w.perm, w.invperm, s));
+    qperm = w.perm;
+    qinv = w.invperm;
+  }
+  if (perm) {
+    if (act_order)
+      PIQ_TRY(cuda_rc(cudaMemcpyAsync(perm, w.perm, sizeof(int32_t) * in, cudaMemcpyDeviceToDevice, s)));
+    else
+      PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
+  }
+  clk.mark();
+  // 3. damping + U (written over H)
+  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, w.H, w.fwork, w.st, s));
+  clk.mark();
+  // 4. blocked sweep on the permuted copy
+  PIQ_TRY(launch_gather_columns(W, out, in, qperm, w.Wq, s));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, w.H, bits, g, w.codes, w.qscale, w.Err, w.st, s));
+  clk.mark();
+  // 5. pack (+ D = W - What for the error)
+  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, qweight, scales,
+                      out_err ? w.dW : nullptr, g_idx, s));
+  clk.mark();
+  // 6. output error
+  if (out_err) {
+    PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
+    PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));
+  }
+  clk.mark();
+  double e = 0.0;
+  if (out_err)
+    PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
+  const int rc = finish_call(w.st, s, nullptr);
+  clk.finish();
+  if (out_err) *out_err = e;
+  return rc;
+}
+
+int piq_awq_workspace_bytes(int64_t out, int64_t in, int64_t n, int n_alpha, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1 || n < 1 || n_alpha < 1 || n_alpha > 64)
+    return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_awq(c, out, in, n, n_alpha);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
+                     int bits, int g, const float* alpha_grid, int n_alpha, float* best_alpha,
+                     float* s_out, uint32_t* qweight, uint16_t* scales, double* err_per_alpha,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || X == nullptr || alpha_grid == nullptr || s_out == nullptr ||
+      qweight == nullptr || scales == nullptr || n < 1 || n_alpha < 1 || n_alpha > 64 ||
+      !aligned16(W) || !aligned16(X) || !aligned16(qweight))
+    return PIQ_ERR_INVALID_ARG;
+  for (int a = 0; a < n_alpha; ++a)
+    if (!(alpha_grid[a] == alpha_grid[a])) return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_awq_workspace_bytes(out, in, n, n_alpha, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  AwqWs w = carve_awq(c, out, in, n, n_alpha);
+  PhaseClock clk(1, s);
+
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  PIQ_TRY(cuda_rc(cudaMemcpyAsync(w.alphas, alpha_grid, sizeof(float) * n_alpha,
+                                  cudaMemcpyHostToDevice, s)));
+  // 1. mean |x_j|
+  PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), w.mean_abs, nullptr, s));
+  clk.mark();
+  // 2. s = m^alpha for the grid, and D_alpha = W - code * scale / s
+  PIQ_TRY(launch_awq_scale_table(w.mean_abs, in, w.alphas, n_alpha, w.s_table, s));
+  PIQ_TRY(launch_awq_delta(W, out, in, bits, g, w.s_table, n_alpha, w.dW, s));
+  clk.mark();
+  // 3. E_alpha = ||X D_alpha^T||^2, every alpha in one tensor-core launch
+  PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, n_alpha, w.partials, w.st, s));
+  PIQ_TRY(launch_reduce_partials(w.partials, n, out, n_alpha, w.err, s));
+  clk.mark();
+  // 4. first minimum, re-quantize at it, pack
+  PIQ_TRY(launch_argmin(w.err, n_alpha, w.alphas, w.best, w.best_alpha, s));
+  PIQ_TRY(launch_group_quant(W, out, in, bits, g, w.s_table, w.best, w.codes, w.qscale, s_out, s));
+  PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
+                      nullptr, nullptr, s));
+  clk.mark();
+  double errs[64];
+  float ba = 0.f;
+  PIQ_TRY(cuda_rc(cudaMemcpyAsync(errs, w.err, sizeof(double) * n_alpha, cudaMemcpyDeviceToHost, s)));
+  PIQ_TRY(cuda_rc(cudaMemcpyAsync(&ba, w.best_alpha, sizeof(float), cudaMemcpyDeviceToHost, s)));
+  const int rc = finish_call(w.st, s, nullptr);
+  clk.finish();
+  if (err_per_alpha) std::memcpy(err_per_alpha, errs, sizeof(double) * n_alpha);
+  if (best_alpha) *best_alpha = ba;
+  return rc;
+}
+
+int piq_rtn_workspace_bytes(int64_t out, int64_t in, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_rtn(c, out, in);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, int g,
+                           uint32_t* qweight, uint16_t* scales, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || qweight == nullptr || scales == nullptr || !aligned16(W) ||
+      !aligned16(qweight))
+    return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_rtn_workspace_bytes(out, in, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  RtnWs w = carve_rtn(c, out, in);
+  PIQ_TRY(launch_group_quant(W, out, in, bits, g, nullptr, nullptr, w.codes, w.qscale, nullptr, s));
+  return launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
+                     nullptr, nullptr, s);
+}
+
+int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1 || n < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_err(c, out, in, n);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
+                           const uint16_t* scales, const int32_t* g_idx, const float* s_ch,
+                           int bits, int g, const uint16_t* X, int64_t n, double* out_err,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || qweight == nullptr || scales == nullptr || X == nullptr ||
+      out_err == nullptr || n < 1 || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
+    return PIQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_output_error_workspace_bytes(out, in, n, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  Carver c(workspace);
+  ErrWs w = carve_err(c, out, in, n);
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, w.dW, w.st, s));
+  PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
+  PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));
+  double e = 0.0;
+  PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
+  const int rc = finish_call(w.st, s, nullptr);
+  *out_err = e;
+  return rc;
+}
+
+int piq_set_timing(int enable) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  g_timing.enabled = enable != 0;
+  return PIQ_OK;
+}
+
+int piq_last_phase_times(double* ms, int max_phases, int* n_phases) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  const int n = std::min(max_phases, g_timing.last_n);
+  for (int i = 0; i < n; ++i) ms[i] = g_timing.last_ms[i];
+  if (n_phases) *n_phases = g_timing.last_n;
+  return PIQ_OK;
+}
+
+uint64_t piq_kernel_launches(void) { return g_launches.load(); }
+
+const char* piq_phase_name(int i) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (i < 0 || i >= kMaxPhases) return nullptr;
+  return kPhaseNames[g_timing.last_kind][i];
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace piq {
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+  int sm_count = 0;
+  int major = 0;
+  int minor = 0;
+};
+int device_info(DeviceInfo* out);  // PIQ_OK / PIQ_ERR_CUDA / PIQ_ERR_UNSUPPORTED_DEVICE
+
+// Count one kernel launch (piq_kernel_launches).
+void note_launch(int count = 1);
+
+// ------------------------------------------------------ tensor-core GEMMs (tc_gemm.cu)
+// H (+)= X^T X: upper-triangle tiles of a [in, in] fp32 matrix (row-major).
+int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
+                    DeviceStatus* st, cudaStream_t stream);
+// Fused ||X D_b^T||_F^2 for b < batch, D stacked [batch][rows][in] bf16.
+// Writes four doubles per output tile into `partials` (size: sumsq_partials_count).
+int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D, int64_t rows,
+                     int batch, double* partials, DeviceStatus* st, cudaStream_t stream);
+int64_t sumsq_partials_count(int64_t n, int64_t rows, int batch);
+// Fixed-order sum of the partials of each batch entry into out[batch].
+int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,
+                           double* out, cudaStream_t stream);
+
+// ------------------------------------------------------ FP32 SIMT GEMM (simt_gemm.cu)
+// C = alpha * A * op(B) + beta * C, row-major; op(B) = B or B^T (trans_b).
+// mode 0: plain; 1: only tiles touching the lower triangle of C (M == N);
+// 2: A lower triangular (entries right of the diagonal are skipped per row tile).
+int launch_simt_gemm(int M, int N, int K, float alpha, const float* A, int64_t lda,
+                     const float* B, int64_t ldb, bool trans_b, float beta, float* C,
+                     int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream);
+
+// ------------------------------------------------------------- factor (factor.cu)
+constexpr int kFactorNB = 128;  // panel width of the blocked Cholesky / inverse
+int64_t factor_workspace_floats(int64_t in);  // P + Dinv + T
+int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm, float* U,
+                     float* work, DeviceStatus* st, cudaStream_t stream);
+int launch_act_order_perm(const double* sumsq, int64_t in, int32_t* perm, int32_t* invperm,
+                          cudaStream_t stream);
+int launch_identity_perm(int64_t in, int32_t* perm, int32_t* invperm, cudaStream_t stream);
+
+// ---------------------------------------------------------------- sweep (sweep.cu)
+constexpr int kSweepB = 128;
+// Full blocked sweep over quantization-order weights Wq (updated in place).
+int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits, int g,
+                   int8_t* codes, float* qscale, float* Err, DeviceStatus* st,
+                   cudaStream_t stream);
+
+// ------------------------------------------------- quantize / pack / stats (quant.cu)
+int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, int splits,
+                    double* mean_abs, double* sumsq, cudaStream_t stream);
+int colstats_splits(int64_t n, int64_t in);
+int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
+                          float* Wq, cudaStream_t stream);
+int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
+                int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
+                uint16_t* scales16, uint16_t* dW, int32_t* g_idx, cudaStream_t stream);
+int launch_awq_scale_table(const double* mean_abs, int64_t in, const float* alphas_dev,
+                           int n_alpha, float* s_table, cudaStream_t stream);
+int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,
+                     const float* s_table, int n_alpha, uint16_t* dW, cudaStream_t stream);
+int launch_group_quant(const float* W, int64_t out, int64_t in, int bits, int g,
+                       const float* s_table, const int* sel, int8_t* codes, float* qscale,
+                       float* s_out, cudaStream_t stream);
+int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_idx,
+                  float* best_alpha, cudaStream_t stream);
+int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
+                         const uint16_t* scales16, const int32_t* g_idx, const float* s,
+                         int bits, int g, uint16_t* dW, DeviceStatus* st,
+                         cudaStream_t stream);
+
+}  // namespace piq

@@ -1,0 +1,393 @@
+// Bandwidth-bound kernels of the quantization path.
+//
+//   colstats      per input channel: sum |x| (AWQ's mean|x_j|, "GPTQ versus AWQ
+//                 objectives", AWQ paragraph of "A strong answer") and sum x^2
+//                 (= diag(X^T X), the act-order key of "What interviewers probe
+//                 next"), one pass over X, FP64 accumulation.
+//   awq_delta     for every alpha of the grid: s = mean|x|^alpha, W' = W diag(s),
+//                 symmetric group round-to-nearest of W', and
+//                 D = W - code * scale / s stored as bf16 for the error GEMM.
+//   group_quant   codes + fp32 scales of W diag(s) for one s (AWQ's chosen alpha;
+//                 s = 1 gives plain group RTN, the toy table's first column).
+//   pack          codes -> uint32 nibbles, fp32 -> fp16 scales, act-order
+//                 column un-permutation and g_idx, and D = W - code * fp16(scale)
+//                 (bf16) for the output-error GEMM, in one pass.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace piq {
+
+namespace {
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// ------------------------------------------------------------------- colstats
+// grid (ceil(in/256), splits); 8 warps; lane owns 8 consecutive columns.
+__global__ void __launch_bounds__(256) colstats_kernel(const uint16_t* __restrict__ X, int64_t n,
+                                                       int64_t in, int splits,
+                                                       double* __restrict__ part) {
+  __shared__ double sh_abs[8][256];
+  __shared__ double sh_sq[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const int64_t rows_per = (n + splits - 1) / splits;
+  const int64_t r0 = blockIdx.y * rows_per;
+  const int64_t r1 = std::min<int64_t>(n, r0 + rows_per);
+  double sa[8], sq[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sa[i] = sq[i] = 0.0;
+  if (col < in) {
+    for (int64_t r = r0 + warp; r < r1; r += 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(X + r * in + col);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = bf16_bits_to_float(static_cast<uint16_t>(w[i] & 0xFFFFu));
+        const float hi = bf16_bits_to_float(static_cast<uint16_t>(w[i] >> 16));
+        sa[2 * i] += static_cast<double>(fabsf(lo));
+        sa[2 * i + 1] += static_cast<double>(fabsf(hi));
+        sq[2 * i] += static_cast<double>(lo * lo);  // exact: bf16 square fits fp32
+        sq[2 * i + 1] += static_cast<double>(hi * hi);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sh_abs[warp][lane * 8 + i] = sa[i];
+    sh_sq[warp][lane * 8 + i] = sq[i];
+  }
+  __syncthreads();
+  const int c = threadIdx.x;
+  const int64_t gc = static_cast<int64_t>(blockIdx.x) * 256 + c;
+  if (gc < in) {
+    double a = 0.0, q = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      a += sh_abs[w][c];
+      q += sh_sq[w][c];
+    }
+    part[(static_cast<int64_t>(blockIdx.y) * in + gc) * 2] = a;
+    part[(static_cast<int64_t>(blockIdx.y) * in + gc) * 2 + 1] = q;
+  }
+}
+
+__global__ void colstats_finish_kernel(const double* __restrict__ part, int64_t n, int64_t in,
+                                       int splits, double* mean_abs, double* sumsq) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= in) return;
+  double a = 0.0, q = 0.0;
+  for (int s = 0; s < splits; ++s) {
+    a += part[(static_cast<int64_t>(s) * in + c) * 2];
+    q += part[(static_cast<int64_t>(s) * in + c) * 2 + 1];
+  }
+  if (mean_abs) mean_abs[c] = a / static_cast<double>(n);
+  if (sumsq) sumsq[c] = q;
+}
+
+// --------------------------------------------------------------------- gather
+__global__ void gather_columns_kernel(const float* __restrict__ W, int64_t out, int64_t in,
+                                      const int32_t* __restrict__ perm, float* __restrict__ Wq) {
+  const int64_t total = out * in;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / in, p = idx - r * in;
+    Wq[idx] = W[r * in + (perm ? perm[p] : p)];
+  }
+}
+
+// ----------------------------------------------------------------------- pack
+// One thread per uint32 word (8 memory-order columns).
+__global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __restrict__ qscale,
+                            const int32_t* __restrict__ invperm, int64_t out, int64_t in,
+                            int bits, int g, const float* __restrict__ W0,
+                            uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales16,
+                            uint16_t* __restrict__ dW, int32_t* __restrict__ g_idx) {
+  const int64_t words = in / 8;
+  const int64_t ngroups = (in + g - 1) / g;
+  const int64_t total = out * words;
+  const int off = 1 << (bits - 1);
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / words, wd = idx - r * words;
+    const int8_t* crow = codes + r * in;
+    const float* srow = qscale + r * ngroups;
+    uint32_t word = 0;
+    uint16_t d16[8];
+    float w0[8];
+    if (dW) {
+      const float4 a = *reinterpret_cast<const float4*>(W0 + r * in + wd * 8);
+      const float4 b = *reinterpret_cast<const float4*>(W0 + r * in + wd * 8 + 4);
+      w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w;
+      w0[4] = b.x; w0[5] = b.y; w0[6] = b.z; w0[7] = b.w;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t c = wd * 8 + k;
+      const int64_t p = invperm ? invperm[c] : c;
+      const int code = crow[p];
+      word |= static_cast<uint32_t>(code + off) << (4 * k);
+      if (dW) {
+        const float s16 = __half2float(__float2half_rn(srow[p / g]));
+        d16[k] = float_to_bf16_bits(w0[k] - static_cast<float>(code) * s16);
+      }
+    }
+    qweight[idx] = word;
+    if (dW) {
+      uint4 o;
+      o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
+      o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
+      o.z = d16[4] | (static_cast<uint32_t>(d16[5]) << 16);
+      o.w = d16[6] | (static_cast<uint32_t>(d16[7]) << 16);
+      *reinterpret_cast<uint4*>(dW + r * in + wd * 8) = o;
+    }
+  }
+  // fp16 scales and the group index
+  const int64_t ns = out * ngroups;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < ns;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    scales16[idx] = __half_as_ushort(__float2half_rn(qscale[idx]));
+  if (g_idx) {
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < in;
+         c += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      g_idx[c] = static_cast<int32_t>((invperm ? invperm[c] : c) / g);
+  }
+}
+
+// ------------------------------------------------------------------------ AWQ
+__global__ void awq_scale_table_kernel(const double* __restrict__ mean_abs, int64_t in,
+                                       const float* __restrict__ alphas, int n_alpha,
+                                       float* __restrict__ s_table) {
+  const int64_t total = static_cast<int64_t>(n_alpha) * in;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int a = static_cast<int>(idx / in);
+    const double m = mean_abs[idx - a * in];
+    s_table[idx] = m > 0.0 ? static_cast<float>(pow(m, static_cast<double>(alphas[a]))) : 1.f;
+  }
+}
+
+// Group scale and codes of W diag(s) for one (row, group): one warp.
+struct GroupQ {
+  float scale;
+};
+
+__device__ __forceinline__ float group_scale(const float* wrow, const float* s, int64_t c0,
+                                             int64_t c1, float fqmax, int lane) {
+  float m = 0.f;
+  for (int64_t c = c0 + lane; c < c1; c += 32) {
+    const float v = s ? wrow[c] * s[c] : wrow[c];
+    m = fmaxf(m, fabsf(v));
+  }
+  return __fdiv_rn(warp_max(m), fqmax);
+}
+
+__device__ __forceinline__ float quant_code(float v, float scale, float cmin, float cmax) {
+  return scale > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(v, scale)), cmin), cmax) : 0.f;
+}
+
+// D_a[r][c] = W - code * scale / s for every alpha a; one warp per (row, group).
+__global__ void awq_delta_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits,
+                                 int g, const float* __restrict__ s_table, int n_alpha,
+                                 uint16_t* __restrict__ dW) {
+  const int64_t ngroups = (in + g - 1) / g;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int qmax = (1 << (bits - 1)) - 1;
+  const float fqmax = static_cast<float>(qmax), cmin = static_cast<float>(-qmax - 1),
+              cmax = static_cast<float>(qmax);
+  for (int64_t wi = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wi < out * ngroups; wi += nwarps) {
+    const int64_t r = wi / ngroups, grp = wi - r * ngroups;
+    const int64_t c0 = grp * g, c1 = std::min<int64_t>(in, c0 + g);
+    const float* wrow = W + r * in;
+    for (int a = 0; a < n_alpha; ++a) {
+      const float* s = s_table + static_cast<int64_t>(a) * in;
+      const float scale = group_scale(wrow, s, c0, c1, fqmax, lane);
+      uint16_t* drow = dW + (static_cast<int64_t>(a) * out + r) * in;
+      for (int64_t c = c0 + lane; c < c1; c += 32) {
+        const float w = wrow[c];
+        const float q = quant_code(w * s[c], scale, cmin, cmax);
+        drow[c] = float_to_bf16_bits(w - __fdiv_rn(q * scale, s[c]));
+      }
+    }
+  }
+}
+
+// codes + fp32 scales of W diag(s_table[sel]) (s_table == NULL: s = 1).
+__global__ void group_quant_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits,
+                                   int g, const float* __restrict__ s_table,
+                                   const int* __restrict__ sel, int8_t* __restrict__ codes,
+                                   float* __restrict__ qscale, float* __restrict__ s_out) {
+  const int64_t ngroups = (in + g - 1) / g;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int qmax = (1 << (bits - 1)) - 1;
+  const float fqmax = static_cast<float>(qmax), cmin = static_cast<float>(-qmax - 1),
+              cmax = static_cast<float>(qmax);
+  const float* s = s_table ? s_table + static_cast<int64_t>(sel ? *sel : 0) * in : nullptr;
+  for (int64_t wi = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wi < out * ngroups; wi += nwarps) {
+    const int64_t r = wi / ngroups, grp = wi - r * ngroups;
+    const int64_t c0 = grp * g, c1 = std::min<int64_t>(in, c0 + g);
+    const float* wrow = W + r * in;
+    const float scale = group_scale(wrow, s, c0, c1, fqmax, lane);
+    if (lane == 0) qscale[r * ngroups + grp] = scale;
+    for (int64_t c = c0 + lane; c < c1; c += 32) {
+      const float v = s ? wrow[c] * s[c] : wrow[c];
+      codes[r * in + c] = static_cast<int8_t>(quant_code(v, scale, cmin, cmax));
+    }
+  }
+  if (s_out && s) {
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < in;
+         c += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      s_out[c] = s[c];
+  }
+}
+
+__global__ void argmin_kernel(const double* err, int n, const float* alphas, int* best_idx,
+                              float* best_alpha) {
+  if (threadIdx.x != 0) return;
+  int b = 0;
+  for (int i = 1; i < n; ++i)
+    if (err[i] < err[b]) b = i;
+  *best_idx = b;
+  if (best_alpha) *best_alpha = alphas[b];
+}
+
+// D = W - code * fp16(scale) / s, from the packed format; one thread per word.
+__global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, int64_t in,
+                                     const uint32_t* __restrict__ qweight,
+                                     const uint16_t* __restrict__ scales16,
+                                     const int32_t* __restrict__ g_idx,
+                                     const float* __restrict__ s, int bits, int g,
+                                     uint16_t* __restrict__ dW, DeviceStatus* st) {
+  const int64_t words = in / 8;
+  const int64_t ngroups = (in + g - 1) / g;
+  const int off = 1 << (bits - 1);
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       idx < out * words; idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / words, wd = idx - r * words;
+    const uint32_t word = qweight[idx];
+    uint16_t d16[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t c = wd * 8 + k;
+      const int code = static_cast<int>((word >> (4 * k)) & 0xFu) - off;
+      int64_t grp = g_idx ? g_idx[c] : c / g;
+      if (grp < 0 || grp >= ngroups) {  // caller's group index out of range
+        set_status(st, PIQ_ERR_INVALID_ARG, static_cast<int>(c));
+        grp = 0;
+      }
+      const float sc = __half2float(__ushort_as_half(scales16[r * ngroups + grp]));
+      float what = static_cast<float>(code) * sc;
+      if (s) what = __fdiv_rn(what, s[c]);
+      d16[k] = float_to_bf16_bits(W[r * in + c] - what);
+    }
+    uint4 o;
+    o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
+    o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
+    o.z = d16[4] | (static_cast<uint32_t>(d16[5]) << 16);
+    o.w = d16[6] | (static_cast<uint32_t>(d16[7]) << 16);
+    *reinterpret_cast<uint4*>(dW + r * in + wd * 8) = o;
+  }
+}
+
+unsigned grid_for(int64_t work, int threads) {
+  DeviceInfo info;
+  int sms = (device_info(&info) == PIQ_OK) ? info.sm_count : 148;
+  const int64_t want = ceil_div(work, threads);
+  return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, 16LL * sms)));
+}
+
+int last_error() { return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA; }
+
+}  // namespace
+
+// Row splits of the column-statistics pass: about 1024 CTAs in all, at least 64
+// rows each.  Device-independent, so workspace queries can use it.
+int colstats_splits(int64_t n, int64_t in) {
+  const int64_t col_blocks = ceil_div(in, 256);
+  int64_t splits = std::min<int64_t>(ceil_div(1024, col_blocks), ceil_div(n, 64));
+  return static_cast<int>(std::max<int64_t>(1, splits));
+}
+
+int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, int splits,
+                    double* mean_abs, double* sumsq, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(ceil_div(in, 256)), static_cast<unsigned>(splits));
+  note_launch();
+  colstats_kernel<<<grid, 256, 0, stream>>>(X, n, in, splits, partials);
+  note_launch();
+  colstats_finish_kernel<<<static_cast<unsigned>(ceil_div(in, 256)), 256, 0, stream>>>(
+      partials, n, in, splits, mean_abs, sumsq);
+  return last_error();
+}
+
+int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
+                          float* Wq, cudaStream_t stream) {
+  note_launch();
+  gather_columns_kernel<<<grid_for(out * in, 256), 256, 0, stream>>>(W, out, in, perm, Wq);
+  return last_error();
+}
+
+int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
+                int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
+                uint16_t* scales16, uint16_t* dW, int32_t* g_idx, cudaStream_t stream) {
+  note_launch();
+  pack_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
+      codes, qscale, invperm, out, in, bits, g, W0, qweight, scales16, dW, g_idx);
+  return last_error();
+}
+
+int launch_awq_scale_table(const double* mean_abs, int64_t in, const float* alphas_dev,
+                           int n_alpha, float* s_table, cudaStream_t stream) {
+  note_launch();
+  awq_scale_table_kernel<<<grid_for(n_alpha * in, 256), 256, 0, stream>>>(mean_abs, in,
+                                                                          alphas_dev, n_alpha,
+                                                                          s_table);
+  return last_error();
+}
+
+int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,
+                     const float* s_table, int n_alpha, uint16_t* dW, cudaStream_t stream) {
+  const int64_t warps = out * ceil_div(in, g);
+  note_launch();
+  awq_delta_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g, s_table,
+                                                                   n_alpha, dW);
+  return last_error();
+}
+
+int launch_group_quant(const float* W, int64_t out, int64_t in, int bits, int g,
+                       const float* s_table, const int* sel, int8_t* codes, float* qscale,
+                       float* s_out, cudaStream_t stream) {
+  const int64_t warps = out * ceil_div(in, g);
+  note_launch();
+  group_quant_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g, s_table,
+                                                                     sel, codes, qscale, s_out);
+  return last_error();
+}
+
+int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_idx,
+                  float* best_alpha, cudaStream_t stream) {
+  note_launch();
+  argmin_kernel<<<1, 32, 0, stream>>>(err, n, alphas_dev, best_idx, best_alpha);
+  return last_error();
+}
+
+int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
+                         const uint16_t* scales16, const int32_t* g_idx, const float* s,
+                         int bits, int g, uint16_t* dW, DeviceStatus* st,
+                         cudaStream_t stream) {
+  note_launch();
+  dequant_delta_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
+      W, out, in, qweight, scales16, g_idx, s, bits, g, dW, st);
+  return last_error();
+}
+
+}  // namespace piq

@@ -1,0 +1,420 @@
+// Tensor-core GEMMs on sm_100a: tcgen05.mma (kind::f16, bf16 x bf16 -> fp32 in
+// TMEM), operands staged in shared memory by TMA (128-byte swizzle), one
+// persistent CTA per SM.
+//
+//   * syrk_xtx   H = X^T X, the proxy Hessian of "GPTQ versus AWQ objectives"
+//                ("A strong answer", listing: H = X.T @ X).  X[n, in] is
+//                row-major, so both operands are MN-major tiles (the sample
+//                index n is the contraction).  Only tiles touching the upper
+//                triangle are computed.
+//   * err_sumsq  E_b = ||X D_b^T||_F^2 for stacked D_b (D = W - What), the
+//                shared objective of both methods ("How to approach it").  Both
+//                operands are K-major; the epilogue squares and sums the
+//                accumulator straight out of TMEM, so the [n, out] product
+//                never reaches memory.  One double per tile, reduced later in a
+//                fixed order (deterministic).
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads into a 4-stage
+// ring; warp 1 lane 0 issues the MMAs and commits; warps 2..5 drain one of two
+// 256-column accumulators while the MMA warp fills the other.  Every wait is
+// bounded (common.cuh); no multicast loads are used.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace piq {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int GROUP_M = 16;                     // raster group (err_sumsq)
+
+enum { EPI_STORE_UPPER = 0, EPI_SUMSQ = 1 };
+
+struct Params {
+  int M, N, K;
+  int m_tiles, n_tiles, batch;
+  int num_tiles;
+  float* C;
+  int64_t ldc;
+  int accumulate;
+  double* partials;
+  DeviceStatus* st;
+};
+
+// Tile t -> (m tile, n tile, batch entry).
+template <int EPI>
+__device__ __forceinline__ void decode_tile(const Params& p, int t, int& mt, int& nt, int& bz) {
+  if (EPI == EPI_STORE_UPPER) {
+    // n-panel b holds m tiles a with a*BM < (b+1)*BN (they touch j >= i).
+    int acc = 0;
+    bz = 0;
+    for (int b = 0; b < p.n_tiles; ++b) {
+      int cnt = min(p.m_tiles, (int)(((int64_t)(b + 1) * BN + BM - 1) / BM));
+      if (t < acc + cnt) {
+        nt = b;
+        mt = t - acc;
+        return;
+      }
+      acc += cnt;
+    }
+    mt = nt = 0;
+  } else {
+    const int per = p.m_tiles * p.n_tiles;
+    bz = t / per;
+    const int r = t - bz * per;
+    const int grp = r / (GROUP_M * p.n_tiles);
+    const int first_m = grp * GROUP_M;
+    const int gm = min(GROUP_M, p.m_tiles - first_m);
+    const int w = r - grp * GROUP_M * p.n_tiles;
+    mt = first_m + w % gm;
+    nt = w / gm;
+  }
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mt, nt, bz;
+        decode_tile<EPI>(p, t, mt, nt, bz);
+        const int m0 = mt * BM, n0 = nt * BN;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, p.st, 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (A_MN) {
+            tma_load_2d(sa, &tmA, &full[s], m0, k0);
+            tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, k0);
+          } else {
+            tma_load_2d(sa, &tmA, &full[s], k0, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tma_load_2d(sb + c * 8192, &tmB, &full[s], n0 + 64 * c, k0);
+          } else {
+            tma_load_3d(sb, &tmB, &full[s], k0, n0, bz);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        const uint32_t use = static_cast<uint32_t>(lt >> 1);
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, p.st, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kLayoutSw128)
+                                     : smem_desc(a_addr + kk * 32, 16, 1024, kLayoutSw128);
+            const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 8192, 1024, kLayoutSw128)
+                                     : smem_desc(b_addr + kk * 32, 16, 1024, kLayoutSw128);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);  // frees the stage once these MMAs finish
+        }
+        if (ok) umma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int lt = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      const uint32_t use = static_cast<uint32_t>(lt >> 1);
+      int mt, nt, bz;
+      decode_tile<EPI>(p, t, mt, nt, bz);
+      if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) break;
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      const int row = mt * BM + q * 32 + lane;
+      double acc = 0.0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        if (EPI == EPI_SUMSQ) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s = fmaf(v[i], v[i], s);
+          acc += static_cast<double>(s);
+        } else {
+          const int col0 = nt * BN + c * 32;
+          // chunks entirely below the diagonal are not needed
+          if (row < p.M && col0 < p.N && col0 + 32 > row) {
+            float* dst = p.C + static_cast<int64_t>(row) * p.ldc + col0;
+            if (col0 + 32 <= p.N) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                float4 o = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                if (p.accumulate) {
+                  const float4 old = *reinterpret_cast<const float4*>(dst + i);
+                  o.x += old.x;
+                  o.y += old.y;
+                  o.z += old.z;
+                  o.w += old.w;
+                }
+                *reinterpret_cast<float4*>(dst + i) = o;
+              }
+            } else {
+              const int lim = p.N - col0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (i < lim) dst[i] = p.accumulate ? dst[i] + v[i] : v[i];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (EPI == EPI_SUMSQ) {
+        // one partial per (tile, lane quarter): no cross-warp synchronisation
+        acc = warp_sum_d(acc);
+        if (lane == 0) p.partials[static_cast<int64_t>(t) * 4 + q] = acc;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// -------------------------------------------------------------- host helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, innermost dimension first.
+int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+             const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return PIQ_ERR_CUDA;
+  cuuint64_t d[3], s[2];
+  cuuint32_t b[3], e[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b,
+                  e, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PIQ_OK : PIQ_ERR_INVALID_ARG;
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+int launch(const CUtensorMap& a, const CUtensorMap& b, const Params& p, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
+  auto kern = tc_gemm_kernel<A_MN, B_MN, EPI>;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return PIQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  DeviceInfo info;
+  int rc = device_info(&info);
+  if (rc != PIQ_OK) return rc;
+  const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
+  note_launch();
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(a, b, p);
+  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
+                    DeviceStatus* st, cudaStream_t stream) {
+  if (n < 1 || in < 8 || in % 8 != 0 || n > INT32_MAX || in > INT32_MAX / 2)
+    return PIQ_ERR_INVALID_ARG;
+  CUtensorMap map;
+  const uint64_t dims[2] = {static_cast<uint64_t>(in), static_cast<uint64_t>(n)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(in) * 2};
+  const uint32_t box[2] = {64, 64};
+  int rc = make_map(&map, X, 2, dims, strides, box);
+  if (rc != PIQ_OK) return rc;
+  Params p{};
+  p.M = p.N = static_cast<int>(in);
+  p.K = static_cast<int>(n);
+  p.m_tiles = static_cast<int>(ceil_div(in, BM));
+  p.n_tiles = static_cast<int>(ceil_div(in, BN));
+  p.batch = 1;
+  int total = 0;
+  for (int b = 0; b < p.n_tiles; ++b)
+    total += std::min(p.m_tiles, static_cast<int>(((int64_t)(b + 1) * BN + BM - 1) / BM));
+  p.num_tiles = total;
+  p.C = H;
+  p.ldc = in;
+  p.accumulate = accumulate;
+  p.st = st;
+  return launch<true, true, EPI_STORE_UPPER>(map, map, p, stream);
+}
+
+int64_t sumsq_partials_count(int64_t n, int64_t rows, int batch) {
+  return ceil_div(n, BM) * ceil_div(rows, BN) * batch * 4;
+}
+
+int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D, int64_t rows,
+                     int batch, double* partials, DeviceStatus* st, cudaStream_t stream) {
+  if (n < 1 || in < 8 || in % 8 != 0 || rows < 1 || batch < 1 || n > INT32_MAX ||
+      rows > INT32_MAX)
+    return PIQ_ERR_INVALID_ARG;
+  CUtensorMap ma, mb;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(in), static_cast<uint64_t>(n)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(in) * 2};
+    const uint32_t box[2] = {64, BM};
+    int rc = make_map(&ma, X, 2, dims, strides, box);
+    if (rc != PIQ_OK) return rc;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(in), static_cast<uint64_t>(rows),
+                              static_cast<uint64_t>(batch)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(in) * 2,
+                                 static_cast<uint64_t>(in) * static_cast<uint64_t>(rows) * 2};
+    const uint32_t box[3] = {64, BN, 1};
+    int rc = make_map(&mb, D, 3, dims, strides, box);
+    if (rc != PIQ_OK) return rc;
+  }
+  Params p{};
+  p.M = static_cast<int>(n);
+  p.N = static_cast<int>(rows);
+  p.K = static_cast<int>(in);
+  p.m_tiles = static_cast<int>(ceil_div(n, BM));
+  p.n_tiles = static_cast<int>(ceil_div(rows, BN));
+  p.batch = batch;
+  const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * batch;
+  if (total > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+  p.num_tiles = static_cast<int>(total);
+  p.partials = partials;
+  p.st = st;
+  return launch<false, false, EPI_SUMSQ>(ma, mb, p, stream);
+}
+
+// ------------------------------------------------ fixed-order partial reduction
+namespace {
+__global__ void reduce_partials_kernel(const double* partials, int64_t per, double* out) {
+  __shared__ double sh[256];
+  const double* src = partials + static_cast<int64_t>(blockIdx.x) * per;
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < per; i += blockDim.x) acc += src[i];
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[blockIdx.x] = sh[0];
+}
+}  // namespace
+
+int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,
+                           double* out, cudaStream_t stream) {
+  const int64_t per = ceil_div(n, BM) * ceil_div(rows, BN) * 4;
+  note_launch();
+  reduce_partials_kernel<<<batch, 256, 0, stream>>>(partials, per, out);
+  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+}  // namespace piq

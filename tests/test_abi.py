@@ -1,0 +1,77 @@
+"""The C-ABI library builds, loads and exports what include/piq.h declares.
+No GPU: only calls that return before touching a device are made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_int4_weight_gptq_b200 as piq
+from post_int4_weight_gptq_b200 import build as piq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    piq_build.build()
+    return piq.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "piq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", text, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "gptq_quantize_layer" in names and "awq_search_layer" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    # and the binding covers exactly the declared functions, in order
+    assert list(piq.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for code in range(-6, 1):
+        assert piq.status_string(code) != "unknown status"
+    assert piq.status_string(-99) == "unknown status"
+
+
+def test_hessian_bytes_printed_on_the_page(lib):
+    # "GPTQ versus AWQ objectives", sizing block: 8,192^2 x 4 B = 268 MB and
+    # 28,672^2 x 4 B = 3.29 GB.
+    assert piq.hessian_bytes(8192) == 268_435_456
+    assert piq.hessian_bytes(28672) == 3_288_334_336
+
+
+def test_workspace_queries_are_monotone(lib):
+    a = piq.gptq_workspace_bytes(256, 512, 2048)
+    b = piq.gptq_workspace_bytes(512, 512, 2048)
+    c = piq.gptq_workspace_bytes(256, 1024, 2048)
+    assert 0 < a < b and a < c
+    hb = piq.hessian_bytes(512)
+    assert a >= 2 * hb  # H (then U) and the factor's working copy
+    assert piq.gptq_workspace_bytes(256, 512, 2048, act_order=True) >= a
+    assert piq.awq_workspace_bytes(256, 512, 2048, 20) > piq.awq_workspace_bytes(256, 512, 2048, 1)
+
+
+def test_bad_arguments_rejected_before_any_device_work(lib):
+    null = None
+    err = ctypes.c_double()
+    # bits out of range, in not a multiple of 8, g < 1, null pointers
+    for bits, inp, g in ((5, 512, 128), (4, 500, 128), (4, 512, 0), (1, 512, 128)):
+        rc = lib.gptq_quantize_layer(null, 16, inp, null, 64, bits, g, 0.01, 0, null, null, null,
+                                     null, ctypes.byref(err), null, 0, null)
+        assert rc == piq.PIQ_ERR_INVALID_ARG
+    rc = lib.piq_hessian(null, 10, 64, null, 0, null)
+    assert rc == piq.PIQ_ERR_INVALID_ARG
+    out = ctypes.c_size_t()
+    assert lib.piq_awq_workspace_bytes(16, 64, 64, 65, ctypes.byref(out)) == piq.PIQ_ERR_INVALID_ARG
+    assert lib.piq_awq_workspace_bytes(16, 64, 64, 0, ctypes.byref(out)) == piq.PIQ_ERR_INVALID_ARG
+
+
+def test_library_is_sm100a_only(lib):
+    # every kernel was compiled for sm_100a alone
+    assert "-gencode" in piq_build.ARCH and "arch=compute_100a,code=sm_100a" in piq_build.ARCH

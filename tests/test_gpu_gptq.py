@@ -1,0 +1,112 @@
+"""End-to-end GPTQ parity (gptq_quantize_layer) against the FP64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_int4_weight_gptq_b200 as piq
+from oracle.pack import dequant_ref
+from tests.parity import REL_TOL, rel, teacher_forced_compare, to_gpu_w, to_gpu_x, unpack_gpu
+from workloads import C1, make_weight, make_x_bits, small_spec
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_layer(W, X, bits, g, act_order, damp=0.01):
+    out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X), bits=bits, g=g, damp=damp,
+                                  act_order=act_order)
+    perm_gpu = out.perm.cpu().numpy()
+    Hx = O.hessian_ref(X)
+    perm, U, lam = O.gptq_prepare_ref(Hx, damp, act_order)
+    assert np.array_equal(perm_gpu, perm)
+    assert np.array_equal(out.g_idx.cpu().numpy(), O.g_idx_ref(perm, g))
+    codes_mem = unpack_gpu(out.qweight, bits)
+    codes_q = codes_mem[:, perm]
+    Wp = W.astype(np.float64)[:, perm]
+    stats, c_ref, s_ref = teacher_forced_compare(codes_q, Wp, U, bits, g)
+    sc = out.scales.cpu().numpy().astype(np.float64)
+    s16 = s_ref.astype(np.float16).astype(np.float64)
+    assert (np.abs(sc - s16) / np.maximum(s16, 1e-30)).max() < REL_TOL
+    e_ref = O.output_error_ref(W, dequant_ref(c_ref, s_ref, perm, g), X)
+    assert rel(out.err, e_ref) < REL_TOL, (out.err, e_ref)
+    return stats, out, e_ref
+
+
+def test_tiny_layer_config():
+    # W 256x512 ~N(0, 0.02^2); X 2048x512 with 5 channels x20; 4-bit, g128
+    W, X = make_weight(C1), make_x_bits(C1)
+    stats, out, e = _check_layer(W, X, 4, 128, False)
+    c, s = O.rtn_ref(W)
+    e_rtn = O.output_error_ref(W, dequant_ref(c, s, np.arange(512), 128), X)
+    assert out.err < e_rtn
+
+
+@pytest.mark.parametrize("out,inp,n,g,bits,act", [
+    (129, 520, 1500, 128, 4, False),    # ragged rows, ragged last block
+    (64, 600, 1800, 200, 3, False),     # group wider than a block, not a multiple
+    (100, 264, 900, 40, 4, True),       # act-order, small groups
+    (33, 1032, 3000, 128, 3, True),     # act-order, INT3
+    (48, 136, 500, 1000, 4, False),     # one group per row
+    (8, 8, 64, 8, 2, False),            # smallest layer, 2-bit
+])
+def test_layer_variants(out, inp, n, g, bits, act):
+    spec = small_spec(out, inp, n, seed=out + inp + n, sigma_ln=0.8)
+    _check_layer(make_weight(spec), make_x_bits(spec), bits, g, act)
+
+
+def test_diagonal_hessian_equals_rtn():
+    # one-hot rows: X^T X exactly diagonal, so GPTQ reduces to group RTN
+    rng = np.random.default_rng(7)
+    inp, n = 256, 2048
+    Xf = np.zeros((n, inp), dtype=np.float32)
+    Xf[np.arange(n), rng.integers(0, inp, n)] = 1.0
+    from workloads import bf16_bits_from_f32
+    X = bf16_bits_from_f32(Xf)
+    W = make_weight(C1)[:64, :inp].copy()
+    out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X), bits=4, g=64)
+    qw, sc = piq.rtn_quantize_layer(to_gpu_w(W), 4, 64)
+    assert torch.equal(out.qweight, qw) and torch.equal(out.scales, sc)
+
+
+def test_deterministic():
+    W, X = make_weight(C1), make_x_bits(C1)
+    a = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X))
+    b = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X))
+    assert torch.equal(a.qweight, b.qweight) and torch.equal(a.scales, b.scales)
+    assert a.err == b.err
+
+
+def test_zero_inputs_not_positive_definite():
+    W = make_weight(C1)
+    X = np.zeros((256, 512), dtype=np.uint16)
+    with pytest.raises(piq.PiqError) as e:
+        piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X))
+    assert e.value.status == piq.PIQ_ERR_NOT_PD
+
+
+def test_workspace_too_small():
+    W, X = make_weight(C1), make_x_bits(C1)
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    import ctypes
+    lib = piq.load_library()
+    Wg, Xg = to_gpu_w(W), to_gpu_x(X)
+    qw = torch.empty(256, 64, dtype=torch.int32, device="cuda")
+    sc = torch.empty(256, 4, dtype=torch.float16, device="cuda")
+    rc = lib.gptq_quantize_layer(ctypes.c_void_p(Wg.data_ptr()), 256, 512,
+                                 ctypes.c_void_p(Xg.data_ptr()), 2048, 4, 128, 0.01, 0,
+                                 ctypes.c_void_p(qw.data_ptr()), ctypes.c_void_p(sc.data_ptr()),
+                                 None, None, None, ctypes.c_void_p(ws.data_ptr()), 1024, None)
+    assert rc == piq.PIQ_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_shifted_inputs_error_entry():
+    # the held-out / shifted score goes through piq_layer_output_error
+    spec = small_spec(64, 256, 1024, seed=5, sigma_ln=1.0, n_outlier=3, outlier_gain=30.0)
+    W, X = make_weight(spec), make_x_bits(spec)
+    X2 = make_x_bits(spec, seed=1, permute_seed=1)
+    out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X), g=128)
+    e2 = piq.layer_output_error(to_gpu_w(W), out.qweight, out.scales, to_gpu_x(X2), 4, 128,
+                                g_idx=out.g_idx)
+    codes = unpack_gpu(out.qweight, 4)
+    What = codes * np.repeat(out.scales.cpu().numpy().astype(np.float64), 128, axis=1)
+    assert rel(e2, O.output_error_ref(W, What, X2)) < REL_TOL
