@@ -79,7 +79,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait until the phase of `bar` with the given parity has completed.  Bounded:
 // after kWaitLimitNs it records PIQ_ERR_TIMEOUT (detail = `where`) and returns
-// false; callers then stop issuing work.
+// false; callers then stop issuing work.  A status set by an earlier kernel is
+// checked once at kernel entry, not here, so no wait gives up while copies it
+// issued are still in flight.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DeviceStatus* st,
                                           int where) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -91,7 +93,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Device
         set_status(st, PIQ_ERR_TIMEOUT, where);
         return false;
       }
-      if (status_bad(st)) return false;
     }
   }
 }
@@ -206,6 +207,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)       // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ------------------------------------------------------ asynchronous copies
+// global -> shared without staging in registers (the thread does not wait).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // -------------------------------------------------------------- misc helpers

@@ -5,16 +5,18 @@
 // Section "What interviewers probe next": the damping keeps the factorization
 // stable; act-order takes columns by decreasing diag(H).
 //
-// Route (exact identity, no explicit inverse of H): with J the index reversal,
+// Route (exact identity, no inverse of H): with J the index reversal,
 // P = J H_d J = L L^T (lower Cholesky), then inv(H_d) = (J inv(L) J)^T (J inv(L) J)
 // and J inv(L) J is upper triangular with a positive diagonal, so it is U.
-//   1. lambda = damp * mean(diag H)                 (diag_mean_kernel)
+//   1. lambda = damp * mean(diag H)                        (diag_mean_kernel)
 //   2. P[a][b] = H[s(a)][s(b)] + lambda [a == b], s(a) = perm[in-1-a]
-//   3. blocked right-looking Cholesky of P, panel width 128; each diagonal
-//      block is factored and inverted in shared memory (potrf_inv_kernel), the
-//      panel below is L21 = A21 inv(L11)^T and the trailing matrix is updated by
-//      A22 -= L21 L21^T (FP32 SIMT GEMMs)
-//   4. blocked inverse, right to left: X21 = -(X22 L21) inv(L11)
+//   3. right-looking blocked Cholesky, 128-wide panels: each diagonal block is
+//      factored and inverted in shared memory (chol_inv_kernel), the panel
+//      below is L21 = A21 inv(L11)^T and the trailing matrix A22 -= L21 L21^T
+//      (FP32 SIMT GEMMs that skip the zero triangles)
+//   4. X = inv(L) from the diagonal inverses, merging pairs of s-blocks level by
+//      level (s = 128, 256, ...): X21 = -X22 (L21 X11), every pair of a level in
+//      one batched launch
 //   5. U[i][k] = X[in-1-i][in-1-k]
 // A non-positive pivot sets PIQ_ERR_NOT_PD.
 #include <algorithm>
@@ -25,8 +27,8 @@ namespace piq {
 
 namespace {
 
-constexpr int NB = kFactorNB;      // 128
-constexpr int LDS = NB + 1;        // padded shared-memory row
+constexpr int NB = kFactorNB;  // 128
+constexpr int LDS = NB + 1;    // padded shared-memory row
 
 __global__ void diag_mean_kernel(const float* H, int64_t in, float damp, DeviceStatus* st,
                                  float* lambda_f) {
@@ -66,113 +68,179 @@ __global__ void build_rev_kernel(const float* H, int64_t in, const int32_t* perm
   }
 }
 
-// Factor the nb x nb diagonal block at (k0, k0) of P in place (lower Cholesky)
-// and write its inverse, zero-padded to nbp x nbp (nbp = 32, 64 or 128), to
-// Dinv.  Rows/cols >= nb are treated as identity.
-__global__ void __launch_bounds__(256) potrf_inv_kernel(float* P, int64_t ld, int64_t k0, int nb,
-                                                        int nbp, float* Dinv, DeviceStatus* st) {
-  extern __shared__ float sm[];
-  float* S = sm;                 // [NB][LDS] factor
-  float* X = sm + NB * LDS;      // [NB][LDS] inverse
-  float* T = X + NB * LDS;       // [64][65] temp
-  const int tid = threadIdx.x;
-  if (status_bad(st)) return;
+constexpr int SP = 16;  // sub-panel width inside a 128 block
+constexpr unsigned FULL = 0xffffffffu;
 
-  for (int idx = tid; idx < nbp * nbp; idx += 256) {
-    const int i = idx / nbp, j = idx % nbp;
-    float v = 0.f;
-    if (i < nb && j < nb) {
-      if (j <= i) v = P[(k0 + i) * ld + (k0 + j)];
-    } else if (i == j) {
-      v = 1.f;
+// One warp factors a 16 x 16 SPD block and inverts its factor, in registers.
+// Lane i < 16 holds row i: on entry a[k] = A[i][k] (k <= i); on exit a[k] =
+// L[i][k] and x[k] = inv(L)[i][k] (0 above the diagonal).  Lanes >= 16 carry
+// zeros.  Template recursion keeps register indices compile-time; the code is
+// small enough for the instruction cache.
+template <int J>
+__device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lane, bool& ok) {
+  if constexpr (J < SP) {
+    const float d = __shfl_sync(FULL, a[J], J);
+    ok = ok && (d > 0.f);
+    const float ljj = sqrtf(d > 0.f ? d : 1.f);
+    const float r = 1.f / ljj;
+    if (lane == J) rdiag = r;
+    const float lij = (lane > J) ? a[J] * r : (lane == J ? ljj : 0.f);
+    a[J] = lij;
+#pragma unroll
+    for (int k = J + 1; k < SP; ++k) {
+      const float lkj = __shfl_sync(FULL, lij, k);
+      if (k <= lane) a[k] = fmaf(-lij, lkj, a[k]);
     }
-    S[i * LDS + j] = v;
-    X[i * LDS + j] = 0.f;
-  }
-  __syncthreads();
-
-  // unblocked right-looking Cholesky
-  __shared__ int bad;
-  if (tid == 0) bad = 0;
-  for (int j = 0; j < nbp; ++j) {
-    if (tid == 0) {
-      const float d = S[j * LDS + j];
-      if (!(d > 0.f)) {
-        bad = 1;
-        set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(k0 + j));
-        S[j * LDS + j] = 1.f;
-      } else {
-        S[j * LDS + j] = sqrtf(d);
-      }
-    }
-    __syncthreads();
-    const float ljj = S[j * LDS + j];
-    for (int i = j + 1 + tid; i < nbp; i += 256) S[i * LDS + j] = S[i * LDS + j] / ljj;
-    __syncthreads();
-    {  // trailing update of the lower triangle: one warp per row
-      const int w = tid >> 5, ln = tid & 31;
-      for (int i = j + 1 + w; i < nbp; i += 8) {
-        const float lij = S[i * LDS + j];
-        for (int k = j + 1 + ln; k <= i; k += 32)
-          S[i * LDS + k] = fmaf(-lij, S[k * LDS + j], S[i * LDS + k]);
-      }
-    }
-    __syncthreads();
-  }
-  if (bad) return;
-
-  // inverse: 32 x 32 diagonal blocks by one warp each (lane = column) ...
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int blk = warp; blk < nbp / 32; blk += 8) {
-    const int o = blk * 32;
-    const int c = o + lane;
-    X[c * LDS + c] = 1.f / S[c * LDS + c];
-    for (int i = c + 1; i < o + 32; ++i) {
-      float s = 0.f;
-      for (int k = c; k < i; ++k) s = fmaf(S[i * LDS + k], X[k * LDS + c], s);
-      X[i * LDS + c] = -s / S[i * LDS + i];
-    }
-  }
-  __syncthreads();
-  // ... then merged pairwise: inv([[A,0],[B,C]]) has lower block -inv(C) B inv(A)
-  for (int s = 32; s < nbp; s *= 2) {
-    for (int pair = 0; pair < nbp / (2 * s); ++pair) {
-      const int r0 = pair * 2 * s, r1 = r0 + s;
-      for (int idx = tid; idx < s * s; idx += 256) {  // T = B inv(A)
-        const int i = idx / s, j = idx % s;
-        float acc = 0.f;
-        for (int k = j; k < s; ++k) acc = fmaf(S[(r1 + i) * LDS + r0 + k], X[(r0 + k) * LDS + r0 + j], acc);
-        T[i * 65 + j] = acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < s * s; idx += 256) {  // X21 = -inv(C) T
-        const int i = idx / s, j = idx % s;
-        float acc = 0.f;
-        for (int k = 0; k <= i; ++k) acc = fmaf(X[(r1 + i) * LDS + r1 + k], T[k * 65 + j], acc);
-        X[(r1 + i) * LDS + r0 + j] = -acc;
-      }
-      __syncthreads();
-    }
-  }
-
-  for (int idx = tid; idx < nbp * nbp; idx += 256) {
-    const int i = idx / nbp, j = idx % nbp;
-    if (i < nb && j <= i) P[(k0 + i) * ld + (k0 + j)] = S[i * LDS + j];
-    Dinv[idx] = (j <= i) ? X[i * LDS + j] : 0.f;
+    chol16_col<J + 1>(a, rdiag, lane, ok);
   }
 }
 
-// Copy every diagonal block's inverse into P (full nb x nb, zero above the
-// diagonal) before the blocked inverse reads P as a lower-triangular X.
-__global__ void put_diag_inv_kernel(float* P, int64_t in, const float* Dinv, int npanel) {
-  const int pnl = blockIdx.x;
-  const int64_t c0 = static_cast<int64_t>(pnl) * NB;
-  const int nb = static_cast<int>(std::min<int64_t>(NB, in - c0));
-  const int nbp = nb <= 32 ? 32 : (nb <= 64 ? 64 : 128);
-  const float* D = Dinv + static_cast<int64_t>(pnl) * NB * NB;
-  for (int idx = threadIdx.x; idx < nb * nb; idx += blockDim.x) {
-    const int i = idx / nb, j = idx % nb;
-    P[(c0 + i) * in + c0 + j] = D[i * nbp + j];
+// forward substitution by rows: X_K = (e_K - sum_{c<K} L_Kc X_c) / L_KK
+template <int K>
+__device__ __forceinline__ void inv16_row(const float (&a)[SP], float (&x)[SP], float rdiag,
+                                          int lane) {
+  if constexpr (K < SP) {
+    if (lane == K) {
+#pragma unroll
+      for (int c = 0; c <= K; ++c) x[c] *= rdiag;
+    }
+#pragma unroll
+    for (int c = 0; c <= K; ++c) {
+      const float xkc = __shfl_sync(FULL, x[c], K);
+      if (lane > K) x[c] = fmaf(-a[K], xkc, x[c]);
+    }
+    inv16_row<K + 1>(a, x, rdiag, lane);
+  }
+}
+
+// z[c] = sum_{k <= c} y[k] * Xd[c][k]   (row times the transposed lower inverse)
+template <int C>
+__device__ __forceinline__ void trsm_col(const float (&y)[SP], float (&z)[SP], const float* Xd) {
+  if constexpr (C < SP) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k <= C; ++k) acc = fmaf(y[k], Xd[C * LDS + k], acc);
+    z[C] = acc;
+    trsm_col<C + 1>(y, z, Xd);
+  }
+}
+
+// Factor the nb x nb diagonal block of P at (o, o) in place (lower Cholesky) and
+// write its inverse to X at (o, o) (full nb x nb, zeros above the diagonal).
+// Rows/cols >= nb are padded with the identity up to nbp = 32, 64 or 128.
+constexpr int CI_THREADS = 512;
+constexpr int CI_WARPS = CI_THREADS / 32;
+
+__global__ void __launch_bounds__(CI_THREADS)
+    chol_inv_kernel(float* P, float* X, int64_t ld, int64_t o, int nb, int nbp,
+                    DeviceStatus* st) {
+  extern __shared__ float sm[];
+  float* S = sm;              // [NB][LDS] factor
+  float* Xs = sm + NB * LDS;  // [NB][LDS] inverse
+  float* T = Xs + NB * LDS;   // [64][65] temp
+  __shared__ int bad;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (status_bad(st)) return;
+  if (tid == 0) bad = 0;
+
+  for (int i = warp; i < nbp; i += CI_WARPS) {
+    for (int j = lane; j < nbp; j += 32) {
+      if (i < nb && j <= i)
+        cp_async4(S + i * LDS + j, P + (o + i) * ld + (o + j));
+      else
+        S[i * LDS + j] = (i == j) ? 1.f : 0.f;
+      Xs[i * LDS + j] = 0.f;
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // right-looking over 16-wide sub-panels
+  for (int c0 = 0; c0 < nbp; c0 += SP) {
+    if (warp == 0) {
+      float a[SP], x[SP];
+      float rdiag = 0.f;
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < SP; ++k) a[k] = (lane < SP) ? S[(c0 + lane) * LDS + c0 + k] : 0.f;
+      chol16_col<0>(a, rdiag, lane, ok);
+#pragma unroll
+      for (int k = 0; k < SP; ++k) {
+        a[k] = (k <= lane) ? a[k] : 0.f;
+        x[k] = (k == lane) ? 1.f : 0.f;
+      }
+      inv16_row<0>(a, x, rdiag, lane);
+      if (!ok && lane == 0) {
+        bad = 1;
+        set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));
+      }
+      if (lane < SP) {
+#pragma unroll
+        for (int k = 0; k < SP; ++k) {
+          S[(c0 + lane) * LDS + c0 + k] = a[k];
+          Xs[(c0 + lane) * LDS + c0 + k] = x[k];
+        }
+      }
+    }
+    __syncthreads();
+    if (bad) return;
+    const int r0 = c0 + SP;
+    if (r0 < nbp) {
+      // L21 = A21 inv(L11)^T, one thread per row
+      const int r = r0 + tid;
+      if (r < nbp) {
+        float y[SP], z[SP];
+#pragma unroll
+        for (int k = 0; k < SP; ++k) y[k] = S[r * LDS + c0 + k];
+        trsm_col<0>(y, z, Xs + c0 * LDS + c0);
+#pragma unroll
+        for (int cc = 0; cc < SP; ++cc) S[r * LDS + c0 + cc] = z[cc];
+      }
+      __syncthreads();
+      // A22 -= L21 L21^T (lower triangle), one warp per row
+      for (int i = r0 + warp; i < nbp; i += CI_WARPS) {
+        for (int j = r0 + lane; j <= i; j += 32) {
+          float acc = S[i * LDS + j];
+#pragma unroll
+          for (int k = 0; k < SP; ++k)
+            acc = fmaf(-S[i * LDS + c0 + k], S[j * LDS + c0 + k], acc);
+          S[i * LDS + j] = acc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // inverse of the whole block from the diagonal 16-blocks:
+  // inv([[A,0],[B,C]]) has lower-left block -inv(C) B inv(A)
+  for (int s = SP; s < nbp; s *= 2) {
+    for (int pr = 0; pr < nbp / (2 * s); ++pr) {
+      const int q0 = pr * 2 * s, q1 = q0 + s;
+      for (int i = warp; i < s; i += CI_WARPS) {  // T = B inv(A)
+        for (int j = lane; j < s; j += 32) {
+          float acc = 0.f;
+          for (int k = j; k < s; ++k)
+            acc = fmaf(S[(q1 + i) * LDS + q0 + k], Xs[(q0 + k) * LDS + q0 + j], acc);
+          T[i * 65 + j] = acc;
+        }
+      }
+      __syncthreads();
+      for (int i = warp; i < s; i += CI_WARPS) {  // X21 = -inv(C) T
+        for (int j = lane; j < s; j += 32) {
+          float acc = 0.f;
+          for (int k = 0; k <= i; ++k) acc = fmaf(Xs[(q1 + i) * LDS + q1 + k], T[k * 65 + j], acc);
+          Xs[(q1 + i) * LDS + q0 + j] = -acc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  for (int i = warp; i < nb; i += CI_WARPS) {
+    for (int j = lane; j < nb; j += 32) {
+      if (j <= i) P[(o + i) * ld + (o + j)] = S[i * LDS + j];
+      X[(o + i) * ld + (o + j)] = (j <= i) ? Xs[i * LDS + j] : 0.f;
+    }
   }
 }
 
@@ -222,30 +290,40 @@ __global__ void identity_perm_kernel(int64_t in, int32_t* perm, int32_t* invperm
   }
 }
 
-constexpr int kPotrfSmem = (2 * NB * LDS + 64 * 65) * sizeof(float);
+constexpr int kCholSmem = (2 * NB * LDS + 64 * 65) * sizeof(float);
+
+// Floats of the pair scratch of the level-by-level inverse: max over levels of
+// (pairs at that level) * s * s.
+int64_t trtri_scratch_floats(int64_t n) {
+  int64_t best = 0;
+  for (int64_t s = NB; s < n; s *= 2) {
+    const int64_t pairs = ceil_div(n - s, 2 * s);
+    best = std::max(best, pairs * s * s);
+  }
+  return best;
+}
 
 }  // namespace
 
 int64_t factor_workspace_floats(int64_t in) {
-  const int64_t npanel = ceil_div(in, NB);
-  return in * in + npanel * NB * NB + in * NB + 64;
+  return 2 * in * in + trtri_scratch_floats(in) + 64;  // P, X, pair scratch, lambda
 }
 
 int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm, float* U,
                      float* work, DeviceStatus* st, cudaStream_t stream) {
   if (in < 1) return PIQ_ERR_INVALID_ARG;
-  const int64_t npanel = ceil_div(in, NB);
   float* P = work;
-  float* Dinv = P + in * in;
-  float* Tb = Dinv + npanel * NB * NB;
-  float* lam = Tb + in * NB;
+  float* X = P + in * in;
+  float* T = X + in * in;
+  float* lam = T + trtri_scratch_floats(in);
+  const int64_t ld = in;
 
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPotrfSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kCholSmem) != cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
   }
@@ -259,48 +337,49 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
   }
   if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
 
-  // Cholesky, panel by panel
-  for (int64_t p = 0; p < npanel; ++p) {
-    const int64_t k0 = p * NB;
+  // 3. Cholesky, panel by panel; diagonal inverses land in X
+  for (int64_t k0 = 0; k0 < in; k0 += NB) {
     const int nb = static_cast<int>(std::min<int64_t>(NB, in - k0));
     const int nbp = nb <= 32 ? 32 : (nb <= 64 ? 64 : 128);
-    float* D = Dinv + p * NB * NB;
     note_launch();
-    potrf_inv_kernel<<<1, 256, kPotrfSmem, stream>>>(P, in, k0, nb, nbp, D, st);
+    chol_inv_kernel<<<1, CI_THREADS, kCholSmem, stream>>>(P, X, ld, k0, nb, nbp, st);
     if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
-    const int64_t rem = in - k0 - nb;
+    const int rem = static_cast<int>(in - k0 - nb);
     if (rem <= 0) continue;
-    float* A21 = P + (k0 + nb) * in + k0;
-    // L21 = A21 inv(L11)^T  (in place; one CTA column since nb <= 128)
-    int rc = launch_simt_gemm(static_cast<int>(rem), nb, nb, 1.f, A21, in, D, nbp, true, 0.f,
-                              A21, in, 0, st, stream);
+    float* A21 = P + (k0 + nb) * ld + k0;
+    const float* X11 = X + k0 * ld + k0;
+    // L21 = A21 X11^T in place (nb <= 128: one CTA column)
+    int rc = launch_simt_gemm(rem, nb, nb, 1.f, A21, ld, X11, ld, true, 0.f, A21, ld, 3, st,
+                              stream);
     if (rc != PIQ_OK) return rc;
     // A22 -= L21 L21^T (lower tiles)
-    float* A22 = P + (k0 + nb) * in + (k0 + nb);
-    rc = launch_simt_gemm(static_cast<int>(rem), static_cast<int>(rem), nb, -1.f, A21, in, A21,
-                          in, true, 1.f, A22, in, 1, st, stream);
+    rc = launch_simt_gemm(rem, rem, nb, -1.f, A21, ld, A21, ld, true, 1.f,
+                          P + (k0 + nb) * ld + (k0 + nb), ld, 1, st, stream);
     if (rc != PIQ_OK) return rc;
   }
 
-  // inverse of L, right to left; P becomes X = inv(L) (lower)
-  note_launch();
-  put_diag_inv_kernel<<<static_cast<unsigned>(npanel), 256, 0, stream>>>(P, in, Dinv,
-                                                                         static_cast<int>(npanel));
-  if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
-  for (int64_t p = npanel - 2; p >= 0; --p) {
-    const int64_t c0 = p * NB;
-    const int nb = static_cast<int>(std::min<int64_t>(NB, in - c0));  // == NB here
-    const int64_t c1 = c0 + nb;
-    const int64_t rem = in - c1;
-    const int nbp = nb <= 32 ? 32 : (nb <= 64 ? 64 : 128);
-    // T = X22 L21   (X22 lower triangular, already inverted)
-    int rc = launch_simt_gemm(static_cast<int>(rem), nb, static_cast<int>(rem), 1.f,
-                              P + c1 * in + c1, in, P + c1 * in + c0, in, false, 0.f, Tb, NB, 2,
-                              st, stream);
+  // 4. X = inv(L): merge pairs of s-blocks, all pairs of a level per launch
+  for (int64_t s = NB; s < in; s *= 2) {
+    const int64_t pairs = ceil_div(in - s, 2 * s);
+    GemmBatch bt;
+    bt.count = static_cast<int>(pairs);
+    bt.m_total = in - s;
+    bt.m_step = 2 * s;
+    const int si = static_cast<int>(s);
+    // T_p = L21_p X11_p   (X11 lower, used as is)
+    bt.stride_a = 2 * s * (ld + 1);
+    bt.stride_b = 2 * s * (ld + 1);
+    bt.stride_c = s * s;
+    int rc = launch_simt_gemm(si, si, si, 1.f, P + s * ld, ld, X, ld, false, 0.f, T, s, 4, st,
+                              stream, bt);
     if (rc != PIQ_OK) return rc;
-    // X21 = -T inv(L11)
-    rc = launch_simt_gemm(static_cast<int>(rem), nb, nb, -1.f, Tb, NB, Dinv + p * NB * NB, nbp,
-                          false, 0.f, P + c1 * in + c0, in, 0, st, stream);
+    // X21_p = -X22_p T_p   (X22 lower, K = its rows)
+    bt.stride_a = 2 * s * (ld + 1);
+    bt.stride_b = s * s;
+    bt.stride_c = 2 * s * (ld + 1);
+    bt.k_follows_m = true;
+    rc = launch_simt_gemm(si, si, si, -1.f, X + s * ld + s, ld, T, s, false, 0.f, X + s * ld, ld,
+                          2, st, stream, bt);
     if (rc != PIQ_OK) return rc;
   }
 
@@ -308,7 +387,7 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in, 256), 64)),
               static_cast<unsigned>(std::min<int64_t>(in, 65535)));
     note_launch();
-    extract_u_kernel<<<grid, 256, 0, stream>>>(P, in, U);
+    extract_u_kernel<<<grid, 256, 0, stream>>>(X, in, U);
   }
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }

@@ -36,9 +36,19 @@ int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int 
 // C = alpha * A * op(B) + beta * C, row-major; op(B) = B or B^T (trans_b).
 // mode 0: plain; 1: only tiles touching the lower triangle of C (M == N);
 // 2: A lower triangular (entries right of the diagonal are skipped per row tile).
+// Batching over blockIdx.z: entry z uses A + z*stride_a (and B, C alike); with
+// m_total > 0 entry z has min(M, m_total - z*m_step) rows, and K the same when
+// k_follows_m (a square triangular A).
+struct GemmBatch {
+  int count = 1;
+  int64_t stride_a = 0, stride_b = 0, stride_c = 0;
+  int64_t m_total = 0, m_step = 0;
+  bool k_follows_m = false;
+};
 int launch_simt_gemm(int M, int N, int K, float alpha, const float* A, int64_t lda,
                      const float* B, int64_t ldb, bool trans_b, float beta, float* C,
-                     int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream);
+                     int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream,
+                     const GemmBatch& bt = GemmBatch());
 
 // ------------------------------------------------------------- factor (factor.cu)
 constexpr int kFactorNB = 128;  // panel width of the blocked Cholesky / inverse

@@ -5,7 +5,9 @@
 // inverse that produce U.
 //
 // 128 x 128 output tile per 256-thread CTA, 8 x 8 outputs per thread, K staged
-// through double-buffered shared memory 8 at a time.
+// through double-buffered shared memory 8 at a time.  Optional batching over
+// blockIdx.z with element strides, where the last entries may have fewer rows
+// (and, for square triangular factors, a matching shorter K).
 #include "internal.h"
 
 namespace piq {
@@ -18,12 +20,27 @@ template <bool TRANS_B, int MODE>
 __global__ void __launch_bounds__(256)
     simt_gemm_kernel(int M, int N, int K, float alpha, const float* A, int64_t lda,
                      const float* B, int64_t ldb, float beta, float* C, int64_t ldc,
-                     const DeviceStatus* st) {
+                     GemmBatch bt, const DeviceStatus* st) {
   const int m0 = blockIdx.y * TM;
   const int n0 = blockIdx.x * TN;
   if (MODE == 1 && n0 >= m0 + TM) return;  // tile strictly above the diagonal
   if (status_bad(st)) return;
-  const int kend = (MODE == 2) ? min(K, m0 + TM) : K;
+  const int z = blockIdx.z;
+  if (bt.count > 1) {
+    A += z * bt.stride_a;
+    B += z * bt.stride_b;
+    C += z * bt.stride_c;
+  }
+  if (bt.m_total > 0) {  // ragged last entries
+    const int64_t mz = bt.m_total - static_cast<int64_t>(z) * bt.m_step;
+    if (mz < M) M = static_cast<int>(mz);
+    if (bt.k_follows_m) K = M;
+    if (M <= 0 || m0 >= M) return;
+  }
+  // K range that can be nonzero: mode 2, A lower (k <= row); mode 3, B lower
+  // used transposed (k <= col); mode 4, B lower used as is (k >= col)
+  const int kend = (MODE == 2) ? min(K, m0 + TM) : (MODE == 3) ? min(K, n0 + TN) : K;
+  const int kbeg = (MODE == 4) ? min(K, n0) & ~(TK - 1) : 0;
 
   __shared__ __align__(16) float As[2][TK][TM + PAD];
   __shared__ __align__(16) float Bs[2][TK][TN + PAD];
@@ -78,12 +95,12 @@ __global__ void __launch_bounds__(256)
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
   int buf = 0;
-  if (kend > 0) {
-    load_tiles(0);
+  if (kend > kbeg) {
+    load_tiles(kbeg);
     store_tiles(0);
   }
   __syncthreads();
-  for (int k0 = 0; k0 < kend; k0 += TK) {
+  for (int k0 = kbeg; k0 < kend; k0 += TK) {
     const bool more = k0 + TK < kend;
     if (more) load_tiles(k0 + TK);
 #pragma unroll
@@ -126,12 +143,13 @@ __global__ void __launch_bounds__(256)
 
 template <bool TB, int MODE>
 int launch_one(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
-               int64_t ldb, float beta, float* C, int64_t ldc, const DeviceStatus* st,
-               cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(ceil_div(N, TN)), static_cast<unsigned>(ceil_div(M, TM)));
+               int64_t ldb, float beta, float* C, int64_t ldc, const GemmBatch& bt,
+               const DeviceStatus* st, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(ceil_div(N, TN)), static_cast<unsigned>(ceil_div(M, TM)),
+            static_cast<unsigned>(bt.count));
   note_launch();
   simt_gemm_kernel<TB, MODE><<<grid, 256, 0, stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C,
-                                                       ldc, st);
+                                                       ldc, bt, st);
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
@@ -139,18 +157,20 @@ int launch_one(int M, int N, int K, float alpha, const float* A, int64_t lda, co
 
 int launch_simt_gemm(int M, int N, int K, float alpha, const float* A, int64_t lda,
                      const float* B, int64_t ldb, bool trans_b, float beta, float* C,
-                     int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream) {
-  if (M <= 0 || N <= 0) return PIQ_OK;
-  if (ceil_div(M, TM) > 65535) return PIQ_ERR_INVALID_ARG;
-  if (trans_b) {
-    if (mode == 0) return launch_one<true, 0>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-    if (mode == 1) return launch_one<true, 1>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-    if (mode == 2) return launch_one<true, 2>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-  } else {
-    if (mode == 0) return launch_one<false, 0>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-    if (mode == 1) return launch_one<false, 1>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-    if (mode == 2) return launch_one<false, 2>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, st, stream);
-  }
+                     int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream,
+                     const GemmBatch& bt) {
+  if (M <= 0 || N <= 0 || bt.count < 1) return PIQ_OK;
+  if (ceil_div(M, TM) > 65535 || bt.count > 65535) return PIQ_ERR_INVALID_ARG;
+#define PIQ_GEMM_CASE(TB, MD)                                                              \
+  if (trans_b == TB && mode == MD)                                                         \
+    return launch_one<TB, MD>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, bt, st, stream);
+  PIQ_GEMM_CASE(true, 0)
+  PIQ_GEMM_CASE(true, 1)
+  PIQ_GEMM_CASE(true, 3)
+  PIQ_GEMM_CASE(false, 0)
+  PIQ_GEMM_CASE(false, 2)
+  PIQ_GEMM_CASE(false, 4)
+#undef PIQ_GEMM_CASE
   return PIQ_ERR_INVALID_ARG;
 }
 

@@ -14,10 +14,15 @@
 // only reads columns whose updates are all applied (g | 128, 128 | g, or any
 // other g), so the arithmetic is the listing's.
 //
-// Kernel layout: one warp per ROWS rows; lane l holds columns l, l+32, l+64,
-// l+96 of its rows in registers; U[b:e, b:e] sits in shared memory.  Column j
-// is broadcast from its owner lane with a shuffle; the division W/scale is IEEE
-// round-to-nearest and rintf rounds half to even (the listing's np.round).
+// Kernel layout: one thread per row (128 rows per CTA).  The row's block
+// columns live in shared memory; a thread walks them in 32-column windows held
+// in registers (the serial column loop with its in-window updates), then
+// applies the window's errors to the later columns of the block.  The strictly
+// upper part of U[b:e, b:e] sits in shared memory and is read by all lanes at
+// the same address (broadcast).  The code stays small enough for the
+// instruction cache: only the 32-column window is unrolled.  W/scale is an IEEE
+// round-to-nearest division and rintf rounds half to even (the listing's
+// np.round); the error uses the reciprocal of U[j, j].
 #include <algorithm>
 #include <vector>
 
@@ -27,110 +32,202 @@ namespace piq {
 
 namespace {
 
-constexpr int B = kSweepB;    // 128
-constexpr int ROWS = 2;       // rows per warp
-constexpr int WARPS = 8;
-constexpr int LDU = B + 1;
+constexpr int B = kSweepB;   // 128 block columns
+constexpr int SUB = 32;      // columns per register window
+constexpr int R = 128;       // rows per CTA, one per thread
+constexpr int LDW = B + 4;   // row-state stride (float4-aligned, conflict-free per 8 lanes)
+constexpr int LDC = B + 4;   // code staging row (bytes)
+constexpr int kSweepSmem = B * B * 4 + B * 4 + R * LDW * 4 + R * LDC;
 
-__global__ void __launch_bounds__(WARPS * 32)
-    sweep_block_kernel(float* __restrict__ W, int64_t out, int64_t in, const float* __restrict__ U,
-                       int64_t b, int kb, int bits, int g, int8_t* __restrict__ codes,
-                       float* __restrict__ qscale, float* __restrict__ Err, DeviceStatus* st) {
-  extern __shared__ float Us[];  // [kb][LDU]
-  if (status_bad(st)) return;
-  for (int idx = threadIdx.x; idx < kb * kb; idx += blockDim.x) {
-    const int r = idx / kb, c = idx % kb;
-    Us[r * LDU + c] = (c >= r) ? U[(b + r) * in + b + c] : 0.f;
+// Per-row state of the column loop.
+struct SweepRow {
+  float scale;
+  int64_t next_gs;   // block-relative column of the next group start
+  float fqmax, cmin, cmax;
+  int kb;
+  int64_t b, in, g, ngroups, row;
+  bool valid;
+};
+
+// Group start at block column j (window base c0, jj = j - c0): the scale comes
+// from the current weights of [j, j+g): the window in registers, later block
+// columns in shared memory minus the updates still pending from window columns
+// before j, and (only when j is the block start) columns past the block in W.
+__device__ __forceinline__ void group_start(const float (&ws)[SUB], const float (&e)[SUB], int jj,
+                                            int c0, SweepRow& st, const float* __restrict__ W,
+                                            const float* Us, const float* wrow,
+                                            float* __restrict__ qscale) {
+  const int j = c0 + jj;
+  const int64_t gend = std::min<int64_t>(st.b + j + st.g, st.in);
+  const int jend = static_cast<int>(std::min<int64_t>(gend - st.b, st.kb));
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < SUB; ++k)
+    if (k >= jj && c0 + k < jend) m = fmaxf(m, fabsf(ws[k]));
+  for (int c = c0 + SUB; c < jend; ++c) {
+    float v = wrow[c];
+#pragma unroll
+    for (int p = 0; p < SUB; ++p)
+      if (p < jj) v = fmaf(-e[p], Us[(c0 + p) * B + c], v);
+    m = fmaxf(m, fabsf(v));
   }
+  if (gend > st.b + st.kb && st.valid) {
+    const float* src = W + st.row * st.in;
+    for (int64_t c = st.b + st.kb; c < gend; ++c) m = fmaxf(m, fabsf(src[c]));
+  }
+  st.scale = __fdiv_rn(m, st.fqmax);
+  if (st.valid) qscale[st.row * st.ngroups + (st.b + j) / st.g] = st.scale;
+  st.next_gs += st.g;
+}
+
+// Column c0 + JJ of the window, then the next: template recursion keeps every
+// register index a compile-time constant.
+template <bool GENERAL, int JJ>
+__device__ __forceinline__ void sweep_col(float (&ws)[SUB], float (&e)[SUB], int c0, SweepRow& st,
+                                          const float* __restrict__ W, const float* Us,
+                                          const float* inv_u, const float* wrow, int8_t* code_row,
+                                          float* __restrict__ qscale) {
+  if constexpr (JJ < SUB) {
+    const int j = c0 + JJ;
+    if (j < st.kb) {
+      if (GENERAL && j == st.next_gs) group_start(ws, e, JJ, c0, st, W, Us, wrow, qscale);
+      const float wj = ws[JJ];
+      const float sc = st.scale;
+      const float q = sc > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(wj, sc)), st.cmin), st.cmax) : 0.f;
+      const float err = (wj - q * sc) * inv_u[j];
+      code_row[j] = static_cast<int8_t>(q);
+      e[JJ] = err;
+      const float4* urow = reinterpret_cast<const float4*>(Us + j * B + c0);
+#pragma unroll
+      for (int k4 = (JJ + 1) >> 2; k4 < SUB / 4; ++k4) {  // U is 0 on and below the diagonal
+        const float4 u = urow[k4];
+        ws[4 * k4 + 0] = fmaf(-err, u.x, ws[4 * k4 + 0]);
+        ws[4 * k4 + 1] = fmaf(-err, u.y, ws[4 * k4 + 1]);
+        ws[4 * k4 + 2] = fmaf(-err, u.z, ws[4 * k4 + 2]);
+        ws[4 * k4 + 3] = fmaf(-err, u.w, ws[4 * k4 + 3]);
+      }
+    } else {
+      e[JJ] = 0.f;
+    }
+    sweep_col<GENERAL, JJ + 1>(ws, e, c0, st, W, Us, inv_u, wrow, code_row, qscale);
+  }
+}
+
+// GENERAL = false: every group start of the block falls on a 32-column window
+// boundary (g a multiple of 32), so scales are taken once per window, outside
+// the unrolled column chain; GENERAL = true handles any g.
+template <bool GENERAL>
+__global__ void __launch_bounds__(R, 1)
+    sweep_block_kernel(float* __restrict__ W, int64_t out, int64_t in,
+                       const float* __restrict__ U, int64_t b, int kb, int bits, int g,
+                       int8_t* __restrict__ codes, float* __restrict__ qscale,
+                       float* __restrict__ Err, DeviceStatus* st) {
+  extern __shared__ __align__(16) float smem[];
+  float* Us = smem;                     // [B][B], strictly upper part of U[b:e, b:e]
+  float* inv_u = Us + B * B;            // [B], 1 / U[j][j]
+  float* Wr = inv_u + B;                // [R][LDW], row state; errors replace used columns
+  int8_t* Cs = reinterpret_cast<int8_t*>(Wr + R * LDW);  // [R][LDC]
+  if (status_bad(st)) return;
+  const int tid = threadIdx.x;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
+
+  // Tiles arrive by asynchronous copies (16-byte when the block start allows);
+  // a second pass zeroes what the column loop must see as zero.
+  const int rows_here = static_cast<int>(std::min<int64_t>(R, out - row0));
+  const float ujj = (tid < kb) ? U[(b + tid) * in + b + tid] : 1.f;  // in flight meanwhile
+  if ((b & 3) == 0) {
+    const int kq = (kb + 3) >> 2;  // b + 4*kq <= in since in % 8 == 0
+    for (int idx = tid; idx < kb * kq; idx += R) {
+      const int r = idx / kq, c = (idx - r * kq) * 4;
+      cp_async16(Us + r * B + c, U + (b + r) * in + b + c);
+    }
+    for (int idx = tid; idx < rows_here * kq; idx += R) {
+      const int r = idx / kq, c = (idx - r * kq) * 4;
+      cp_async16(Wr + r * LDW + c, W + (row0 + r) * in + b + c);
+    }
+  } else {
+    for (int idx = tid; idx < kb * kb; idx += R) {
+      const int r = idx / kb, c = idx - r * kb;
+      cp_async4(Us + r * B + c, U + (b + r) * in + b + c);
+    }
+    for (int idx = tid; idx < rows_here * kb; idx += R) {
+      const int r = idx / kb, c = idx - r * kb;
+      cp_async4(Wr + r * LDW + c, W + (row0 + r) * in + b + c);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  for (int idx = tid; idx < B * B; idx += R) {
+    const int r = idx >> 7, c = idx & (B - 1);
+    if (r >= kb || c >= kb || c <= r) Us[idx] = 0.f;
+  }
+  for (int idx = tid; idx < R * B; idx += R) {
+    const int r = idx >> 7, c = idx & (B - 1);
+    if (r >= rows_here || c >= kb) Wr[r * LDW + c] = 0.f;
+  }
+  inv_u[tid] = (tid < kb) ? 1.f / ujj : 0.f;
   __syncthreads();
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * WARPS + warp) * ROWS;
-  if (row0 >= out) return;
+  SweepRow rs;
   const int qmax = (1 << (bits - 1)) - 1;
-  const float fqmax = static_cast<float>(qmax);
-  const float cmin = static_cast<float>(-qmax - 1), cmax = static_cast<float>(qmax);
-  const int64_t ngroups = (in + g - 1) / g;
+  rs.fqmax = static_cast<float>(qmax);
+  rs.cmin = static_cast<float>(-qmax - 1);
+  rs.cmax = static_cast<float>(qmax);
+  rs.kb = kb;
+  rs.b = b;
+  rs.in = in;
+  rs.g = g;
+  rs.ngroups = (in + g - 1) / g;
+  rs.row = row0 + tid;
+  rs.valid = rs.row < out;
+  const int64_t boff = b % g;
+  // a group that started in an earlier block keeps its scale
+  rs.scale = (boff != 0 && rs.valid) ? qscale[rs.row * rs.ngroups + b / g] : 0.f;
+  rs.next_gs = (boff == 0) ? 0 : g - boff;
 
-  float w[ROWS][4], e[ROWS][4], sc[ROWS];
-  int cq[ROWS][4];
-  bool valid[ROWS];
+  float* wrow = Wr + tid * LDW;
+  int8_t* crow = Cs + tid * LDC;
+  for (int c0 = 0; c0 < kb; c0 += SUB) {
+    float ws[SUB], e[SUB];
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    valid[r] = row0 + r < out;
-    sc[r] = 0.f;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int c = 32 * t + lane;
-      w[r][t] = (valid[r] && c < kb) ? W[(row0 + r) * in + b + c] : 0.f;
-      e[r][t] = 0.f;
-      cq[r][t] = 0;
+    for (int k4 = 0; k4 < SUB / 4; ++k4) {
+      const float4 v = reinterpret_cast<const float4*>(wrow + c0)[k4];
+      ws[4 * k4] = v.x;
+      ws[4 * k4 + 1] = v.y;
+      ws[4 * k4 + 2] = v.z;
+      ws[4 * k4 + 3] = v.w;
     }
-  }
-  // scale of a group that started before this block (b not a group start)
-  if (b % g != 0) {
-    const int64_t grp = b / g;
+    if (!GENERAL && c0 == rs.next_gs) {
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) sc[r] = valid[r] ? qscale[(row0 + r) * ngroups + grp] : 0.f;
-  }
-
+      for (int p = 0; p < SUB; ++p) e[p] = 0.f;
+      group_start(ws, e, 0, c0, rs, W, Us, wrow, qscale);
+    }
+    sweep_col<GENERAL, 0>(ws, e, c0, rs, W, Us, inv_u, wrow, crow, qscale);
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-#pragma unroll 4
-    for (int o = 0; o < 32; ++o) {
-      const int j = 32 * s + o;
-      if (j >= kb) break;
-      const int64_t p = b + j;
-      if (p % g == 0) {  // group start: scale from the current weights
-        const int64_t gend = std::min<int64_t>(p + g, in);
-        const int jend = static_cast<int>(std::min<int64_t>(gend - b, kb));
+    for (int k4 = 0; k4 < SUB / 4; ++k4)
+      reinterpret_cast<float4*>(wrow + c0)[k4] =
+          make_float4(e[4 * k4], e[4 * k4 + 1], e[4 * k4 + 2], e[4 * k4 + 3]);
+    // the window's errors update every later column of the block
+    for (int k4 = (c0 + SUB) / 4; k4 < B / 4; ++k4) {
+      float4 acc = reinterpret_cast<const float4*>(wrow)[k4];
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-          float m = 0.f;
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int c = 32 * t + lane;
-            if (c >= j && c < jend) m = fmaxf(m, fabsf(w[r][t]));
-          }
-          if (gend > b + kb && valid[r]) {  // group runs past the block: current W in memory
-            const float* src = W + (row0 + r) * in;
-            for (int64_t c = b + kb + lane; c < gend; c += 32) m = fmaxf(m, fabsf(src[c]));
-          }
-          m = warp_max(m);
-          sc[r] = __fdiv_rn(m, fqmax);
-          if (lane == 0 && valid[r]) qscale[(row0 + r) * ngroups + p / g] = sc[r];
-        }
+      for (int p = 0; p < SUB; ++p) {
+        const float4 u = reinterpret_cast<const float4*>(Us + (c0 + p) * B)[k4];
+        acc.x = fmaf(-e[p], u.x, acc.x);
+        acc.y = fmaf(-e[p], u.y, acc.y);
+        acc.z = fmaf(-e[p], u.z, acc.z);
+        acc.w = fmaf(-e[p], u.w, acc.w);
       }
-      const float ujj = Us[j * LDU + j];
-#pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        const float wj = __shfl_sync(0xffffffffu, w[r][s], o);
-        float q = 0.f;
-        if (sc[r] > 0.f) q = fminf(fmaxf(rintf(__fdiv_rn(wj, sc[r])), cmin), cmax);
-        const float err = __fdiv_rn(wj - q * sc[r], ujj);
-        if (lane == o) {
-          cq[r][s] = static_cast<int>(q);
-          e[r][s] = err;
-        }
-#pragma unroll
-        for (int t = s; t < 4; ++t) {
-          const int c = 32 * t + lane;
-          if (c > j) w[r][t] = fmaf(-err, Us[j * LDU + c], w[r][t]);
-        }
-      }
+      reinterpret_cast<float4*>(wrow)[k4] = acc;
     }
   }
 
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    if (!valid[r]) continue;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int c = 32 * t + lane;
-      if (c < kb) {
-        codes[(row0 + r) * in + b + c] = static_cast<int8_t>(cq[r][t]);
-        Err[(row0 + r) * B + c] = e[r][t];
-      }
+  __syncthreads();
+  for (int idx = tid; idx < R * B; idx += R) {  // coalesced write-out
+    const int r = idx / B, c = idx % B;
+    if (row0 + r < out && c < kb) {
+      codes[(row0 + r) * in + b + c] = Cs[r * LDC + c];
+      Err[(row0 + r) * B + c] = Wr[r * LDW + c];
     }
   }
 }
@@ -161,23 +258,33 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
-  const int smem = B * LDU * static_cast<int>(sizeof(float));
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(sweep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(sweep_block_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSweepSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(sweep_block_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSweepSmem) !=
+            cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
   }
   std::vector<std::pair<int64_t, int64_t>> blocks;
   block_partition(in, g, &blocks);
-  const int64_t rows_per_cta = WARPS * ROWS;
-  const unsigned grid = static_cast<unsigned>(ceil_div(out, rows_per_cta));
+  const unsigned grid = static_cast<unsigned>(ceil_div(out, R));
   for (const auto& be : blocks) {
     const int64_t b = be.first, e = be.second;
     const int kb = static_cast<int>(e - b);
+    // do all group starts inside the block fall on window boundaries?
+    bool aligned = true;
+    for (int64_t gs = (b % g == 0) ? b : (b / g + 1) * g; gs < e; gs += g)
+      aligned = aligned && ((gs - b) % SUB == 0);
     note_launch();
-    sweep_block_kernel<<<grid, WARPS * 32, smem, stream>>>(Wq, out, in, U, b, kb, bits, g, codes,
-                                                           qscale, Err, st);
+    if (aligned)
+      sweep_block_kernel<false><<<grid, R, kSweepSmem, stream>>>(Wq, out, in, U, b, kb, bits, g,
+                                                                 codes, qscale, Err, st);
+    else
+      sweep_block_kernel<true><<<grid, R, kSweepSmem, stream>>>(Wq, out, in, U, b, kb, bits, g,
+                                                                codes, qscale, Err, st);
     if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
     if (e < in) {
       // W[:, e:] -= Err[:, :kb] U[b:e, e:]

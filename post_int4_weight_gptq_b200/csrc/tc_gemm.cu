@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // an earlier step already failed: do nothing (uniform over the CTA)
+  if (status_bad(p.st)) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

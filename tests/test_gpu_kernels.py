@@ -19,7 +19,7 @@ def _layer(out, inp, n, seed=0, **kw):
 @pytest.mark.parametrize("n,inp", [(2048, 512), (1000, 136), (77, 264), (4100, 1032), (64, 8)])
 def test_hessian_matches_exact(n, inp):
     W, X = _layer(8, inp, n, seed=n + inp)
-    H = piq.hessian(to_gpu_x(X)).cpu().numpy().astype(np.float64)
+    H = np.triu(piq.hessian(to_gpu_x(X)).cpu().numpy()).astype(np.float64)
     Hx = O.hessian_ref(X)
     d = np.sqrt(np.outer(np.diag(Hx), np.diag(Hx)))
     iu = np.triu_indices(inp)
@@ -70,7 +70,7 @@ def test_sweep_given_u(out, inp, g, bits):
     W, X = _layer(out, inp, 3 * inp, seed=out * inp)
     Hx = O.hessian_ref(X)
     _, Ux, _ = O.gptq_prepare_ref(Hx, 0.01, False)
-    U32 = Ux.astype(np.float32)
+    U32 = np.ascontiguousarray(Ux, dtype=np.float32)
     codes, qscale = piq.gptq_sweep(to_gpu_w(W), torch.from_numpy(U32).cuda(), bits, g)
     stats, c_ref, s_ref = teacher_forced_compare(codes.cpu().numpy(), W.astype(np.float64),
                                                  U32.astype(np.float64), bits, g)
@@ -87,7 +87,7 @@ def test_output_error_gemm_matches_oracle():
     codes = unpack_gpu(qw, 4)
     What = codes * np.repeat(sc.cpu().numpy().astype(np.float64), 128, axis=1)[:, :520]
     ex = O.output_error_ref(W, What, X)
-    assert rel(e, ex) < 1e-4
+    assert rel(e, ex) < REL_TOL  # bf16 rounding of W - What is the dominant term
 
 
 def test_rtn_matches_oracle():
