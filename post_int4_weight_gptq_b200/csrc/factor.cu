@@ -349,11 +349,11 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     float* A21 = P + (k0 + nb) * ld + k0;
     const float* X11 = X + k0 * ld + k0;
     // L21 = A21 X11^T in place (nb <= 128: one CTA column)
-    int rc = launch_simt_gemm(rem, nb, nb, 1.f, A21, ld, X11, ld, true, 0.f, A21, ld, 3, st,
+    int rc = launch_gemm_f32(rem, nb, nb, 1.f, A21, ld, X11, ld, true, 0.f, A21, ld, 3, st,
                               stream);
     if (rc != PIQ_OK) return rc;
     // A22 -= L21 L21^T (lower tiles)
-    rc = launch_simt_gemm(rem, rem, nb, -1.f, A21, ld, A21, ld, true, 1.f,
+    rc = launch_gemm_f32(rem, rem, nb, -1.f, A21, ld, A21, ld, true, 1.f,
                           P + (k0 + nb) * ld + (k0 + nb), ld, 1, st, stream);
     if (rc != PIQ_OK) return rc;
   }
@@ -370,7 +370,7 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     bt.stride_a = 2 * s * (ld + 1);
     bt.stride_b = 2 * s * (ld + 1);
     bt.stride_c = s * s;
-    int rc = launch_simt_gemm(si, si, si, 1.f, P + s * ld, ld, X, ld, false, 0.f, T, s, 4, st,
+    int rc = launch_gemm_f32(si, si, si, 1.f, P + s * ld, ld, X, ld, false, 0.f, T, s, 4, st,
                               stream, bt);
     if (rc != PIQ_OK) return rc;
     // X21_p = -X22_p T_p   (X22 lower, K = its rows)
@@ -378,7 +378,7 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     bt.stride_b = s * s;
     bt.stride_c = 2 * s * (ld + 1);
     bt.k_follows_m = true;
-    rc = launch_simt_gemm(si, si, si, -1.f, X + s * ld + s, ld, T, s, false, 0.f, X + s * ld, ld,
+    rc = launch_gemm_f32(si, si, si, -1.f, X + s * ld + s, ld, T, s, false, 0.f, X + s * ld, ld,
                           2, st, stream, bt);
     if (rc != PIQ_OK) return rc;
   }

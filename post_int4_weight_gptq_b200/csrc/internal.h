@@ -50,6 +50,18 @@ int launch_simt_gemm(int M, int N, int K, float alpha, const float* A, int64_t l
                      int64_t ldc, int mode, const DeviceStatus* st, cudaStream_t stream,
                      const GemmBatch& bt = GemmBatch());
 
+// ------------------------------------------- FP32-accurate tensor-core GEMM (tc_sgemm.cu)
+// Same contract as launch_simt_gemm, on tcgen05 (three TF32 passes).  Returns
+// PIQ_ERR_INVALID_ARG when an operand is not TMA-compatible (16-byte aligned
+// base and row stride); launch_gemm_f32 then falls back to the SIMT kernel.
+int launch_tc_sgemm(int M, int N, int K, float alpha, const float* A, int64_t lda,
+                    const float* B, int64_t ldb, bool trans_b, float beta, float* C, int64_t ldc,
+                    int mode, DeviceStatus* st, cudaStream_t stream,
+                    const GemmBatch& bt = GemmBatch());
+int launch_gemm_f32(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
+                    int64_t ldb, bool trans_b, float beta, float* C, int64_t ldc, int mode,
+                    DeviceStatus* st, cudaStream_t stream, const GemmBatch& bt = GemmBatch());
+
 // ------------------------------------------------------------- factor (factor.cu)
 constexpr int kFactorNB = 128;  // panel width of the blocked Cholesky / inverse
 int64_t factor_workspace_floats(int64_t in);  // P + Dinv + T

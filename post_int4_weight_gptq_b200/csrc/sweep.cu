@@ -288,7 +288,7 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
     if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
     if (e < in) {
       // W[:, e:] -= Err[:, :kb] U[b:e, e:]
-      int rc = launch_simt_gemm(static_cast<int>(out), static_cast<int>(in - e), kb, -1.f, Err, B,
+      int rc = launch_gemm_f32(static_cast<int>(out), static_cast<int>(in - e), kb, -1.f, Err, B,
                                 U + b * in + e, in, false, 1.f, Wq + e, in, 0, st, stream);
       if (rc != PIQ_OK) return rc;
     }
