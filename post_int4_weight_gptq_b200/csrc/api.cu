@@ -216,7 +216,7 @@ AwqWs carve_awq(Carver& c, int64_t out, int64_t in, int64_t n, int n_alpha) {
   w.colpart = c.take<double>(static_cast<int64_t>(colstats_splits(n, in)) * in * 2);
   w.mean_abs = c.take<double>(in);
   w.alphas = c.take<float>(64);
-  w.s_table = c.take<float>(static_cast<int64_t>(n_alpha) * in);
+  w.s_table = c.take<float>(2 * static_cast<int64_t>(n_alpha) * in);  // s, then 1/s
   w.dW = c.take<uint16_t>(static_cast<int64_t>(n_alpha) * out * in);
   w.partials = c.take<double>(sumsq_partials_count(n, out, n_alpha));
   w.err = c.take<double>(64);

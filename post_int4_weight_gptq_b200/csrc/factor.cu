@@ -81,8 +81,9 @@ __device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lan
   if constexpr (J < SP) {
     const float d = __shfl_sync(FULL, a[J], J);
     ok = ok && (d > 0.f);
-    const float ljj = sqrtf(d > 0.f ? d : 1.f);
-    const float r = 1.f / ljj;
+    const float dd = d > 0.f ? d : 1.f;
+    const float r = rsqrtf(dd);  // 1 / L_JJ
+    const float ljj = dd * r;     // L_JJ
     if (lane == J) rdiag = r;
     const float lij = (lane > J) ? a[J] * r : (lane == J ? ljj : 0.f);
     a[J] = lij;

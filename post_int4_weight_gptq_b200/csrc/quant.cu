@@ -169,7 +169,9 @@ __global__ void awq_scale_table_kernel(const double* __restrict__ mean_abs, int6
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int a = static_cast<int>(idx / in);
     const double m = mean_abs[idx - a * in];
-    s_table[idx] = m > 0.0 ? static_cast<float>(pow(m, static_cast<double>(alphas[a]))) : 1.f;
+    const float sv = m > 0.0 ? static_cast<float>(pow(m, static_cast<double>(alphas[a]))) : 1.f;
+    s_table[idx] = sv;
+    s_table[total + idx] = 1.f / sv;  // reciprocals follow the scales
   }
 }
 
@@ -215,6 +217,53 @@ __global__ void awq_delta_kernel(const float* __restrict__ W, int64_t out, int64
         const float w = wrow[c];
         const float q = quant_code(w * s[c], scale, cmin, cmax);
         drow[c] = float_to_bf16_bits(w - __fdiv_rn(q * scale, s[c]));
+      }
+    }
+  }
+}
+
+// Vector form of awq_delta_kernel for g % 4 == 0 and g <= 128: lane l holds
+// columns [4l, 4l+4) of one (row, group); W is read once for every alpha.  The
+// code decision keeps the IEEE quotient W'/scale; the dequantised weight uses
+// the precomputed reciprocal of s.
+__global__ void __launch_bounds__(256)
+    awq_delta_vec_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits, int g,
+                         const float* __restrict__ s_table, int n_alpha,
+                         uint16_t* __restrict__ dW) {
+  const int64_t ngroups = (in + g - 1) / g;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int qmax = (1 << (bits - 1)) - 1;
+  const float fqmax = static_cast<float>(qmax), cmin = static_cast<float>(-qmax - 1),
+              cmax = static_cast<float>(qmax);
+  const float* inv_table = s_table + static_cast<int64_t>(n_alpha) * in;
+  for (int64_t wi = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wi < out * ngroups; wi += nwarps) {
+    const int64_t r = wi / ngroups, grp = wi - r * ngroups;
+    const int64_t c0 = grp * g;
+    const int len = static_cast<int>(std::min<int64_t>(g, in - c0));  // multiple of 4
+    const bool act = 4 * lane < len;
+    const int64_t col = c0 + 4 * lane;
+    const float4 w = act ? *reinterpret_cast<const float4*>(W + r * in + col)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int a = 0; a < n_alpha; ++a) {
+      const int64_t off = static_cast<int64_t>(a) * in + col;
+      const float4 sv = act ? *reinterpret_cast<const float4*>(s_table + off)
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+      const float4 iv = act ? *reinterpret_cast<const float4*>(inv_table + off)
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+      const float p0 = w.x * sv.x, p1 = w.y * sv.y, p2 = w.z * sv.z, p3 = w.w * sv.w;
+      float m = fmaxf(fmaxf(fabsf(p0), fabsf(p1)), fmaxf(fabsf(p2), fabsf(p3)));
+      const float scale = __fdiv_rn(warp_max(m), fqmax);
+      const float q0 = quant_code(p0, scale, cmin, cmax), q1 = quant_code(p1, scale, cmin, cmax);
+      const float q2 = quant_code(p2, scale, cmin, cmax), q3 = quant_code(p3, scale, cmin, cmax);
+      if (act) {
+        uint2 o;
+        o.x = float_to_bf16_bits(w.x - q0 * scale * iv.x) |
+              (static_cast<uint32_t>(float_to_bf16_bits(w.y - q1 * scale * iv.y)) << 16);
+        o.y = float_to_bf16_bits(w.z - q2 * scale * iv.z) |
+              (static_cast<uint32_t>(float_to_bf16_bits(w.w - q3 * scale * iv.w)) << 16);
+        *reinterpret_cast<uint2*>(dW + (static_cast<int64_t>(a) * out + r) * in + col) = o;
       }
     }
   }
@@ -358,8 +407,12 @@ int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,
                      const float* s_table, int n_alpha, uint16_t* dW, cudaStream_t stream) {
   const int64_t warps = out * ceil_div(in, g);
   note_launch();
-  awq_delta_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g, s_table,
-                                                                   n_alpha, dW);
+  if (g % 4 == 0 && g <= 128)
+    awq_delta_vec_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g,
+                                                                        s_table, n_alpha, dW);
+  else
+    awq_delta_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g, s_table,
+                                                                     n_alpha, dW);
   return last_error();
 }
 
