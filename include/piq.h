@@ -174,6 +174,29 @@ const char* piq_phase_name(int i);
  * a monotone diagnostic counter. */
 uint64_t piq_kernel_launches(void);
 
+/* piq_upper_factor without a caller workspace.  (The source pages have no
+ * counterpart: this is a deployment variant of the damping + upper-factor step
+ * above, same arguments minus the workspace, same results.)
+ *
+ * For callers that must not allocate device memory: code that runs inside
+ * another framework's hook or plugin, where every device byte belongs to a
+ * pool that framework owns, and callers that cannot afford cudaMalloc's
+ * implicit device-wide synchronisation.  The scratch lives instead in a fixed
+ * region inside this library (a file-scope __device__ array of about 2.4 MB
+ * that every GPU which loads the library keeps until the process exits).
+ *   - in <= PIQ_NOALLOC_MAX_IN (512); a larger in returns PIQ_ERR_INVALID_ARG
+ *     and does nothing.  No device memory is allocated or freed.
+ *   - The first call on a device looks up the region's device address for that
+ *     device (cudaGetSymbolAddress, with that device current); make that first
+ *     call before capturing any stream.
+ *   - All calls on a device share the one region, which keeps the last call's
+ *     contents (the status word is cleared on every call).  Calls that overlap
+ *     on the GPU (different streams or threads) race on it: serialise them.
+ *   - Synchronizes `stream` once, like piq_upper_factor. */
+#define PIQ_NOALLOC_MAX_IN 512
+int piq_upper_factor_noalloc(const float* H, int64_t in, float damp, const int32_t* perm,
+                             float* U, double* lambda_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -74,6 +74,8 @@ SIGNATURES = {
                                       ctypes.POINTER(_c_int)]),
     "piq_phase_name": (ctypes.c_char_p, [_c_int]),
     "piq_kernel_launches": (ctypes.c_uint64, []),
+    "piq_upper_factor_noalloc": (_c_int, [_vp, _c_i64, _c_float, _vp, _vp,
+                                          ctypes.POINTER(ctypes.c_double), _vp]),
 }
 
 _lib = None
@@ -300,3 +302,22 @@ def last_phase_times() -> dict:
 def kernel_launches() -> int:
     """Kernels launched by libpiq in this process so far."""
     return int(load_library().piq_kernel_launches())
+
+
+NOALLOC_MAX_IN = 512
+
+
+def upper_factor_noalloc(H, damp=0.01, perm=None, stream=None):
+    """upper_factor for callers that must not allocate device memory: the
+    scratch is a fixed region inside the library (in <= NOALLOC_MAX_IN).  Only
+    the output U is created here (pass-through of the C entry point)."""
+    lib = load_library()
+    _need(H, torch.float32, "H")
+    if perm is not None:
+        _need(perm, torch.int32, "perm")
+    U = torch.empty_like(H)
+    lam = ctypes.c_double(0.0)
+    _check(lib.piq_upper_factor_noalloc(_ptr(H), H.shape[0], float(damp), _ptr(perm), _ptr(U),
+                                        ctypes.byref(lam), _stream(stream)),
+           "piq_upper_factor_noalloc")
+    return U, lam.value
