@@ -261,7 +261,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks, peak_src = load_peaks()
 
-    W, X, X2 = make_inputs(rank)
+    W, X, X2 = make_inputs(rank, n=args.samples)
     out_rows, inp = W.shape
     n = X.shape[0]
     Wg, Xg, X2g = to_gpu_w(W, dev), to_gpu_x(X, dev), to_gpu_x(X2, dev)
@@ -428,6 +428,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--awq", action="store_true", help="also time the AWQ search (8192^2 layer)")
+    ap.add_argument("--samples", type=int, default=None,
+                    help="calibration rows per layer (default: the workload's 131072); a smaller "
+                         "value is for profiler captures, not for reported numbers")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per err_sumsq launch from an ncu capture, if current")
     args = ap.parse_args(argv)

@@ -72,8 +72,11 @@ int piq_hessian_bytes(int64_t in, size_t* bytes);
  *   X  device bf16 [n, in] row-major, read-only.
  *   H  device fp32 [in, in] row-major.  Every element on or above the diagonal
  *      is written (H[i][j], j >= i); elements below the diagonal are
- *      unspecified.  BF16 products, FP32 accumulation on the tensor cores.
- * n >= 1, in >= 8 and in % 8 == 0. */
+ *      unspecified.  BF16 products, FP32 accumulation on the tensor cores in
+ *      chunks of 4096 samples; the chunks are added into H in sample order
+ *      (FP32), so the result is deterministic.
+ * n >= 1, in >= 8, in % 8 == 0; X and H 16-byte aligned (else
+ * PIQ_ERR_INVALID_ARG). */
 int piq_hessian(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
                 void* stream);
 

@@ -6,7 +6,12 @@
 //                ("A strong answer", listing: H = X.T @ X).  X[n, in] is
 //                row-major, so both operands are MN-major tiles (the sample
 //                index n is the contraction).  Only tiles touching the upper
-//                triangle are computed.
+//                triangle are computed.  The sample range is cut into chunks of
+//                KC samples: each chunk's fp32 tile leaves TMEM and is added into
+//                H by a TMA reduce (the first chunk stores), one chunk after the
+//                other by the CTA that owns the tile, so the sum is deterministic
+//                and the tensor-core accumulation error grows with KC rather
+//                than with n.
 //   * err_sumsq  E_b = ||X D_b^T||_F^2 for stacked D_b (D = W - What), the
 //                shared objective of both methods ("How to approach it").  Both
 //                operands are K-major; the epilogue squares and sums the
@@ -37,10 +42,21 @@ constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int GROUP_M = 16;                     // raster group (err_sumsq)
+// Samples per TMEM accumulation before the tile is flushed into H.  The
+// relative error of the tensor-core fp32 sum grows about linearly with the
+// number of MMAs accumulated in place; 4096 samples (256 MMAs of k = 16) keep
+// it near 2e-5 of sqrt(H_ii H_jj) whatever n is.
+constexpr int KC = 4096;
+constexpr int STG_BYTES = 4 * 2 * 32 * 32 * 4;  // H epilogue: two 32x32 fp32 slabs per warp
 
 enum { EPI_STORE_UPPER = 0, EPI_SUMSQ = 1 };
+
+template <int EPI>
+constexpr int smem_bytes() {
+  return STAGES * STAGE_BYTES + (EPI == EPI_STORE_UPPER ? STG_BYTES : 0) + 1024 /*align*/ +
+         256 /*barriers*/;
+}
 
 struct Params {
   int M, N, K;
@@ -49,6 +65,7 @@ struct Params {
   float* C;
   int64_t ldc;
   int accumulate;
+  int kb_chunk;  // k blocks per accumulation chunk (>= number of k blocks: one chunk)
   double* partials;
   DeviceStatus* st;
 };
@@ -86,11 +103,14 @@ __device__ __forceinline__ void decode_tile(const Params& p, int t, int& mt, int
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                   const __grid_constant__ CUtensorMap tmB, Params p) {
+                   const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  float* stg_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // H epilogue only
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      smem + STAGES * STAGE_BYTES + (EPI == EPI_STORE_UPPER ? STG_BYTES : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
@@ -113,6 +133,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI == EPI_STORE_UPPER) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -123,6 +144,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (p.K + BK - 1) / BK;
+  const int n_chunks = num_kb <= p.kb_chunk ? 1 : 1 + (num_kb - 1) / p.kb_chunk;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -166,94 +188,129 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t it = 0;
       int lt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++lt) {
-        const int buf = lt & 1;
-        const uint32_t use = static_cast<uint32_t>(lt >> 1);
-        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 2)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph, p.st, 3)) {
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        for (int ch = 0; ch < n_chunks && ok; ++ch, ++lt) {
+          const int buf = lt & 1;
+          const uint32_t use = static_cast<uint32_t>(lt >> 1);
+          if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 2)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+          const int kb0 = ch * p.kb_chunk;
+          const int kb1 = num_kb - kb0 <= p.kb_chunk ? num_kb : kb0 + p.kb_chunk;
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!mbar_wait(&full[s], ph, p.st, 3)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kLayoutSw128)
-                                     : smem_desc(a_addr + kk * 32, 16, 1024, kLayoutSw128);
-            const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 8192, 1024, kLayoutSw128)
-                                     : smem_desc(b_addr + kk * 32, 16, 1024, kLayoutSw128);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kLayoutSw128)
+                                       : smem_desc(a_addr + kk * 32, 16, 1024, kLayoutSw128);
+              const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 8192, 1024, kLayoutSw128)
+                                       : smem_desc(b_addr + kk * 32, 16, 1024, kLayoutSw128);
+              umma_bf16(d_tmem, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[s]);  // frees the stage once these MMAs finish
           }
-          umma_commit(&empty[s]);  // frees the stage once these MMAs finish
+          if (ok) umma_commit(&acc_full[buf]);
         }
-        if (ok) umma_commit(&acc_full[buf]);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
     int lt = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
-      const int buf = lt & 1;
-      const uint32_t use = static_cast<uint32_t>(lt >> 1);
-      int mt, nt, bz;
-      decode_tile<EPI>(p, t, mt, nt, bz);
-      if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) break;
-      tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
-      const int row = mt * BM + q * 32 + lane;
-      double acc = 0.0;
+    if (EPI == EPI_SUMSQ) {
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        const uint32_t use = static_cast<uint32_t>(lt >> 1);
+        if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) break;
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+        double acc = 0.0;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        if (EPI == EPI_SUMSQ) {
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
           float s = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) s = fmaf(v[i], v[i], s);
           acc += static_cast<double>(s);
-        } else {
-          const int col0 = nt * BN + c * 32;
-          // chunks entirely below the diagonal are not needed
-          if (row < p.M && col0 < p.N && col0 + 32 > row) {
-            float* dst = p.C + static_cast<int64_t>(row) * p.ldc + col0;
-            if (col0 + 32 <= p.N) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                float4 o = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                if (p.accumulate) {
-                  const float4 old = *reinterpret_cast<const float4*>(dst + i);
-                  o.x += old.x;
-                  o.y += old.y;
-                  o.z += old.z;
-                  o.w += old.w;
-                }
-                *reinterpret_cast<float4*>(dst + i) = o;
-              }
-            } else {
-              const int lim = p.N - col0;
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (i < lim) dst[i] = p.accumulate ? dst[i] + v[i] : v[i];
-            }
-          }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      if (EPI == EPI_SUMSQ) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
         // one partial per (tile, lane quarter): no cross-warp synchronisation
         acc = warp_sum_d(acc);
         if (lane == 0) p.partials[static_cast<int64_t>(t) * 4 + q] = acc;
       }
+    } else {
+      // Each warp owns 32 rows of the tile and moves them out in 32x32 slabs
+      // through a double-buffered staging tile in the TMA 128-byte swizzle
+      // (16-byte chunk k of row r sits at chunk k ^ (r % 8)).  A chunk's slabs
+      // are stored (first chunk, accumulate == 0) or reduce-added into H; the
+      // next chunk of the same tile waits until they have all landed, so the
+      // additions into H happen in chunk order.
+      float* stg = stg_all + q * 2 * 1024;
+      uint32_t nst = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mt, nt, bz;
+        decode_tile<EPI>(p, t, mt, nt, bz);
+        const int row0 = mt * BM + q * 32;
+        for (int ch = 0; ch < n_chunks; ++ch, ++lt) {
+          const int buf = lt & 1;
+          const uint32_t use = static_cast<uint32_t>(lt >> 1);
+          if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0 && ch > 0) bulk_wait_all();  // previous chunk's additions landed
+          __syncwarp();
+          const bool store = ch == 0 && p.accumulate == 0;
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            const int col0 = nt * BN + c * 32;
+            // slabs wholly below the diagonal, or outside H, are not needed
+            if (row0 >= p.M || col0 >= p.N || col0 + 32 <= row0) continue;
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);  // lane = row, v[i] = column i
+            float* sb = stg + (nst & 1) * 1024;
+            if (lane == 0) bulk_wait_read<1>();  // this buffer's previous copy has read it
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              *reinterpret_cast<float4*>(sb + lane * 32 + ((k ^ (lane & 7)) << 2)) =
+                  make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (store)
+                tma_store_3d(&tmC, sb, col0, row0, 0);
+              else
+                tma_reduce_add_3d(&tmC, sb, col0, row0, 0);
+              bulk_commit();
+            }
+            ++nst;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+      }
+      if (lane == 0) bulk_wait_all();  // every copy of this warp has landed
     }
   }
 
@@ -285,9 +342,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map, innermost dimension first.
+// Tensor map (bf16 operands or the fp32 H), innermost dimension first, 128-byte swizzle.
 int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-             const uint64_t* strides_bytes, const uint32_t* box) {
+             const uint64_t* strides_bytes, const uint32_t* box,
+             CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return PIQ_ERR_CUDA;
   cuuint64_t d[3], s[2];
@@ -297,20 +355,22 @@ int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
     b[i] = box[i];
   }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b,
-                  e, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, type, rank, const_cast<void*>(base), d, s, b, e,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PIQ_OK : PIQ_ERR_INVALID_ARG;
 }
 
 template <bool A_MN, bool B_MN, int EPI>
-int launch(const CUtensorMap& a, const CUtensorMap& b, const Params& p, cudaStream_t stream) {
+int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, const Params& p,
+           cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   auto kern = tc_gemm_kernel<A_MN, B_MN, EPI>;
+  constexpr int smem = smem_bytes<EPI>();
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
@@ -320,7 +380,7 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const Params& p, cudaStre
   if (rc != PIQ_OK) return rc;
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
   note_launch();
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(a, b, p);
+  kern<<<grid, THREADS, smem, stream>>>(a, b, c, p);
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
@@ -330,12 +390,22 @@ int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accu
                     DeviceStatus* st, cudaStream_t stream) {
   if (n < 1 || in < 8 || in % 8 != 0 || n > INT32_MAX || in > INT32_MAX / 2)
     return PIQ_ERR_INVALID_ARG;
-  CUtensorMap map;
+  if ((reinterpret_cast<uintptr_t>(X) & 15u) != 0 || (reinterpret_cast<uintptr_t>(H) & 15u) != 0)
+    return PIQ_ERR_INVALID_ARG;
+  CUtensorMap map, mc;
   const uint64_t dims[2] = {static_cast<uint64_t>(in), static_cast<uint64_t>(n)};
   const uint64_t strides[1] = {static_cast<uint64_t>(in) * 2};
   const uint32_t box[2] = {64, 64};
   int rc = make_map(&map, X, 2, dims, strides, box);
   if (rc != PIQ_OK) return rc;
+  {
+    const uint64_t cd[3] = {static_cast<uint64_t>(in), static_cast<uint64_t>(in), 1};
+    const uint64_t cs[2] = {static_cast<uint64_t>(in) * 4,
+                            static_cast<uint64_t>(in) * static_cast<uint64_t>(in) * 4};
+    const uint32_t cb[3] = {32, 32, 1};
+    rc = make_map(&mc, H, 3, cd, cs, cb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    if (rc != PIQ_OK) return rc;
+  }
   Params p{};
   p.M = p.N = static_cast<int>(in);
   p.K = static_cast<int>(n);
@@ -349,8 +419,9 @@ int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accu
   p.C = H;
   p.ldc = in;
   p.accumulate = accumulate;
+  p.kb_chunk = KC / BK;
   p.st = st;
-  return launch<true, true, EPI_STORE_UPPER>(map, map, p, stream);
+  return launch<true, true, EPI_STORE_UPPER>(map, map, mc, p, stream);
 }
 
 int64_t sumsq_partials_count(int64_t n, int64_t rows, int batch) {
@@ -390,8 +461,9 @@ int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D
   if (total > INT32_MAX) return PIQ_ERR_INVALID_ARG;
   p.num_tiles = static_cast<int>(total);
   p.partials = partials;
+  p.kb_chunk = INT32_MAX;  // one accumulation per tile
   p.st = st;
-  return launch<false, false, EPI_SUMSQ>(ma, mb, p, stream);
+  return launch<false, false, EPI_SUMSQ>(ma, mb, ma, p, stream);
 }
 
 // ------------------------------------------------ fixed-order partial reduction

@@ -101,10 +101,6 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
   return r;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Instruction descriptor: kind::tf32, fp32 accumulate, M = 128, N = 128.
 __host__ __device__ constexpr uint32_t idesc_tf32(bool b_mn_major) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn_major ? 1u : 0u) << 16) |

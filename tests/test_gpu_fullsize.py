@@ -1,0 +1,91 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py uses.
+
+The oracle builds H and U in float64 on the host cores (seconds to minutes at
+these sizes), then:
+  * codes and scales: a seeded sample of rows is swept by the literal loop and
+    compared teacher-forced with the GPU's codes (rows are independent given U);
+  * output error: the oracle's own blocked sweep of every row, dequantized with
+    fp16 scales, scored in float64 on X (and on the shifted X' for q_proj).
+The 70B-shaped layer and the AWQ 8192^2 search take several minutes of host
+float64 work; they run when PIQ_FULLSIZE_SLOW=1.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+import post_int4_weight_gptq_b200 as piq
+from oracle.gptq import gptq_sweep_blocked_ref
+from oracle.pack import dequant_ref
+from tests.parity import REL_TOL, rel, teacher_forced_compare, to_gpu_w, to_gpu_x, unpack_gpu
+from workloads import AWQ_GRID, C2, C3, C4, C5, make_weight, make_x_bits
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+SLOW = os.environ.get("PIQ_FULLSIZE_SLOW") == "1"
+
+
+def _gptq_full(spec, bits=None, shift=False, sample_rows=48):
+    bits = spec.bits if bits is None else bits
+    W = make_weight(spec)
+    X = make_x_bits(spec)
+    out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X), bits=bits, g=spec.g,
+                                  damp=spec.damp, act_order=spec.act_order)
+    qweight, scales = out.qweight, out.scales
+    e2_gpu = None
+    if shift:
+        X2 = make_x_bits(spec, seed=spec.seed + 1, permute_seed=spec.seed + 1)
+        e2_gpu = piq.layer_output_error(to_gpu_w(W), qweight, scales, to_gpu_x(X2), bits,
+                                        spec.g, g_idx=out.g_idx)
+    codes_mem = unpack_gpu(qweight, bits)
+    sc_gpu = scales.cpu().numpy().astype(np.float64)
+
+    H = O.hessian_ref(X)
+    perm, U, lam = O.gptq_prepare_ref(H, spec.damp, spec.act_order)
+    del H
+    assert np.array_equal(out.perm.cpu().numpy(), perm)
+    Wp = W.astype(np.float64)[:, perm]
+    rows = np.sort(np.random.default_rng(123).choice(W.shape[0], sample_rows, replace=False))
+    stats, c_ref, s_ref = teacher_forced_compare(codes_mem[rows][:, perm], Wp[rows], U, bits,
+                                                 spec.g)
+    s16 = s_ref.astype(np.float16).astype(np.float64)
+    assert (np.abs(sc_gpu[rows] - s16) / np.maximum(s16, 1e-30)).max() < REL_TOL
+
+    codes_all, scales_all, _ = gptq_sweep_blocked_ref(Wp, U, bits, spec.g)
+    What = dequant_ref(codes_all, scales_all, perm, spec.g)
+    e_ref = O.output_error_ref(W, What, X)
+    assert rel(out.err, e_ref) < REL_TOL, (out.err, e_ref)
+    if shift:
+        e2_ref = O.output_error_ref(W, What, X2)
+        assert rel(e2_gpu, e2_ref) < REL_TOL, (e2_gpu, e2_ref)
+    return stats
+
+
+def test_q_proj_7b_full():
+    # W 4096x4096, X 131072x4096 (lognormal channel stds, 41 channels x30),
+    # 4-bit g128; also the error on the shifted X'
+    _gptq_full(C2, shift=True)
+
+
+def test_down_proj_7b_act_order_full():
+    # W 4096x11008, X 65536x11008 Student-t(4), act-order
+    _gptq_full(C3)
+
+
+@pytest.mark.skipif(not SLOW, reason="several minutes of host float64; PIQ_FULLSIZE_SLOW=1")
+@pytest.mark.parametrize("bits", [4, 3])
+def test_down_proj_70b_full(bits):
+    # W 8192x28672, X 32768x28672, H 28672^2
+    _gptq_full(C4, bits=bits, sample_rows=16)
+
+
+@pytest.mark.skipif(not SLOW, reason="several minutes of host float64; PIQ_FULLSIZE_SLOW=1")
+def test_awq_8192_full():
+    W, X = make_weight(C5), make_x_bits(C5)
+    res = piq.awq_search_layer(to_gpu_w(W), to_gpu_x(X), C5.bits, C5.g, AWQ_GRID)
+    ref = O.awq_ref(W, X, C5.bits, C5.g, grid=list(AWQ_GRID))
+    errs = np.array(res.err_per_alpha)
+    assert (np.abs(errs - ref.err) / ref.err).max() < REL_TOL
+    srt = np.sort(ref.err)
+    if (srt[1] - srt[0]) / srt[0] >= 1e-4:
+        assert res.best_alpha == np.float32(ref.best_alpha)
