@@ -28,7 +28,7 @@ namespace piq {
 namespace {
 
 constexpr int NB = kFactorNB;  // 128
-constexpr int LDS = NB + 1;    // padded shared-memory row
+constexpr int SLD = NB + 4;    // shared-memory row stride (float4-aligned rows)
 
 __global__ void diag_mean_kernel(const float* H, int64_t in, float damp, DeviceStatus* st,
                                  float* lambda_f) {
@@ -114,31 +114,62 @@ __device__ __forceinline__ void inv16_row(const float (&a)[SP], float (&x)[SP], 
   }
 }
 
-// z[c] = sum_{k <= c} y[k] * Xd[c][k]   (row times the transposed lower inverse)
+// Forward substitution of one row against the 16 x 16 factor L11 (rows of
+// Ld, stride SLD) with the reciprocal pivots rv: on entry y = a row of A21, on
+// exit y = that row of A21 inv(L11)^T.
 template <int C>
-__device__ __forceinline__ void trsm_col(const float (&y)[SP], float (&z)[SP], const float* Xd) {
+__device__ __forceinline__ void trsm_sub(float (&y)[SP], const float* Ld, const float* rv) {
   if constexpr (C < SP) {
-    float acc = 0.f;
+    y[C] *= rv[C];
 #pragma unroll
-    for (int k = 0; k <= C; ++k) acc = fmaf(y[k], Xd[C * LDS + k], acc);
-    z[C] = acc;
-    trsm_col<C + 1>(y, z, Xd);
+    for (int c = C + 1; c < SP; ++c) y[c] = fmaf(-y[C], Ld[c * SLD + C], y[c]);
+    trsm_sub<C + 1>(y, Ld, rv);
   }
+}
+
+__device__ __forceinline__ void fma4x4(float (&acc)[4][4], const float4 a, const float4 b) {
+  const float av[4] = {a.x, a.y, a.z, a.w};
+  const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+}
+
+// Triangular index t -> (row tile bi, col tile bj), bj <= bi.
+__device__ __forceinline__ void tri_index(int t, int& bi, int& bj) {
+  int r = static_cast<int>((sqrtf(8.f * static_cast<float>(t) + 1.f) - 1.f) * 0.5f);
+  while ((r + 1) * (r + 2) / 2 <= t) ++r;
+  while (r * (r + 1) / 2 > t) --r;
+  bi = r;
+  bj = t - r * (r + 1) / 2;
 }
 
 // Factor the nb x nb diagonal block of P at (o, o) in place (lower Cholesky) and
 // write its inverse to X at (o, o) (full nb x nb, zeros above the diagonal).
 // Rows/cols >= nb are padded with the identity up to nbp = 32, 64 or 128.
+//
+// Right-looking over 16-wide sub-panels: warp 0 factors the 16 x 16 diagonal
+// block in registers (the only serial part: one pivot after the other); the
+// rows below are solved against it by substitution, one thread per row, and
+// the trailing lower triangle is updated in 4 x 4 register tiles from a
+// transposed copy of the panel (float4 loads).  The inverse is formed at the
+// end: the 16 x 16 diagonal inverses in parallel (one warp each), then pairs of
+// s-blocks merged level by level, inv([[A,0],[B,C]]) having lower-left block
+// -inv(C) B inv(A), again in 4 x 4 register tiles.
 constexpr int CI_THREADS = 512;
 constexpr int CI_WARPS = CI_THREADS / 32;
+constexpr int TLD = 64 + 4;  // merge temp row stride
 
 __global__ void __launch_bounds__(CI_THREADS)
     chol_inv_kernel(float* P, float* X, int64_t ld, int64_t o, int nb, int nbp,
                     DeviceStatus* st) {
-  extern __shared__ float sm[];
-  float* S = sm;              // [NB][LDS] factor
-  float* Xs = sm + NB * LDS;  // [NB][LDS] inverse
-  float* T = Xs + NB * LDS;   // [64][65] temp
+  extern __shared__ __align__(16) float sm[];
+  float* S = sm;                 // [NB][SLD] factor
+  float* Xs = S + NB * SLD;      // [NB][SLD] inverse
+  float* LT = Xs + NB * SLD;     // [SP][SLD] current panel, transposed
+  float* Tm = LT + SP * SLD;     // [64][TLD] merge temp
+  float* rinv = Tm + 64 * TLD;   // [NB] reciprocal pivots
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (status_bad(st)) return;
@@ -147,100 +178,170 @@ __global__ void __launch_bounds__(CI_THREADS)
   for (int i = warp; i < nbp; i += CI_WARPS) {
     for (int j = lane; j < nbp; j += 32) {
       if (i < nb && j <= i)
-        cp_async4(S + i * LDS + j, P + (o + i) * ld + (o + j));
+        cp_async4(S + i * SLD + j, P + (o + i) * ld + (o + j));
       else
-        S[i * LDS + j] = (i == j) ? 1.f : 0.f;
-      Xs[i * LDS + j] = 0.f;
+        S[i * SLD + j] = (i == j) ? 1.f : 0.f;
+      Xs[i * SLD + j] = 0.f;
     }
   }
   cp_async_wait_all();
   __syncthreads();
 
-  // right-looking over 16-wide sub-panels
   for (int c0 = 0; c0 < nbp; c0 += SP) {
+    // ---- the 16 x 16 diagonal block (warp 0)
     if (warp == 0) {
-      float a[SP], x[SP];
+      float a[SP];
       float rdiag = 0.f;
       bool ok = true;
+      if (lane < SP) {
+        const float4* row = reinterpret_cast<const float4*>(S + (c0 + lane) * SLD + c0);
 #pragma unroll
-      for (int k = 0; k < SP; ++k) a[k] = (lane < SP) ? S[(c0 + lane) * LDS + c0 + k] : 0.f;
-      chol16_col<0>(a, rdiag, lane, ok);
+        for (int q = 0; q < SP / 4; ++q) {
+          const float4 v = row[q];
+          a[4 * q] = v.x;
+          a[4 * q + 1] = v.y;
+          a[4 * q + 2] = v.z;
+          a[4 * q + 3] = v.w;
+        }
+      } else {
 #pragma unroll
-      for (int k = 0; k < SP; ++k) {
-        a[k] = (k <= lane) ? a[k] : 0.f;
-        x[k] = (k == lane) ? 1.f : 0.f;
+        for (int k = 0; k < SP; ++k) a[k] = 0.f;
       }
-      inv16_row<0>(a, x, rdiag, lane);
+      chol16_col<0>(a, rdiag, lane, ok);
       if (!ok && lane == 0) {
         bad = 1;
         set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));
       }
       if (lane < SP) {
+        float4* row = reinterpret_cast<float4*>(S + (c0 + lane) * SLD + c0);
 #pragma unroll
-        for (int k = 0; k < SP; ++k) {
-          S[(c0 + lane) * LDS + c0 + k] = a[k];
-          Xs[(c0 + lane) * LDS + c0 + k] = x[k];
-        }
+        for (int q = 0; q < SP / 4; ++q)
+          row[q] = make_float4(4 * q <= lane ? a[4 * q] : 0.f, 4 * q + 1 <= lane ? a[4 * q + 1] : 0.f,
+                               4 * q + 2 <= lane ? a[4 * q + 2] : 0.f,
+                               4 * q + 3 <= lane ? a[4 * q + 3] : 0.f);
+        rinv[c0 + lane] = rdiag;
       }
     }
     __syncthreads();
     if (bad) return;
     const int r0 = c0 + SP;
-    if (r0 < nbp) {
-      // L21 = A21 inv(L11)^T, one thread per row
+    if (r0 >= nbp) break;
+    // ---- L21 = A21 inv(L11)^T, one thread per row; also the transposed copy
+    {
       const int r = r0 + tid;
       if (r < nbp) {
-        float y[SP], z[SP];
+        float y[SP];
+        float4* row = reinterpret_cast<float4*>(S + r * SLD + c0);
 #pragma unroll
-        for (int k = 0; k < SP; ++k) y[k] = S[r * LDS + c0 + k];
-        trsm_col<0>(y, z, Xs + c0 * LDS + c0);
+        for (int q = 0; q < SP / 4; ++q) {
+          const float4 v = row[q];
+          y[4 * q] = v.x;
+          y[4 * q + 1] = v.y;
+          y[4 * q + 2] = v.z;
+          y[4 * q + 3] = v.w;
+        }
+        trsm_sub<0>(y, S + c0 * SLD + c0, rinv + c0);
 #pragma unroll
-        for (int cc = 0; cc < SP; ++cc) S[r * LDS + c0 + cc] = z[cc];
+        for (int q = 0; q < SP / 4; ++q)
+          row[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+#pragma unroll
+        for (int k = 0; k < SP; ++k) LT[k * SLD + r] = y[k];
       }
-      __syncthreads();
-      // A22 -= L21 L21^T (lower triangle), one warp per row
-      for (int i = r0 + warp; i < nbp; i += CI_WARPS) {
-        for (int j = r0 + lane; j <= i; j += 32) {
-          float acc = S[i * LDS + j];
+    }
+    __syncthreads();
+    // ---- A22 -= L21 L21^T on the lower 4 x 4 tiles
+    {
+      const int mt = (nbp - r0) / 4;
+      const int ntile = mt * (mt + 1) / 2;
+      for (int t = tid; t < ntile; t += CI_THREADS) {
+        int bi, bj;
+        tri_index(t, bi, bj);
+        const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
+        float acc[4][4] = {};
 #pragma unroll
-          for (int k = 0; k < SP; ++k)
-            acc = fmaf(-S[i * LDS + c0 + k], S[j * LDS + c0 + k], acc);
-          S[i * LDS + j] = acc;
+        for (int k = 0; k < SP; ++k)
+          fma4x4(acc, *reinterpret_cast<const float4*>(LT + k * SLD + i0),
+                 *reinterpret_cast<const float4*>(LT + k * SLD + j0));
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          float4* dst = reinterpret_cast<float4*>(S + (i0 + x) * SLD + j0);
+          float4 v = *dst;
+          v.x -= acc[x][0];
+          v.y -= acc[x][1];
+          v.z -= acc[x][2];
+          v.w -= acc[x][3];
+          *dst = v;
         }
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
 
-  // inverse of the whole block from the diagonal 16-blocks:
-  // inv([[A,0],[B,C]]) has lower-left block -inv(C) B inv(A)
-  for (int s = SP; s < nbp; s *= 2) {
-    for (int pr = 0; pr < nbp / (2 * s); ++pr) {
-      const int q0 = pr * 2 * s, q1 = q0 + s;
-      for (int i = warp; i < s; i += CI_WARPS) {  // T = B inv(A)
-        for (int j = lane; j < s; j += 32) {
-          float acc = 0.f;
-          for (int k = j; k < s; ++k)
-            acc = fmaf(S[(q1 + i) * LDS + q0 + k], Xs[(q0 + k) * LDS + q0 + j], acc);
-          T[i * 65 + j] = acc;
-        }
-      }
-      __syncthreads();
-      for (int i = warp; i < s; i += CI_WARPS) {  // X21 = -inv(C) T
-        for (int j = lane; j < s; j += 32) {
-          float acc = 0.f;
-          for (int k = 0; k <= i; ++k) acc = fmaf(Xs[(q1 + i) * LDS + q1 + k], T[k * 65 + j], acc);
-          Xs[(q1 + i) * LDS + q0 + j] = -acc;
-        }
-      }
-      __syncthreads();
+  // ---- diagonal 16 x 16 inverses, one warp each
+  for (int w = warp; w < nbp / SP; w += CI_WARPS) {
+    const int c0 = w * SP;
+    float a[SP], x[SP];
+    const float rdiag = lane < SP ? rinv[c0 + lane] : 0.f;
+#pragma unroll
+    for (int k = 0; k < SP; ++k) {
+      a[k] = (lane < SP && k <= lane) ? S[(c0 + lane) * SLD + c0 + k] : 0.f;
+      x[k] = (k == lane) ? 1.f : 0.f;
     }
+    inv16_row<0>(a, x, rdiag, lane);
+    if (lane < SP) {
+#pragma unroll
+      for (int k = 0; k < SP; ++k) Xs[(c0 + lane) * SLD + c0 + k] = x[k];
+    }
+  }
+  __syncthreads();
+
+  // ---- merges: for each pair (q0, q1 = q0 + s) at level s,
+  //      T = L[q1.., q0..] inv(L)[q0.., q0..]   then   X21 = -inv(L)[q1.., q1..] T
+  for (int s = SP; s < nbp; s *= 2) {
+    const int per = (s / 4) * (s / 4);   // 4 x 4 tiles per pair
+    const int npair = nbp / (2 * s);
+    for (int t = tid; t < per * npair; t += CI_THREADS) {
+      const int pr = t / per, u = t - pr * per;
+      const int q0 = pr * 2 * s, q1 = q0 + s;
+      const int i0 = 4 * (u / (s / 4)), j0 = 4 * (u % (s / 4));
+      float acc[4][4] = {};
+      for (int k = j0; k < s; ++k) {  // inv(L) block is lower: rows k >= j0 only
+        const float4 av = make_float4(S[(q1 + i0) * SLD + q0 + k], S[(q1 + i0 + 1) * SLD + q0 + k],
+                                      S[(q1 + i0 + 2) * SLD + q0 + k],
+                                      S[(q1 + i0 + 3) * SLD + q0 + k]);
+        fma4x4(acc, av, *reinterpret_cast<const float4*>(Xs + (q0 + k) * SLD + q0 + j0));
+      }
+      float* T = Tm + pr * s * (s + 4);
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        *reinterpret_cast<float4*>(T + (i0 + x) * (s + 4) + j0) =
+            make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+    }
+    __syncthreads();
+    for (int t = tid; t < per * npair; t += CI_THREADS) {
+      const int pr = t / per, u = t - pr * per;
+      const int q0 = pr * 2 * s, q1 = q0 + s;
+      const int i0 = 4 * (u / (s / 4)), j0 = 4 * (u % (s / 4));
+      const float* T = Tm + pr * s * (s + 4);
+      float acc[4][4] = {};
+      for (int k = 0; k <= i0 + 3; ++k) {  // inv(L) block is lower: columns k <= row
+        const float4 av =
+            make_float4(Xs[(q1 + i0) * SLD + q1 + k], Xs[(q1 + i0 + 1) * SLD + q1 + k],
+                        Xs[(q1 + i0 + 2) * SLD + q1 + k], Xs[(q1 + i0 + 3) * SLD + q1 + k]);
+        fma4x4(acc, av, *reinterpret_cast<const float4*>(T + k * (s + 4) + j0));
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        *reinterpret_cast<float4*>(Xs + (q1 + i0 + x) * SLD + q0 + j0) =
+            make_float4(-acc[x][0], -acc[x][1], -acc[x][2], -acc[x][3]);
+    }
+    __syncthreads();
   }
 
   for (int i = warp; i < nb; i += CI_WARPS) {
     for (int j = lane; j < nb; j += 32) {
-      if (j <= i) P[(o + i) * ld + (o + j)] = S[i * LDS + j];
-      X[(o + i) * ld + (o + j)] = (j <= i) ? Xs[i * LDS + j] : 0.f;
+      if (j <= i) P[(o + i) * ld + (o + j)] = S[i * SLD + j];
+      X[(o + i) * ld + (o + j)] = (j <= i) ? Xs[i * SLD + j] : 0.f;
     }
   }
 }
@@ -251,6 +352,27 @@ __global__ void extract_u_kernel(const float* X, int64_t in, float* U) {
     for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < in;
          k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
       U[i * in + k] = (k >= i) ? X[(in - 1 - i) * in + (in - 1 - k)] : 0.f;
+    }
+  }
+}
+
+// Same, four columns per thread (in % 4 == 0): U[i][k..k+3] is the float4 of
+// row in-1-i of X that starts at column in-4-k, reversed.  Only the upper part
+// of X's row is read.
+__global__ void extract_u_vec_kernel(const float* X, int64_t in, float* U) {
+  const int64_t in4 = in >> 2;
+  for (int64_t i = blockIdx.y; i < in; i += gridDim.y) {
+    const float* src = X + (in - 1 - i) * in;
+    float4* dst = reinterpret_cast<float4*>(U + i * in);
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < in4;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t k = 4 * t;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k + 3 >= i) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (in - 4 - k));
+        o = make_float4(k >= i ? v.w : 0.f, k + 1 >= i ? v.z : 0.f, k + 2 >= i ? v.y : 0.f, v.x);
+      }
+      dst[t] = o;
     }
   }
 }
@@ -291,7 +413,7 @@ __global__ void identity_perm_kernel(int64_t in, int32_t* perm, int32_t* invperm
   }
 }
 
-constexpr int kCholSmem = (2 * NB * LDS + 64 * 65) * sizeof(float);
+constexpr int kCholSmem = (2 * NB * SLD + SP * SLD + 64 * TLD + NB) * sizeof(float);
 
 // Floats of the pair scratch of the level-by-level inverse: max over levels of
 // (pairs at that level) * s * s.
@@ -385,10 +507,16 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
   }
 
   {
-    dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in, 256), 64)),
+    const bool vec = in % 4 == 0 && (reinterpret_cast<uintptr_t>(X) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(U) & 15u) == 0;
+    const int64_t cols = vec ? in / 4 : in;
+    dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(cols, 256), 64)),
               static_cast<unsigned>(std::min<int64_t>(in, 65535)));
     note_launch();
-    extract_u_kernel<<<grid, 256, 0, stream>>>(X, in, U);
+    if (vec)
+      extract_u_vec_kernel<<<grid, 256, 0, stream>>>(X, in, U);
+    else
+      extract_u_kernel<<<grid, 256, 0, stream>>>(X, in, U);
   }
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }

@@ -468,14 +468,26 @@ int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D
 
 // ------------------------------------------------ fixed-order partial reduction
 namespace {
-__global__ void reduce_partials_kernel(const double* partials, int64_t per, double* out) {
-  __shared__ double sh[256];
+constexpr int RP_THREADS = 512;
+// One block per batch entry.  Thread t sums the elements t, t + 512, ... in four
+// interleaved accumulators (so four loads are in flight), then the block folds
+// the per-thread sums in a fixed tree: the order never depends on timing.
+__global__ void __launch_bounds__(RP_THREADS)
+    reduce_partials_kernel(const double* partials, int64_t per, double* out) {
+  __shared__ double sh[RP_THREADS];
   const double* src = partials + static_cast<int64_t>(blockIdx.x) * per;
-  double acc = 0.0;
-  for (int64_t i = threadIdx.x; i < per; i += blockDim.x) acc += src[i];
-  sh[threadIdx.x] = acc;
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  int64_t i = threadIdx.x;
+  for (; i + 3 * RP_THREADS < per; i += 4 * RP_THREADS) {
+    a0 += src[i];
+    a1 += src[i + RP_THREADS];
+    a2 += src[i + 2 * RP_THREADS];
+    a3 += src[i + 3 * RP_THREADS];
+  }
+  for (; i < per; i += RP_THREADS) a0 += src[i];
+  sh[threadIdx.x] = (a0 + a1) + (a2 + a3);
   __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
+  for (int s = RP_THREADS / 2; s > 0; s >>= 1) {
     if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
     __syncthreads();
   }
@@ -487,7 +499,7 @@ int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int 
                            double* out, cudaStream_t stream) {
   const int64_t per = ceil_div(n, BM) * ceil_div(rows, BN) * 4;
   note_launch();
-  reduce_partials_kernel<<<batch, 256, 0, stream>>>(partials, per, out);
+  reduce_partials_kernel<<<batch, RP_THREADS, 0, stream>>>(partials, per, out);
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
