@@ -117,10 +117,12 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
  *   perm     device int32 [in] or NULL: memory column quantized at position p.
  *   g_idx    device int32 [in] or NULL: group of each memory-order column.
  *   out_err  host double, may be NULL: ||X W^T - X What^T||_F^2 with
- *            What = code * fp16(scale) (the layer a user reconstructs).
+ *            What = code * fp16(scale) (the layer a user reconstructs),
+ *            evaluated as sum_r D_r H D_r^T (D = W - What in fp32) from the H
+ *            of the first step: the same quantity, without a second pass over X.
  * Runs every step on the GPU: H (tensor cores), act-order, damping, blocked
  * Cholesky and triangular inverse, per-block sweep + trailing GEMM, packing,
- * output-error GEMM.  Synchronizes `stream` once at the end. */
+ * output error.  Synchronizes `stream` once at the end. */
 int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int act_order, size_t* bytes);
 int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
                         int bits, int g, float damp, int act_order, uint32_t* qweight,
@@ -158,6 +160,11 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
  * approach it"; e.g. a held-out or shifted X'):
  *   ||X W^T - X What^T||_F^2,  What[r, k] = code * fp16(scale[r, grp(k)]) / s[k]
  * grp(k) = g_idx[k] (or k / g when g_idx == NULL); s == NULL means s = 1.
+ * Two exact routes, picked from (out, in, n) alone so the workspace size is
+ * fixed by them: directly, a BF16 tensor-core product X D^T (D = W - What
+ * rounded to bf16) squared and summed; or, when n is large against out and in
+ * (n in + 6 out in < 2 n out), through H = X^T X as sum_r D_r H D_r^T with D
+ * in fp32 (FP32-accurate tensor-core GEMM).
  * All pointers device except out_err (host).  Synchronizes `stream`. */
 int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t* bytes);
 int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32_t* qweight,

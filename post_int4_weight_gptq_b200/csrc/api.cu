@@ -163,13 +163,14 @@ SweepWs carve_sweep(Carver& c, int64_t out, int64_t in) {
 
 struct GptqWs {
   DeviceStatus* st;
-  float* H;  // becomes U
-  float* fwork;
-  float* Wq;
+  float* H;      // X^T X, kept for the output error
+  float* fwork;  // factor scratch; U is written over its first in * in floats, then
+                 // the error's bf16 split of H goes after it
+  float* Wq;     // sweep copy of W; later the error's bf16 split of D
   float* Err;
   int8_t* codes;
   float* qscale;
-  uint16_t* dW;
+  float* dW;     // W - What (fp32, memory order)
   int32_t* perm;
   int32_t* invperm;
   double* colpart;
@@ -186,12 +187,12 @@ GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int act_order) 
   w.Err = c.take<float>(out * kSweepB);
   w.codes = c.take<int8_t>(out * in);
   w.qscale = c.take<float>(out * ceil_div(in, 1));  // sized for g >= 1
-  w.dW = c.take<uint16_t>(out * in);
+  w.dW = c.take<float>(out * in);
   w.perm = c.take<int32_t>(in);
   w.invperm = c.take<int32_t>(in);
   w.colpart = c.take<double>(act_order ? static_cast<int64_t>(colstats_splits(n, in)) * in * 2 : 1);
   w.sumsq = c.take<double>(in);
-  w.partials = c.take<double>(sumsq_partials_count(n, out, 1));
+  w.partials = c.take<double>(err_via_h_partials(out, in));
   w.err = c.take<double>(1);
   return w;
 }
@@ -238,17 +239,38 @@ RtnWs carve_rtn(Carver& c, int64_t out, int64_t in) {
   return w;
 }
 
+// Route of piq_layer_output_error, in BF16 tensor-core flops: through X,
+// 2 n in out; through H, n in^2 for X^T X plus three bf16 passes over the
+// triangular out x in x in product, 3 out in^2.
+bool error_route_h(int64_t out, int64_t in, int64_t n) {
+  const double via_x = 2.0 * n * in * out;
+  const double via_h = static_cast<double>(n) * in * in + 3.0 * out * in * in;
+  return via_h < via_x;
+}
+
 struct ErrWs {
   DeviceStatus* st;
-  uint16_t* dW;
+  uint16_t* dW;      // X route: bf16 delta
+  float* dW32;       // H route: fp32 delta, H and the bf16 splits
+  float* H;
+  uint16_t* dsplit;
+  uint16_t* hsplit;
   double* partials;
   double* err;
 };
 ErrWs carve_err(Carver& c, int64_t out, int64_t in, int64_t n) {
-  ErrWs w;
+  ErrWs w{};
   w.st = c.take<DeviceStatus>(1);
-  w.dW = c.take<uint16_t>(out * in);
-  w.partials = c.take<double>(sumsq_partials_count(n, out, 1));
+  if (error_route_h(out, in, n)) {
+    w.dW32 = c.take<float>(out * in);
+    w.H = c.take<float>(in * in);
+    w.dsplit = c.take<uint16_t>(2 * out * in);
+    w.hsplit = c.take<uint16_t>(2 * in * in);
+    w.partials = c.take<double>(err_via_h_partials(out, in));
+  } else {
+    w.dW = c.take<uint16_t>(out * in);
+    w.partials = c.take<double>(sumsq_partials_count(n, out, 1));
+  }
   w.err = c.take<double>(1);
   return w;
 }
@@ -394,22 +416,24 @@ int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t*
       PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
   }
   clk.mark();
-  // 3. damping + U (written over H)
-  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, w.H, w.fwork, w.st, s));
+  // 3. damping + U (H is kept; U goes over the factor's own scratch)
+  float* U = w.fwork;
+  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, U, w.fwork, w.st, s));
   clk.mark();
   // 4. blocked sweep on the permuted copy
   PIQ_TRY(launch_gather_columns(W, out, in, qperm, w.Wq, s));
-  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, w.H, bits, g, w.codes, w.qscale, w.Err, w.st, s));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, w.Err, w.st, s));
   clk.mark();
   // 5. pack (+ D = W - What for the error)
-  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, qweight, scales,
+  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, qweight, scales, nullptr,
                       out_err ? w.dW : nullptr, g_idx, s));
   clk.mark();
-  // 6. output error
-  if (out_err) {
-    PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
-    PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));
-  }
+  // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from the H built in step 1
+  //    (scratch: the sweep copy, and the factor's inverse region after U)
+  if (out_err)
+    PIQ_TRY(run_error_via_h(w.dW, out, in, w.H, reinterpret_cast<uint16_t*>(w.Wq),
+                            reinterpret_cast<uint16_t*>(w.fwork + in * in), w.partials, w.err,
+                            w.st, s));
   clk.mark();
   double e = 0.0;
   if (out_err)
@@ -468,7 +492,7 @@ int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
   PIQ_TRY(launch_argmin(w.err, n_alpha, w.alphas, w.best, w.best_alpha, s));
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, w.s_table, w.best, w.codes, w.qscale, s_out, s));
   PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
-                      nullptr, nullptr, s));
+                      nullptr, nullptr, nullptr, s));
   clk.mark();
   double errs[64];
   float ba = 0.f;
@@ -506,7 +530,7 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
   RtnWs w = carve_rtn(c, out, in);
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, nullptr, nullptr, w.codes, w.qscale, nullptr, s));
   return launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
-                     nullptr, nullptr, s);
+                     nullptr, nullptr, nullptr, s);
 }
 
 int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t* bytes) {
@@ -534,9 +558,18 @@ int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32
   Carver c(workspace);
   ErrWs w = carve_err(c, out, in, n);
   PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
-  PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, w.dW, w.st, s));
-  PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
-  PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));
+  if (error_route_h(out, in, n)) {
+    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, nullptr,
+                                 w.dW32, w.st, s));
+    PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
+    PIQ_TRY(run_error_via_h(w.dW32, out, in, w.H, w.dsplit, w.hsplit, w.partials, w.err, w.st,
+                            s));
+  } else {
+    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, w.dW,
+                                 nullptr, w.st, s));
+    PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
+    PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));
+  }
   double e = 0.0;
   PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
   const int rc = finish_call(w.st, s, nullptr);

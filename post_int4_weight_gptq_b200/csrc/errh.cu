@@ -1,0 +1,109 @@
+// Layer output error through the Hessian: for D = W - What,
+//   ||X D^T||_F^2 = sum_r D_r (X^T X) D_r^T = 2 sum_r D_r Hu D_r^T,
+// where Hu is the upper triangle of H = X^T X with its diagonal halved (the
+// shared objective of "GPTQ versus AWQ objectives", section "How to approach
+// it", with the proxy Hessian of the listing under "A strong answer").  The
+// identity is exact; it replaces a 2 n in out contraction by an out x in x in
+// one, which is much smaller when n >> out, and GPTQ has H already.
+//
+//   1. D (fp32) and Hu (from the upper triangle of H) split into bf16 pairs,
+//      x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): 16 significant bits
+//   2. one tensor-core launch accumulates D Hu as hi.hi + hi.lo + lo.hi (the
+//      dropped lo.lo is ~2^-16 of each product) and multiplies the product
+//      tile by D in its epilogue; column tiles skip the zero triangle of Hu
+//   3. fixed-order FP64 reduction of the per-tile partial sums
+#include "internal.h"
+
+namespace piq {
+
+namespace {
+
+__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+  hi = float_to_bf16_bits(x);
+  lo = float_to_bf16_bits(x - bf16_bits_to_float(hi));
+}
+
+// D [count] fp32 -> hi, lo (count % 4 == 0).
+__global__ void split_vec_kernel(const float4* __restrict__ d, int64_t n4, uint2* __restrict__ hi,
+                                 uint2* __restrict__ lo) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = d[i];
+    uint16_t h[4], l[4];
+    split_bf16(v.x, h[0], l[0]);
+    split_bf16(v.y, h[1], l[1]);
+    split_bf16(v.z, h[2], l[2]);
+    split_bf16(v.w, h[3], l[3]);
+    hi[i] = make_uint2(h[0] | (static_cast<uint32_t>(h[1]) << 16),
+                       h[2] | (static_cast<uint32_t>(h[3]) << 16));
+    lo[i] = make_uint2(l[0] | (static_cast<uint32_t>(l[1]) << 16),
+                       l[2] | (static_cast<uint32_t>(l[3]) << 16));
+  }
+}
+
+// Hu[k][j] = H[k][j] (k < j), H[k][k] / 2, 0 (k > j), split; in % 4 == 0.
+__global__ void split_upper_half_kernel(const float* __restrict__ H, int64_t in,
+                                        uint2* __restrict__ hi, uint2* __restrict__ lo) {
+  const int64_t in4 = in >> 2;
+  for (int64_t k = blockIdx.y; k < in; k += gridDim.y) {
+    const float4* row = reinterpret_cast<const float4*>(H + k * in);
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < in4;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t j = 4 * t;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j + 3 >= k) {  // some column on or above the diagonal
+        const float4 x = row[t];
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          v[e] = (j + e > k) ? xs[e] : (j + e == k ? 0.5f * xs[e] : 0.f);
+      }
+      uint16_t h[4], l[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) split_bf16(v[e], h[e], l[e]);
+      hi[k * in4 + t] = make_uint2(h[0] | (static_cast<uint32_t>(h[1]) << 16),
+                                   h[2] | (static_cast<uint32_t>(h[3]) << 16));
+      lo[k * in4 + t] = make_uint2(l[0] | (static_cast<uint32_t>(l[1]) << 16),
+                                   l[2] | (static_cast<uint32_t>(l[3]) << 16));
+    }
+  }
+}
+
+unsigned grid_1d(int64_t work) {
+  DeviceInfo info;
+  const int sms = device_info(&info) == PIQ_OK ? info.sm_count : 148;
+  return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(work, 256),
+                                                                      static_cast<int64_t>(sms) * 8)));
+}
+
+}  // namespace
+
+int64_t err_via_h_partials(int64_t out, int64_t in) { return err_dot_partials_count(out, in); }
+
+int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uint16_t* dsplit,
+                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                    cudaStream_t stream) {
+  if (out < 1 || in < 8 || in % 8 != 0) return PIQ_ERR_INVALID_ARG;
+  uint16_t* d_hi = dsplit;
+  uint16_t* d_lo = dsplit + out * in;
+  uint16_t* h_hi = hsplit;
+  uint16_t* h_lo = hsplit + in * in;
+  note_launch();
+  split_vec_kernel<<<grid_1d(out * in / 4), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(D), out * in / 4, reinterpret_cast<uint2*>(d_hi),
+      reinterpret_cast<uint2*>(d_lo));
+  if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+  {
+    dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in / 4, 256), 16)),
+              static_cast<unsigned>(std::min<int64_t>(in, 65535)));
+    note_launch();
+    split_upper_half_kernel<<<grid, 256, 0, stream>>>(H, in, reinterpret_cast<uint2*>(h_hi),
+                                                      reinterpret_cast<uint2*>(h_lo));
+    if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+  }
+  int rc = launch_err_dot(d_hi, d_lo, h_hi, h_lo, D, out, in, partials, st, stream);
+  if (rc != PIQ_OK) return rc;
+  return launch_reduce_sum(partials, err_dot_partials_count(out, in), 1, err, stream);
+}
+
+}  // namespace piq

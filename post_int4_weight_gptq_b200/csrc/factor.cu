@@ -71,15 +71,17 @@ __global__ void build_rev_kernel(const float* H, int64_t in, const int32_t* perm
 constexpr int SP = 16;  // sub-panel width inside a 128 block
 constexpr unsigned FULL = 0xffffffffu;
 
-// One warp factors a 16 x 16 SPD block and inverts its factor, in registers.
-// Lane i < 16 holds row i: on entry a[k] = A[i][k] (k <= i); on exit a[k] =
-// L[i][k] and x[k] = inv(L)[i][k] (0 above the diagonal).  Lanes >= 16 carry
-// zeros.  Template recursion keeps register indices compile-time; the code is
-// small enough for the instruction cache.
+// One warp factors a 16 x 16 SPD block, in registers.  Lane i < 16 holds row
+// i: on entry a[k] = A[i][k] (k <= i); on exit a[k] = L[i][k] (k <= i) and
+// rdiag = 1 / L_ii.  Lanes >= 16 carry zeros.  d is pivot J, already
+// broadcast; the next pivot is formed by lane J+1 from its own values and
+// broadcast before the rest of the column update, so the serial chain per
+// pivot is one shuffle, one rsqrt, one multiply and one FMA.  Template
+// recursion keeps register indices compile-time.
 template <int J>
-__device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lane, bool& ok) {
+__device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lane, bool& ok,
+                                           float d) {
   if constexpr (J < SP) {
-    const float d = __shfl_sync(FULL, a[J], J);
     ok = ok && (d > 0.f);
     const float dd = d > 0.f ? d : 1.f;
     const float r = rsqrtf(dd);  // 1 / L_JJ
@@ -87,12 +89,14 @@ __device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lan
     if (lane == J) rdiag = r;
     const float lij = (lane > J) ? a[J] * r : (lane == J ? ljj : 0.f);
     a[J] = lij;
+    float dn = 0.f;
+    if constexpr (J + 1 < SP) dn = __shfl_sync(FULL, fmaf(-lij, lij, a[J + 1]), J + 1);
 #pragma unroll
     for (int k = J + 1; k < SP; ++k) {
       const float lkj = __shfl_sync(FULL, lij, k);
       if (k <= lane) a[k] = fmaf(-lij, lkj, a[k]);
     }
-    chol16_col<J + 1>(a, rdiag, lane, ok);
+    chol16_col<J + 1>(a, rdiag, lane, ok, dn);
   }
 }
 
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(CI_THREADS)
 #pragma unroll
         for (int k = 0; k < SP; ++k) a[k] = 0.f;
       }
-      chol16_col<0>(a, rdiag, lane, ok);
+      chol16_col<0>(a, rdiag, lane, ok, __shfl_sync(FULL, a[0], 0));
       if (!ok && lane == 0) {
         bad = 1;
         set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));

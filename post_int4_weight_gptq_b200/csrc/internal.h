@@ -31,11 +31,33 @@ int64_t sumsq_partials_count(int64_t n, int64_t rows, int batch);
 // Fixed-order sum of the partials of each batch entry into out[batch].
 int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,
                            double* out, cudaStream_t stream);
+// out[b] = fixed-order sum of partials[b * per .. (b + 1) * per).
+int launch_reduce_sum(const double* partials, int64_t per, int batch, double* out,
+                      cudaStream_t stream);
+
+// E = 2 sum_r D_r Hu D_r^T from bf16 hi/lo pairs (tc_gemm.cu): D_hi, D_lo [out][in],
+// Hu_hi, Hu_lo [in][in] (Hu = upper triangle of H, diagonal halved), D fp32 [out][in].
+// Writes err_dot_partials_count(out, in) doubles.
+int launch_err_dot(const uint16_t* D_hi, const uint16_t* D_lo, const uint16_t* Hu_hi,
+                   const uint16_t* Hu_lo, const float* D, int64_t out, int64_t in,
+                   double* partials, DeviceStatus* st, cudaStream_t stream);
+int64_t err_dot_partials_count(int64_t out, int64_t in);
+
+// ------------------------------------------ output error through H (errh.cu)
+// err = ||X D^T||_F^2 = 2 sum_r D_r Hu D_r^T with D [out, in] fp32 and H = X^T X
+// (upper triangle read).  Scratch: dsplit 2 out in, hsplit 2 in in bf16;
+// partials err_via_h_partials(out, in) doubles.
+int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uint16_t* dsplit,
+                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                    cudaStream_t stream);
+int64_t err_via_h_partials(int64_t out, int64_t in);
 
 // ------------------------------------------------------ FP32 SIMT GEMM (simt_gemm.cu)
 // C = alpha * A * op(B) + beta * C, row-major; op(B) = B or B^T (trans_b).
 // mode 0: plain; 1: only tiles touching the lower triangle of C (M == N);
-// 2: A lower triangular (entries right of the diagonal are skipped per row tile).
+// 2: A lower triangular (entries right of the diagonal are skipped per row tile);
+// 3: op(B)[k][n] = 0 for k > n (k stops at the column tile's end);
+// 4: op(B)[k][n] = 0 for k < n (k starts at the column tile's start).
 // Batching over blockIdx.z: entry z uses A + z*stride_a (and B, C alike); with
 // m_total > 0 entry z has min(M, m_total - z*m_step) rows, and K the same when
 // k_follows_m (a square triangular A).
@@ -65,6 +87,8 @@ int launch_gemm_f32(int M, int N, int K, float alpha, const float* A, int64_t ld
 // ------------------------------------------------------------- factor (factor.cu)
 constexpr int kFactorNB = 128;  // panel width of the blocked Cholesky / inverse
 int64_t factor_workspace_floats(int64_t in);  // P + Dinv + T
+// U may be `work` itself: U is written last, from the inverse, when the first
+// in * in floats of work (P) are no longer read.  H is only read.
 int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm, float* U,
                      float* work, DeviceStatus* st, cudaStream_t stream);
 int launch_act_order_perm(const double* sumsq, int64_t in, int32_t* perm, int32_t* invperm,
@@ -84,9 +108,11 @@ int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, 
 int colstats_splits(int64_t n, int64_t in);
 int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
                           float* Wq, cudaStream_t stream);
+// dW (bf16) and dW32 (fp32), when given, receive W0 - code * fp16(scale).
 int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
                 int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
-                uint16_t* scales16, uint16_t* dW, int32_t* g_idx, cudaStream_t stream);
+                uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
+                cudaStream_t stream);
 int launch_awq_scale_table(const double* mean_abs, int64_t in, const float* alphas_dev,
                            int n_alpha, float* s_table, cudaStream_t stream);
 int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,
@@ -96,9 +122,10 @@ int launch_group_quant(const float* W, int64_t out, int64_t in, int bits, int g,
                        float* s_out, cudaStream_t stream);
 int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_idx,
                   float* best_alpha, cudaStream_t stream);
+// W - What from a packed layer, into dW (bf16) or dW32 (fp32), whichever is given.
 int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
                          const uint16_t* scales16, const int32_t* g_idx, const float* s,
-                         int bits, int g, uint16_t* dW, DeviceStatus* st,
+                         int bits, int g, uint16_t* dW, float* dW32, DeviceStatus* st,
                          cudaStream_t stream);
 
 }  // namespace piq

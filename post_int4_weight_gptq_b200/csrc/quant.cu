@@ -20,14 +20,6 @@ namespace piq {
 
 namespace {
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
-__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
-  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
-}
-
 // ------------------------------------------------------------------- colstats
 // grid (ceil(in/256), splits); 8 warps; lane owns 8 consecutive columns.
 __global__ void __launch_bounds__(256) colstats_kernel(const uint16_t* __restrict__ X, int64_t n,
@@ -108,7 +100,8 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
                             const int32_t* __restrict__ invperm, int64_t out, int64_t in,
                             int bits, int g, const float* __restrict__ W0,
                             uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales16,
-                            uint16_t* __restrict__ dW, int32_t* __restrict__ g_idx) {
+                            uint16_t* __restrict__ dW, float* __restrict__ dW32,
+                            int32_t* __restrict__ g_idx) {
   const int64_t words = in / 8;
   const int64_t ngroups = (in + g - 1) / g;
   const int64_t total = out * words;
@@ -119,9 +112,10 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
     const int8_t* crow = codes + r * in;
     const float* srow = qscale + r * ngroups;
     uint32_t word = 0;
-    uint16_t d16[8];
+    float d32[8];
     float w0[8];
-    if (dW) {
+    const bool delta = dW != nullptr || dW32 != nullptr;
+    if (delta) {
       const float4 a = *reinterpret_cast<const float4*>(W0 + r * in + wd * 8);
       const float4 b = *reinterpret_cast<const float4*>(W0 + r * in + wd * 8 + 4);
       w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w;
@@ -133,13 +127,21 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
       const int64_t p = invperm ? invperm[c] : c;
       const int code = crow[p];
       word |= static_cast<uint32_t>(code + off) << (4 * k);
-      if (dW) {
+      if (delta) {
         const float s16 = __half2float(__float2half_rn(srow[p / g]));
-        d16[k] = float_to_bf16_bits(w0[k] - static_cast<float>(code) * s16);
+        d32[k] = w0[k] - static_cast<float>(code) * s16;
       }
     }
     qweight[idx] = word;
+    if (dW32) {
+      float4* dst = reinterpret_cast<float4*>(dW32 + r * in + wd * 8);
+      dst[0] = make_float4(d32[0], d32[1], d32[2], d32[3]);
+      dst[1] = make_float4(d32[4], d32[5], d32[6], d32[7]);
+    }
     if (dW) {
+      uint16_t d16[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) d16[k] = float_to_bf16_bits(d32[k]);
       uint4 o;
       o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
       o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
@@ -316,7 +318,8 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
                                      const uint16_t* __restrict__ scales16,
                                      const int32_t* __restrict__ g_idx,
                                      const float* __restrict__ s, int bits, int g,
-                                     uint16_t* __restrict__ dW, DeviceStatus* st) {
+                                     uint16_t* __restrict__ dW, float* __restrict__ dW32,
+                                     DeviceStatus* st) {
   const int64_t words = in / 8;
   const int64_t ngroups = (in + g - 1) / g;
   const int off = 1 << (bits - 1);
@@ -324,7 +327,7 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
        idx < out * words; idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = idx / words, wd = idx - r * words;
     const uint32_t word = qweight[idx];
-    uint16_t d16[8];
+    float d32[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int64_t c = wd * 8 + k;
@@ -337,8 +340,17 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
       const float sc = __half2float(__ushort_as_half(scales16[r * ngroups + grp]));
       float what = static_cast<float>(code) * sc;
       if (s) what = __fdiv_rn(what, s[c]);
-      d16[k] = float_to_bf16_bits(W[r * in + c] - what);
+      d32[k] = W[r * in + c] - what;
     }
+    if (dW32) {
+      float4* dst = reinterpret_cast<float4*>(dW32 + r * in + wd * 8);
+      dst[0] = make_float4(d32[0], d32[1], d32[2], d32[3]);
+      dst[1] = make_float4(d32[4], d32[5], d32[6], d32[7]);
+      continue;
+    }
+    uint16_t d16[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) d16[k] = float_to_bf16_bits(d32[k]);
     uint4 o;
     o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
     o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
@@ -387,10 +399,12 @@ int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t
 
 int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
                 int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
-                uint16_t* scales16, uint16_t* dW, int32_t* g_idx, cudaStream_t stream) {
+                uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
+                cudaStream_t stream) {
+  if ((dW != nullptr || dW32 != nullptr) && W0 == nullptr) return PIQ_ERR_INVALID_ARG;
   note_launch();
   pack_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
-      codes, qscale, invperm, out, in, bits, g, W0, qweight, scales16, dW, g_idx);
+      codes, qscale, invperm, out, in, bits, g, W0, qweight, scales16, dW, dW32, g_idx);
   return last_error();
 }
 
@@ -435,11 +449,12 @@ int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_i
 
 int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
                          const uint16_t* scales16, const int32_t* g_idx, const float* s,
-                         int bits, int g, uint16_t* dW, DeviceStatus* st,
+                         int bits, int g, uint16_t* dW, float* dW32, DeviceStatus* st,
                          cudaStream_t stream) {
+  if ((dW == nullptr) == (dW32 == nullptr)) return PIQ_ERR_INVALID_ARG;
   note_launch();
   dequant_delta_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
-      W, out, in, qweight, scales16, g_idx, s, bits, g, dW, st);
+      W, out, in, qweight, scales16, g_idx, s, bits, g, dW, dW32, st);
   return last_error();
 }
 

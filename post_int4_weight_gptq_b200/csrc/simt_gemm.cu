@@ -37,8 +37,8 @@ __global__ void __launch_bounds__(256)
     if (bt.k_follows_m) K = M;
     if (M <= 0 || m0 >= M) return;
   }
-  // K range that can be nonzero: mode 2, A lower (k <= row); mode 3, B lower
-  // used transposed (k <= col); mode 4, B lower used as is (k >= col)
+  // K range that can be nonzero: mode 2, A lower (k <= row); mode 3, op(B)
+  // upper (k <= col); mode 4, op(B) lower (k >= col)
   const int kend = (MODE == 2) ? min(K, m0 + TM) : (MODE == 3) ? min(K, n0 + TN) : K;
   const int kbeg = (MODE == 4) ? min(K, n0) & ~(TK - 1) : 0;
 
@@ -169,6 +169,7 @@ int launch_simt_gemm(int M, int N, int K, float alpha, const float* A, int64_t l
   PIQ_GEMM_CASE(true, 3)
   PIQ_GEMM_CASE(false, 0)
   PIQ_GEMM_CASE(false, 2)
+  PIQ_GEMM_CASE(false, 3)
   PIQ_GEMM_CASE(false, 4)
 #undef PIQ_GEMM_CASE
   return PIQ_ERR_INVALID_ARG;

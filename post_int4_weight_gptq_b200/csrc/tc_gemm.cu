@@ -7,22 +7,30 @@
 //                row-major, so both operands are MN-major tiles (the sample
 //                index n is the contraction).  Only tiles touching the upper
 //                triangle are computed.  The sample range is cut into chunks of
-//                KC samples: each chunk's fp32 tile leaves TMEM and is added into
-//                H by a TMA reduce (the first chunk stores), one chunk after the
-//                other by the CTA that owns the tile, so the sum is deterministic
-//                and the tensor-core accumulation error grows with KC rather
-//                than with n.
+//                KC samples: each chunk's fp32 tile leaves TMEM and is added to
+//                a running sum held in the epilogue threads' registers, in chunk
+//                order, so the sum is deterministic and the tensor-core
+//                accumulation error grows with KC rather than with n.
 //   * err_sumsq  E_b = ||X D_b^T||_F^2 for stacked D_b (D = W - What), the
 //                shared objective of both methods ("How to approach it").  Both
 //                operands are K-major; the epilogue squares and sums the
 //                accumulator straight out of TMEM, so the [n, out] product
-//                never reaches memory.  One double per tile, reduced later in a
-//                fixed order (deterministic).
+//                never reaches memory.
+//   * err_dot    E = 2 sum_r D_r Hu D_r^T (the same objective through H, Hu the
+//                upper triangle of H with its diagonal halved), with D and Hu
+//                split into bf16 pairs x = hi + lo and the product accumulated
+//                as hi.hi + hi.lo + lo.hi: three K segments of one launch.  The
+//                epilogue multiplies the product tile by D (fp32) and sums, so
+//                D Hu never reaches memory either.  Column tiles stop their k
+//                range at the tile's end (Hu[k][j] = 0 for k > j).
+// Partial sums (err_sumsq, err_dot) are one double per (tile, epilogue warp),
+// reduced later in a fixed order: results are deterministic.
 //
-// Warp roles (192 threads): warp 0 lane 0 issues TMA loads into a 4-stage
-// ring; warp 1 lane 0 issues the MMAs and commits; warps 2..5 drain one of two
-// 256-column accumulators while the MMA warp fills the other.  Every wait is
-// bounded (common.cuh); no multicast loads are used.
+// Warp roles (320 threads): warp 0 lane 0 issues TMA loads into a 4-stage
+// ring; warp 1 lane 0 issues the MMAs and commits; warps 2..9 drain one of two
+// 256-column accumulators while the MMA warp fills the other (warp w reads TMEM
+// lanes 32 (w % 4) .. and columns 128 ((w - 2) / 4) ..).  Every wait is bounded
+// (common.cuh); no multicast loads are used.
 #include <cuda.h>
 
 #include <mutex>
@@ -40,23 +48,18 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
 constexpr int GROUP_M = 16;                     // raster group (err_sumsq)
-// Samples per TMEM accumulation before the tile is flushed into H.  The
-// relative error of the tensor-core fp32 sum grows about linearly with the
-// number of MMAs accumulated in place; 4096 samples (256 MMAs of k = 16) keep
-// it near 2e-5 of sqrt(H_ii H_jj) whatever n is.
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// Samples per TMEM accumulation of H.  The relative error of the tensor-core
+// fp32 sum grows about linearly with the number of MMAs accumulated in place;
+// 4096 samples (256 MMAs of k = 16) keep it near 2e-5 of sqrt(H_ii H_jj)
+// whatever n is.
 constexpr int KC = 4096;
-constexpr int STG_BYTES = 4 * 2 * 32 * 32 * 4;  // H epilogue: two 32x32 fp32 slabs per warp
 
-enum { EPI_STORE_UPPER = 0, EPI_SUMSQ = 1 };
-
-template <int EPI>
-constexpr int smem_bytes() {
-  return STAGES * STAGE_BYTES + (EPI == EPI_STORE_UPPER ? STG_BYTES : 0) + 1024 /*align*/ +
-         256 /*barriers*/;
-}
+enum { EPI_SYRK = 0, EPI_SUMSQ = 1, EPI_DOT = 2 };
 
 struct Params {
   int M, N, K;
@@ -65,7 +68,9 @@ struct Params {
   float* C;
   int64_t ldc;
   int accumulate;
-  int kb_chunk;  // k blocks per accumulation chunk (>= number of k blocks: one chunk)
+  int kb_chunk;  // k blocks per accumulation chunk (>= a tile's k blocks: one chunk)
+  const float* D;  // err_dot: D [M][K] fp32, row stride ldd
+  int64_t ldd;
   double* partials;
   DeviceStatus* st;
 };
@@ -73,10 +78,10 @@ struct Params {
 // Tile t -> (m tile, n tile, batch entry).
 template <int EPI>
 __device__ __forceinline__ void decode_tile(const Params& p, int t, int& mt, int& nt, int& bz) {
-  if (EPI == EPI_STORE_UPPER) {
+  bz = 0;
+  if (EPI == EPI_SYRK) {
     // n-panel b holds m tiles a with a*BM < (b+1)*BN (they touch j >= i).
     int acc = 0;
-    bz = 0;
     for (int b = 0; b < p.n_tiles; ++b) {
       int cnt = min(p.m_tiles, (int)(((int64_t)(b + 1) * BN + BM - 1) / BM));
       if (t < acc + cnt) {
@@ -87,6 +92,10 @@ __device__ __forceinline__ void decode_tile(const Params& p, int t, int& mt, int
       acc += cnt;
     }
     mt = nt = 0;
+  } else if (EPI == EPI_DOT) {
+    // longest k ranges (last column tiles) first, so the round robin balances
+    nt = p.n_tiles - 1 - t / p.m_tiles;
+    mt = t - (p.n_tiles - 1 - nt) * p.m_tiles;
   } else {
     const int per = p.m_tiles * p.n_tiles;
     bz = t / per;
@@ -100,17 +109,27 @@ __device__ __forceinline__ void decode_tile(const Params& p, int t, int& mt, int
   }
 }
 
+// k blocks of a K segment for column tile nt (err_dot: k < (nt + 1) BN only).
+template <int EPI>
+__device__ __forceinline__ int seg_kblocks(const Params& p, int nt, int num_kb) {
+  if (EPI != EPI_DOT) return num_kb;
+  return min(num_kb, (int)(((int64_t)(nt + 1) * BN + BK - 1) / BK));
+}
+template <int EPI>
+constexpr int n_segments() {
+  return EPI == EPI_DOT ? 3 : 1;
+}
+
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, Params p) {
+                   const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmB2, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* stg_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // H epilogue only
-  uint64_t* full = reinterpret_cast<uint64_t*>(
-      smem + STAGES * STAGE_BYTES + (EPI == EPI_STORE_UPPER ? STG_BYTES : 0));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
@@ -128,12 +147,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], EPI_WARPS);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI == EPI_STORE_UPPER) tma_prefetch_desc(&tmC);
+    if (EPI == EPI_DOT) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -144,7 +166,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (p.K + BK - 1) / BK;
-  const int n_chunks = num_kb <= p.kb_chunk ? 1 : 1 + (num_kb - 1) / p.kb_chunk;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -155,7 +176,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         int mt, nt, bz;
         decode_tile<EPI>(p, t, mt, nt, bz);
         const int m0 = mt * BM, n0 = nt * BN;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int L = seg_kblocks<EPI>(p, nt, num_kb);
+        for (int j = 0; j < n_segments<EPI>() * L && ok; ++j, ++it) {
+          const int seg = j / L, kb = j - seg * L;
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, p.st, 1)) {
@@ -166,17 +189,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           const int k0 = kb * BK;
+          // err_dot segments: A = D_hi, D_hi, D_lo;  B = Hu_hi, Hu_lo, Hu_hi
+          const CUtensorMap* ma = (EPI == EPI_DOT && seg == 2) ? &tmA2 : &tmA;
+          const CUtensorMap* mb = (EPI == EPI_DOT && seg == 1) ? &tmB2 : &tmB;
           if (A_MN) {
-            tma_load_2d(sa, &tmA, &full[s], m0, k0);
-            tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, k0);
+            tma_load_2d(sa, ma, &full[s], m0, k0);
+            tma_load_2d(sa + 8192, ma, &full[s], m0 + 64, k0);
           } else {
-            tma_load_2d(sa, &tmA, &full[s], k0, m0);
+            tma_load_2d(sa, ma, &full[s], k0, m0);
           }
           if (B_MN) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tma_load_2d(sb + c * 8192, &tmB, &full[s], n0 + 64 * c, k0);
+            for (int c = 0; c < 4; ++c) tma_load_2d(sb + c * 8192, mb, &full[s], n0 + 64 * c, k0);
           } else {
-            tma_load_3d(sb, &tmB, &full[s], k0, n0, bz);
+            tma_load_3d(sb, mb, &full[s], k0, n0, bz);
           }
         }
       }
@@ -189,6 +215,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       int lt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mt, nt, bz;
+        decode_tile<EPI>(p, t, mt, nt, bz);
+        const int nkb = n_segments<EPI>() * seg_kblocks<EPI>(p, nt, num_kb);
+        const int n_chunks = nkb <= p.kb_chunk ? 1 : 1 + (nkb - 1) / p.kb_chunk;
         for (int ch = 0; ch < n_chunks && ok; ++ch, ++lt) {
           const int buf = lt & 1;
           const uint32_t use = static_cast<uint32_t>(lt >> 1);
@@ -199,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
           const int kb0 = ch * p.kb_chunk;
-          const int kb1 = num_kb - kb0 <= p.kb_chunk ? num_kb : kb0 + p.kb_chunk;
+          const int kb1 = nkb - kb0 <= p.kb_chunk ? nkb : kb0 + p.kb_chunk;
           for (int kb = kb0; kb < kb1; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
@@ -226,91 +256,123 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int h = (warp - 2) >> 2;          // column half of the accumulator
+    const int slot = warp - 2;              // partial-sum slot of this warp
     int lt = 0;
-    if (EPI == EPI_SUMSQ) {
-      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      int mt, nt, bz;
+      decode_tile<EPI>(p, t, mt, nt, bz);
+      const int row0 = mt * BM + q * 32;
+      const int colh = nt * BN + h * 128;
+      const int nkb = n_segments<EPI>() * seg_kblocks<EPI>(p, nt, num_kb);
+      const int n_chunks = nkb <= p.kb_chunk ? 1 : 1 + (nkb - 1) / p.kb_chunk;
+      float sum[EPI == EPI_SYRK ? 128 : 1];
+      if (EPI == EPI_SYRK) {
+#pragma unroll
+        for (int i = 0; i < (EPI == EPI_SYRK ? 128 : 1); ++i) sum[i] = 0.f;
+      }
+      double acc = 0.0;
+      for (int ch = 0; ch < n_chunks; ++ch, ++lt) {
         const int buf = lt & 1;
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
-        if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) break;
+        if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
-        double acc = 0.0;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v);
-          float s = 0.f;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(buf * BN + h * 128);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s = fmaf(v[i], v[i], s);
-          acc += static_cast<double>(s);
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = colh + c * 32;
+          if (EPI == EPI_SYRK) {
+            // slabs wholly below the diagonal, or outside H, are never stored
+            if (row0 >= p.M || col0 >= p.N || col0 + 32 <= row0) continue;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float v[16];
+              tmem_ld_32x32b_x16(taddr + c * 32 + hh * 16, v);  // lane = row, v[i] = column
+#pragma unroll
+              for (int i = 0; i < 16; ++i) sum[(EPI == EPI_SYRK ? c * 32 + hh * 16 + i : 0)] += v[i];
+            }
+          } else if (EPI == EPI_SUMSQ) {
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s = fmaf(v[i], v[i], s);
+            acc += static_cast<double>(s);
+          } else {
+            if (row0 >= p.M || col0 >= p.N) continue;
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            const int row = row0 + lane;
+            if (row < p.M) {
+              const float* drow = p.D + static_cast<int64_t>(row) * p.ldd + col0;
+              float s = 0.f;
+              if (col0 + 32 <= p.N) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                  const float4 d = __ldg(reinterpret_cast<const float4*>(drow + i));
+                  s = fmaf(v[i], d.x, s);
+                  s = fmaf(v[i + 1], d.y, s);
+                  s = fmaf(v[i + 2], d.z, s);
+                  s = fmaf(v[i + 3], d.w, s);
+                }
+              } else {
+                const int lim = p.N - col0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (i < lim) s = fmaf(v[i], __ldg(drow + i), s);
+              }
+              acc += static_cast<double>(s);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        // one partial per (tile, lane quarter): no cross-warp synchronisation
-        acc = warp_sum_d(acc);
-        if (lane == 0) p.partials[static_cast<int64_t>(t) * 4 + q] = acc;
       }
-    } else {
-      // Each warp owns 32 rows of the tile and moves them out in 32x32 slabs
-      // through a double-buffered staging tile in the TMA 128-byte swizzle
-      // (16-byte chunk k of row r sits at chunk k ^ (r % 8)).  A chunk's slabs
-      // are stored (first chunk, accumulate == 0) or reduce-added into H; the
-      // next chunk of the same tile waits until they have all landed, so the
-      // additions into H happen in chunk order.
-      float* stg = stg_all + q * 2 * 1024;
-      uint32_t nst = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        int mt, nt, bz;
-        decode_tile<EPI>(p, t, mt, nt, bz);
-        const int row0 = mt * BM + q * 32;
-        for (int ch = 0; ch < n_chunks; ++ch, ++lt) {
-          const int buf = lt & 1;
-          const uint32_t use = static_cast<uint32_t>(lt >> 1);
-          if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 4)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (lane == 0 && ch > 0) bulk_wait_all();  // previous chunk's additions landed
-          __syncwarp();
-          const bool store = ch == 0 && p.accumulate == 0;
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                 static_cast<uint32_t>(buf * BN);
-#pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
-            const int col0 = nt * BN + c * 32;
-            // slabs wholly below the diagonal, or outside H, are not needed
-            if (row0 >= p.M || col0 >= p.N || col0 + 32 <= row0) continue;
-            float v[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, v);  // lane = row, v[i] = column i
-            float* sb = stg + (nst & 1) * 1024;
-            if (lane == 0) bulk_wait_read<1>();  // this buffer's previous copy has read it
-            __syncwarp();
+      if (!ok) break;
+      if (EPI == EPI_SYRK) {
+        // the finished tile: this thread's row, straight from registers
+        const int row = row0 + lane;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<float4*>(sb + lane * 32 + ((k ^ (lane & 7)) << 2)) =
-                  make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (store)
-                tma_store_3d(&tmC, sb, col0, row0, 0);
-              else
-                tma_reduce_add_3d(&tmC, sb, col0, row0, 0);
-              bulk_commit();
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = colh + c * 32;
+          if (row0 >= p.M || col0 >= p.N || col0 + 32 <= row0 || row >= p.M) continue;
+          float* dst = p.C + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const int j = EPI == EPI_SYRK ? c * 32 + i : 0;
+              float4 o = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+              if (p.accumulate) {
+                const float4 old = *reinterpret_cast<const float4*>(dst + i);
+                o.x += old.x;
+                o.y += old.y;
+                o.z += old.z;
+                o.w += old.w;
+              }
+              *reinterpret_cast<float4*>(dst + i) = o;
             }
-            ++nst;
+          } else {
+            const int lim = p.N - col0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int j = EPI == EPI_SYRK ? c * 32 + i : 0;
+              if (i < lim) dst[i] = p.accumulate ? dst[i] + sum[j] : sum[j];
+            }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
+      } else {
+        // one partial per (tile, epilogue warp): no cross-warp synchronisation
+        acc = warp_sum_d(acc);
+        if (EPI == EPI_DOT) acc *= 2.0;
+        if (lane == 0) p.partials[static_cast<int64_t>(t) * EPI_WARPS + slot] = acc;
       }
-      if (lane == 0) bulk_wait_all();  // every copy of this warp has landed
     }
   }
 
@@ -362,15 +424,14 @@ int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
 }
 
 template <bool A_MN, bool B_MN, int EPI>
-int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, const Params& p,
-           cudaStream_t stream) {
+int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+           const CUtensorMap& b2, const Params& p, cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   auto kern = tc_gemm_kernel<A_MN, B_MN, EPI>;
-  constexpr int smem = smem_bytes<EPI>();
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
         cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
@@ -380,8 +441,18 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, con
   if (rc != PIQ_OK) return rc;
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
   note_launch();
-  kern<<<grid, THREADS, smem, stream>>>(a, b, c, p);
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(a, b, a2, b2, p);
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 2-D bf16 map of a row-major [rows][cols] matrix with box {bc, br}.
+int map2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t bc, uint32_t br) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * 2};
+  const uint32_t box[2] = {bc, br};
+  return make_map(m, base, 2, dims, strides, box);
 }
 
 }  // namespace
@@ -390,22 +461,10 @@ int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accu
                     DeviceStatus* st, cudaStream_t stream) {
   if (n < 1 || in < 8 || in % 8 != 0 || n > INT32_MAX || in > INT32_MAX / 2)
     return PIQ_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(X) & 15u) != 0 || (reinterpret_cast<uintptr_t>(H) & 15u) != 0)
-    return PIQ_ERR_INVALID_ARG;
-  CUtensorMap map, mc;
-  const uint64_t dims[2] = {static_cast<uint64_t>(in), static_cast<uint64_t>(n)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(in) * 2};
-  const uint32_t box[2] = {64, 64};
-  int rc = make_map(&map, X, 2, dims, strides, box);
+  if (!aligned16(X) || !aligned16(H)) return PIQ_ERR_INVALID_ARG;
+  CUtensorMap map;
+  int rc = map2d(&map, X, n, in, 64, 64);
   if (rc != PIQ_OK) return rc;
-  {
-    const uint64_t cd[3] = {static_cast<uint64_t>(in), static_cast<uint64_t>(in), 1};
-    const uint64_t cs[2] = {static_cast<uint64_t>(in) * 4,
-                            static_cast<uint64_t>(in) * static_cast<uint64_t>(in) * 4};
-    const uint32_t cb[3] = {32, 32, 1};
-    rc = make_map(&mc, H, 3, cd, cs, cb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
-    if (rc != PIQ_OK) return rc;
-  }
   Params p{};
   p.M = p.N = static_cast<int>(in);
   p.K = static_cast<int>(n);
@@ -421,11 +480,11 @@ int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accu
   p.accumulate = accumulate;
   p.kb_chunk = KC / BK;
   p.st = st;
-  return launch<true, true, EPI_STORE_UPPER>(map, map, mc, p, stream);
+  return launch<true, true, EPI_SYRK>(map, map, map, map, p, stream);
 }
 
 int64_t sumsq_partials_count(int64_t n, int64_t rows, int batch) {
-  return ceil_div(n, BM) * ceil_div(rows, BN) * batch * 4;
+  return ceil_div(n, BM) * ceil_div(rows, BN) * batch * EPI_WARPS;
 }
 
 int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D, int64_t rows,
@@ -433,21 +492,17 @@ int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D
   if (n < 1 || in < 8 || in % 8 != 0 || rows < 1 || batch < 1 || n > INT32_MAX ||
       rows > INT32_MAX)
     return PIQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(D)) return PIQ_ERR_INVALID_ARG;
   CUtensorMap ma, mb;
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(in), static_cast<uint64_t>(n)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(in) * 2};
-    const uint32_t box[2] = {64, BM};
-    int rc = make_map(&ma, X, 2, dims, strides, box);
-    if (rc != PIQ_OK) return rc;
-  }
+  int rc = map2d(&ma, X, n, in, 64, BM);
+  if (rc != PIQ_OK) return rc;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(in), static_cast<uint64_t>(rows),
                               static_cast<uint64_t>(batch)};
     const uint64_t strides[2] = {static_cast<uint64_t>(in) * 2,
                                  static_cast<uint64_t>(in) * static_cast<uint64_t>(rows) * 2};
     const uint32_t box[3] = {64, BN, 1};
-    int rc = make_map(&mb, D, 3, dims, strides, box);
+    rc = make_map(&mb, D, 3, dims, strides, box);
     if (rc != PIQ_OK) return rc;
   }
   Params p{};
@@ -463,7 +518,43 @@ int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D
   p.partials = partials;
   p.kb_chunk = INT32_MAX;  // one accumulation per tile
   p.st = st;
-  return launch<false, false, EPI_SUMSQ>(ma, mb, ma, p, stream);
+  return launch<false, false, EPI_SUMSQ>(ma, mb, ma, mb, p, stream);
+}
+
+int64_t err_dot_partials_count(int64_t out, int64_t in) {
+  return ceil_div(out, BM) * ceil_div(in, BN) * EPI_WARPS;
+}
+
+int launch_err_dot(const uint16_t* D_hi, const uint16_t* D_lo, const uint16_t* Hu_hi,
+                   const uint16_t* Hu_lo, const float* D, int64_t out, int64_t in,
+                   double* partials, DeviceStatus* st, cudaStream_t stream) {
+  if (out < 1 || in < 8 || in % 8 != 0 || out > INT32_MAX || in > INT32_MAX / 4)
+    return PIQ_ERR_INVALID_ARG;
+  if (!aligned16(D_hi) || !aligned16(D_lo) || !aligned16(Hu_hi) || !aligned16(Hu_lo) ||
+      !aligned16(D))
+    return PIQ_ERR_INVALID_ARG;
+  CUtensorMap ma, ma2, mb, mb2;
+  int rc = map2d(&ma, D_hi, out, in, 64, BM);
+  if (rc == PIQ_OK) rc = map2d(&ma2, D_lo, out, in, 64, BM);
+  if (rc == PIQ_OK) rc = map2d(&mb, Hu_hi, in, in, 64, 64);
+  if (rc == PIQ_OK) rc = map2d(&mb2, Hu_lo, in, in, 64, 64);
+  if (rc != PIQ_OK) return rc;
+  Params p{};
+  p.M = static_cast<int>(out);
+  p.N = static_cast<int>(in);
+  p.K = static_cast<int>(in);
+  p.m_tiles = static_cast<int>(ceil_div(out, BM));
+  p.n_tiles = static_cast<int>(ceil_div(in, BN));
+  p.batch = 1;
+  const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  if (total > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+  p.num_tiles = static_cast<int>(total);
+  p.D = D;
+  p.ldd = in;
+  p.partials = partials;
+  p.kb_chunk = INT32_MAX;  // three segments of at most in / 64 k blocks each, one accumulation
+  p.st = st;
+  return launch<false, true, EPI_DOT>(ma, mb, ma2, mb2, p, stream);
 }
 
 // ------------------------------------------------ fixed-order partial reduction
@@ -495,12 +586,18 @@ __global__ void __launch_bounds__(RP_THREADS)
 }
 }  // namespace
 
-int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,
-                           double* out, cudaStream_t stream) {
-  const int64_t per = ceil_div(n, BM) * ceil_div(rows, BN) * 4;
+int launch_reduce_sum(const double* partials, int64_t per, int batch, double* out,
+                      cudaStream_t stream) {
+  if (per < 1 || batch < 1) return PIQ_ERR_INVALID_ARG;
   note_launch();
   reduce_partials_kernel<<<batch, RP_THREADS, 0, stream>>>(partials, per, out);
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,
+                           double* out, cudaStream_t stream) {
+  return launch_reduce_sum(partials, ceil_div(n, BM) * ceil_div(rows, BN) * EPI_WARPS, batch,
+                           out, stream);
 }
 
 }  // namespace piq

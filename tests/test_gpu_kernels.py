@@ -16,7 +16,8 @@ def _layer(out, inp, n, seed=0, **kw):
     return make_weight(spec), make_x_bits(spec)
 
 
-@pytest.mark.parametrize("n,inp", [(2048, 512), (1000, 136), (77, 264), (4100, 1032), (64, 8)])
+@pytest.mark.parametrize("n,inp", [(2048, 512), (1000, 136), (77, 264), (4100, 1032), (64, 8),
+                                   (12300, 264)])
 def test_hessian_matches_exact(n, inp):
     W, X = _layer(8, inp, n, seed=n + inp)
     H = np.triu(piq.hessian(to_gpu_x(X)).cpu().numpy()).astype(np.float64)
@@ -88,6 +89,31 @@ def test_output_error_gemm_matches_oracle():
     What = codes * np.repeat(sc.cpu().numpy().astype(np.float64), 128, axis=1)[:, :520]
     ex = O.output_error_ref(W, What, X)
     assert rel(e, ex) < REL_TOL  # bf16 rounding of W - What is the dominant term
+
+
+@pytest.mark.parametrize("out,inp,n", [
+    (300, 520, 1500),  # n small against in: the direct product X D^T
+    (520, 264, 4100),  # n large against in and out: the route through H = X^T X
+])
+def test_output_error_routes(out, inp, n):
+    # a packed layer with act-order groups and AWQ channel scales, on ragged sizes
+    W, X = _layer(out, inp, n, seed=out + n, sigma_ln=1.0, n_outlier=3, outlier_gain=30.0)
+    rng = np.random.default_rng(out)
+    g, bits = 64, 4
+    ng = -(-inp // g)
+    perm = rng.permutation(inp)
+    g_idx = np.empty(inp, np.int32)
+    g_idx[perm] = np.arange(inp) // g
+    s = np.exp(rng.normal(0.0, 0.5, inp)).astype(np.float32)
+    codes = rng.integers(-8, 8, (out, inp))
+    sc16 = rng.uniform(0.002, 0.01, (out, ng)).astype(np.float16)
+    qw = torch.from_numpy(O.pack_ref(codes, bits).view(np.int32)).cuda()
+    e = piq.layer_output_error(to_gpu_w(W), qw, torch.from_numpy(sc16).cuda(),
+                               to_gpu_x(X), bits, g,
+                               g_idx=torch.from_numpy(g_idx).cuda(),
+                               s=torch.from_numpy(s).cuda())
+    What = codes * sc16.astype(np.float64)[:, g_idx] / s.astype(np.float64)
+    assert rel(e, O.output_error_ref(W, What, X)) < REL_TOL
 
 
 def test_rtn_matches_oracle():
