@@ -134,7 +134,6 @@ __global__ void __launch_bounds__(R, 1)
   // Tiles arrive by asynchronous copies (16-byte when the block start allows);
   // a second pass zeroes what the column loop must see as zero.
   const int rows_here = static_cast<int>(std::min<int64_t>(R, out - row0));
-  const float ujj = (tid < kb) ? U[(b + tid) * in + b + tid] : 1.f;  // in flight meanwhile
   if ((b & 3) == 0) {
     const int kq = (kb + 3) >> 2;  // b + 4*kq <= in since in % 8 == 0
     for (int idx = tid; idx < kb * kq; idx += R) {
@@ -165,7 +164,7 @@ __global__ void __launch_bounds__(R, 1)
     const int r = idx >> 7, c = idx & (B - 1);
     if (r >= rows_here || c >= kb) Wr[r * LDW + c] = 0.f;
   }
-  inv_u[tid] = (tid < kb) ? 1.f / ujj : 0.f;
+  for (int j = tid; j < B; j += R) inv_u[j] = (j < kb) ? 1.f / U[(b + j) * in + b + j] : 0.f;
   __syncthreads();
 
   SweepRow rs;

@@ -3,10 +3,12 @@
 // The FP32 products of the path (the GPTQ trailing update W[:, e:] -= Err U and
 // the panel updates of the Cholesky and the triangular inverse that produce U)
 // need about FP32 accuracy; a single TF32 pass (10-bit mantissa) is too coarse.
-// Each operand is split in shared memory into x = hi + lo, hi = tf32(x) (round
-// to nearest), lo = x - hi (exact in fp32), and the tile is accumulated in TMEM
-// as  A_hi B_hi + A_hi B_lo + A_lo B_hi  (the dropped A_lo B_lo is ~2^-22 of
-// the product).
+// Each operand is split into x = hi + lo with hi = x with its 13 low mantissa
+// bits cleared and lo = x - hi (exact in fp32).  The tensor core reads only the
+// top 19 bits of a 32-bit operand, so the TMA-landed tile itself serves as hi
+// and only lo is written; the tile is accumulated in TMEM as
+// A_hi B_hi + A_hi B_lo + A_lo B_hi  (lo is itself cut to 19 bits by the
+// tensor core, and the dropped A_lo B_lo is ~2^-20 of the product).
 //
 // C = alpha A op(B) + beta C, all fp32 row-major: A [M][K] (K-major tiles), B
 // [K][N] (MN-major tiles) or, with trans_b, [N][K] (K-major).  Modes: 0 plain;
@@ -15,7 +17,7 @@
 // Batched over entries with element strides; entry z may have fewer rows.
 //
 // Warp roles (320 threads): warp 0 lane 0 issues TMA loads of fp32 tiles into a
-// 3-stage ring; warps 6..9 split each landed tile into hi/lo; warp 1 lane 0
+// 3-stage ring; warps 6..9 write the lo part of each landed tile; warp 1 lane 0
 // issues the MMAs; warps 2..5 drain one of two 128-column accumulators.  Every
 // wait is bounded; no multicast loads.
 #include <cuda.h>
@@ -93,12 +95,6 @@ __device__ __forceinline__ TileInfo tile_info(const SgParams& p, int t) {
   ti.kb1 = (kend + BK - 1) / BK;
   if (ti.kb1 < ti.kb0) ti.kb1 = ti.kb0;
   return ti;
-}
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
 }
 
 // Instruction descriptor: kind::tf32, fp32 accumulate, M = 128, N = 128.
@@ -218,15 +214,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
           uint4 h, l;
-          h.x = to_tf32(__uint_as_float(v.x));
-          h.y = to_tf32(__uint_as_float(v.y));
-          h.z = to_tf32(__uint_as_float(v.z));
-          h.w = to_tf32(__uint_as_float(v.w));
+          h.x = v.x & 0xFFFFE000u;
+          h.y = v.y & 0xFFFFE000u;
+          h.z = v.z & 0xFFFFE000u;
+          h.w = v.w & 0xFFFFE000u;
           l.x = __float_as_uint(__uint_as_float(v.x) - __uint_as_float(h.x));
           l.y = __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h.y));
           l.z = __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h.z));
           l.w = __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h.w));
-          hi[i] = h;
+          if (klim < BK) hi[i] = v;  // a short k block: the zeroed columns
           lo[i] = l;
         }
         fence_proxy_async_smem();  // generic writes -> visible to the tensor cores
