@@ -38,6 +38,9 @@ METRIC = "GPTQ INT4 sec/layer & Mweights/s; XᵀX TFLOPS; AWQ α-search ms/layer
 UNIT = "Mweights/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one syrk_xtx launch on the 131072 x 4096 workload, from the ncu
+# capture summarised in profiles/syrk_xtx_q_proj_7b.md; None once the kernel changes.
+SYRK_TRAFFIC_BYTES = 1.88e9 + 21.69e6
 
 
 def load_peaks():
@@ -358,7 +361,10 @@ def run_ours(args):
     ach_h = flops_h / (t_h / 1e3) / 1e12
     roof = {"kernel": "syrk_xtx (tcgen05 H = X^T X, 4096-sample chunks summed in registers)",
             "bound": "tensor", "achieved": ach_h, "peak": peak, "unit": "TFLOP/s",
-            "frac": ach_h / peak, "traffic": args.traffic, "flops_per_launch": flops_h,
+            "frac": ach_h / peak,
+            "traffic": args.traffic if args.traffic is not None else (
+                SYRK_TRAFFIC_BYTES if args.samples is None else None),
+            "flops_per_launch": flops_h,
             "flops_formula": "n*in*(in+1) (upper triangle)", "ms_per_launch": t_h,
             "peak_source": f"{peak_src} {peak_key}"}
 
