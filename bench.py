@@ -38,8 +38,9 @@ METRIC = "GPTQ INT4 sec/layer & Mweights/s; XᵀX TFLOPS; AWQ α-search ms/layer
 UNIT = "Mweights/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one syrk_xtx launch on the 131072 x 4096 workload, from the ncu
-# capture summarised in profiles/syrk_xtx_q_proj_7b.md; None once the kernel changes.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one syrk_xtx launch on the
+# 131072 x 4096 workload, from one ncu capture of the current kernel; to be retaken (or set to
+# None) whenever that kernel changes.
 SYRK_TRAFFIC_BYTES = 1.88e9 + 21.69e6
 
 
