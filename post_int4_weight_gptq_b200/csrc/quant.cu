@@ -35,20 +35,32 @@ __global__ void __launch_bounds__(256) colstats_kernel(const uint16_t* __restric
   double sa[8], sq[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) sa[i] = sq[i] = 0.0;
-  if (col < in) {
-    for (int64_t r = r0 + warp; r < r1; r += 8) {
-      const uint4 v = *reinterpret_cast<const uint4*>(X + r * in + col);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  auto add = [&](const uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = bf16_bits_to_float(static_cast<uint16_t>(w[i] & 0xFFFFu));
-        const float hi = bf16_bits_to_float(static_cast<uint16_t>(w[i] >> 16));
-        sa[2 * i] += static_cast<double>(fabsf(lo));
-        sa[2 * i + 1] += static_cast<double>(fabsf(hi));
-        sq[2 * i] += static_cast<double>(lo * lo);  // exact: bf16 square fits fp32
-        sq[2 * i + 1] += static_cast<double>(hi * hi);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const float lo = bf16_bits_to_float(static_cast<uint16_t>(w[i] & 0xFFFFu));
+      const float hi = bf16_bits_to_float(static_cast<uint16_t>(w[i] >> 16));
+      sa[2 * i] += static_cast<double>(fabsf(lo));
+      sa[2 * i + 1] += static_cast<double>(fabsf(hi));
+      sq[2 * i] += static_cast<double>(lo * lo);  // exact: bf16 square fits fp32
+      sq[2 * i + 1] += static_cast<double>(hi * hi);
     }
+  };
+  if (col < in) {
+    // four rows in flight per thread; rows are added in the same order either way
+    int64_t r = r0 + warp;
+    for (; r + 24 < r1; r += 32) {
+      const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(X + r * in + col));
+      const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(X + (r + 8) * in + col));
+      const uint4 v2 = __ldg(reinterpret_cast<const uint4*>(X + (r + 16) * in + col));
+      const uint4 v3 = __ldg(reinterpret_cast<const uint4*>(X + (r + 24) * in + col));
+      add(v0);
+      add(v1);
+      add(v2);
+      add(v3);
+    }
+    for (; r < r1; r += 8) add(__ldg(reinterpret_cast<const uint4*>(X + r * in + col)));
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -84,13 +96,24 @@ __global__ void colstats_finish_kernel(const double* __restrict__ part, int64_t 
 }
 
 // --------------------------------------------------------------------- gather
+// Wq[r][p] = W[r][perm[p]] (perm == NULL: a copy), four positions per thread
+// (in % 4 == 0 and 16-byte aligned rows; the launcher checks).
 __global__ void gather_columns_kernel(const float* __restrict__ W, int64_t out, int64_t in,
                                       const int32_t* __restrict__ perm, float* __restrict__ Wq) {
-  const int64_t total = out * in;
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+  const int64_t total4 = out * in / 4;
+  const int64_t in4 = in / 4;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total4;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = idx / in, p = idx - r * in;
-    Wq[idx] = W[r * in + (perm ? perm[p] : p)];
+    float4 v;
+    if (perm == nullptr) {
+      v = __ldg(reinterpret_cast<const float4*>(W) + idx);
+    } else {
+      const int64_t r = idx / in4, p = (idx - r * in4) * 4;
+      const int4 c = __ldg(reinterpret_cast<const int4*>(perm + p));
+      const float* wr = W + r * in;
+      v = make_float4(__ldg(wr + c.x), __ldg(wr + c.y), __ldg(wr + c.z), __ldg(wr + c.w));
+    }
+    reinterpret_cast<float4*>(Wq)[idx] = v;
   }
 }
 
@@ -328,19 +351,45 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
     const int64_t r = idx / words, wd = idx - r * words;
     const uint32_t word = qweight[idx];
     float d32[8];
+    const float4 wa = __ldg(reinterpret_cast<const float4*>(W + r * in + wd * 8));
+    const float4 wb = __ldg(reinterpret_cast<const float4*>(W + r * in + wd * 8 + 4));
+    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    int gi[8];
+    if (g_idx && (reinterpret_cast<uintptr_t>(g_idx) & 15u) != 0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gi[k] = g_idx[wd * 8 + k];
+    } else if (g_idx) {
+      const int4 ga = __ldg(reinterpret_cast<const int4*>(g_idx + wd * 8));
+      const int4 gb = __ldg(reinterpret_cast<const int4*>(g_idx + wd * 8 + 4));
+      gi[0] = ga.x; gi[1] = ga.y; gi[2] = ga.z; gi[3] = ga.w;
+      gi[4] = gb.x; gi[5] = gb.y; gi[6] = gb.z; gi[7] = gb.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gi[k] = static_cast<int>((wd * 8 + k) / g);
+    }
+    float sv[8];
+    if (s && (reinterpret_cast<uintptr_t>(s) & 15u) != 0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sv[k] = s[wd * 8 + k];
+    } else if (s) {
+      const float4 sa = __ldg(reinterpret_cast<const float4*>(s + wd * 8));
+      const float4 sb = __ldg(reinterpret_cast<const float4*>(s + wd * 8 + 4));
+      sv[0] = sa.x; sv[1] = sa.y; sv[2] = sa.z; sv[3] = sa.w;
+      sv[4] = sb.x; sv[5] = sb.y; sv[6] = sb.z; sv[7] = sb.w;
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int64_t c = wd * 8 + k;
       const int code = static_cast<int>((word >> (4 * k)) & 0xFu) - off;
-      int64_t grp = g_idx ? g_idx[c] : c / g;
+      int64_t grp = gi[k];
       if (grp < 0 || grp >= ngroups) {  // caller's group index out of range
         set_status(st, PIQ_ERR_INVALID_ARG, static_cast<int>(c));
         grp = 0;
       }
       const float sc = __half2float(__ushort_as_half(scales16[r * ngroups + grp]));
       float what = static_cast<float>(code) * sc;
-      if (s) what = __fdiv_rn(what, s[c]);
-      d32[k] = W[r * in + c] - what;
+      if (s) what = __fdiv_rn(what, sv[k]);
+      d32[k] = wv[k] - what;
     }
     if (dW32) {
       float4* dst = reinterpret_cast<float4*>(dW32 + r * in + wd * 8);
@@ -392,8 +441,11 @@ int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, 
 
 int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
                           float* Wq, cudaStream_t stream) {
+  if (in % 4 != 0 || (reinterpret_cast<uintptr_t>(W) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(Wq) & 15u) != 0 || (reinterpret_cast<uintptr_t>(perm) & 15u) != 0)
+    return PIQ_ERR_INVALID_ARG;
   note_launch();
-  gather_columns_kernel<<<grid_for(out * in, 256), 256, 0, stream>>>(W, out, in, perm, Wq);
+  gather_columns_kernel<<<grid_for(out * in / 4, 256), 256, 0, stream>>>(W, out, in, perm, Wq);
   return last_error();
 }
 
