@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(CI_THREADS)
   float* rinv = Tm + 64 * TLD;   // [NB] reciprocal pivots
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_launch_dependents();
+  pdl_wait();  // P comes from the previous kernel
   if (status_bad(st)) return;
   if (tid == 0) bad = 0;
 
@@ -469,8 +471,9 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     const int nb = static_cast<int>(std::min<int64_t>(NB, in - k0));
     const int nbp = nb <= 32 ? 32 : (nb <= 64 ? 64 : 128);
     note_launch();
-    chol_inv_kernel<<<1, CI_THREADS, kCholSmem, stream>>>(P, X, ld, k0, nb, nbp, st);
-    if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+    if (launch_pdl(chol_inv_kernel, dim3(1), dim3(CI_THREADS), kCholSmem, stream, P, X, ld, k0,
+                   nb, nbp, st) != cudaSuccess)
+      return PIQ_ERR_CUDA;
     const int rem = static_cast<int>(in - k0 - nb);
     if (rem <= 0) continue;
     float* A21 = P + (k0 + nb) * ld + k0;

@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(R, 1)
   float* inv_u = Us + B * B;            // [B], 1 / U[j][j]
   float* Wr = inv_u + B;                // [R][LDW], row state; errors replace used columns
   int8_t* Cs = reinterpret_cast<int8_t*>(Wr + R * LDW);  // [R][LDC]
+  pdl_launch_dependents();
+  pdl_wait();  // W and U come from the previous kernels
   if (status_bad(st)) return;
   const int tid = threadIdx.x;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
@@ -278,13 +280,12 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
     for (int64_t gs = (b % g == 0) ? b : (b / g + 1) * g; gs < e; gs += g)
       aligned = aligned && ((gs - b) % SUB == 0);
     note_launch();
-    if (aligned)
-      sweep_block_kernel<false><<<grid, R, kSweepSmem, stream>>>(Wq, out, in, U, b, kb, bits, g,
-                                                                 codes, qscale, Err, st);
-    else
-      sweep_block_kernel<true><<<grid, R, kSweepSmem, stream>>>(Wq, out, in, U, b, kb, bits, g,
-                                                                codes, qscale, Err, st);
-    if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+    const cudaError_t le =
+        aligned ? launch_pdl(sweep_block_kernel<false>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
+                             out, in, U, b, kb, bits, g, codes, qscale, Err, st)
+                : launch_pdl(sweep_block_kernel<true>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
+                             out, in, U, b, kb, bits, g, codes, qscale, Err, st);
+    if (le != cudaSuccess) return PIQ_ERR_CUDA;
     if (e < in) {
       // W[:, e:] -= Err[:, :kb] U[b:e, e:]
       int rc = launch_gemm_f32(static_cast<int>(out), static_cast<int>(in - e), kb, -1.f, Err, B,

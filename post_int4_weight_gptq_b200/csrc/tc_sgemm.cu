@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (status_bad(p.st)) return;
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -145,8 +145,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // inputs come from the previous kernel; an earlier failure skips the work
+  // (uniform over the CTA, which still frees its TMEM below)
+  pdl_wait();
+  const bool skip = status_bad(p.st);
 
-  if (warp == 0) {
+  if (skip) {
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       uint32_t it = 0;
@@ -465,7 +470,9 @@ int launch_tc_sgemm(int M, int N, int K, float alpha, const float* A, int64_t ld
   }
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
   note_launch();
-  tf32x3_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, p);
+  if (launch_pdl(tf32x3_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, ma, mb, mc,
+                 p) != cudaSuccess)
+    return PIQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
