@@ -294,6 +294,103 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The code rint(v / scale) clipped, from v * (1 / scale): the product differs
+// from the IEEE quotient by at most two units in the last place, so it can only
+// round differently within ~1e-6 of a half-integer; there the IEEE division
+// decides.  Same result as quant_code.
+__device__ __noinline__ float code_by_division(float v, float scale) {
+  return rintf(__fdiv_rn(v, scale));
+}
+__device__ __forceinline__ float quant_code_rcp(float v, float scale, float rs, float cmin,
+                                                float cmax) {
+  const float t = v * rs;
+  float q = rintf(t);
+  if (fabsf(fabsf(t - q) - 0.5f) < 1e-5f) q = code_by_division(v, scale);  // rare
+  return scale > 0.f ? fminf(fmaxf(q, cmin), cmax) : 0.f;
+}
+
+// D_a[r][c] = W - code * scale / s for every alpha a, for power-of-two g with
+// 8 <= g <= 256 and in % 8 == 0.  Lane l of a warp holds columns 8l .. 8l+7 of a
+// 256-column slice (g / 8 lanes per group) for kRows rows; per alpha the s and
+// 1 / s of its columns are read once for all kRows rows.
+constexpr int kRows = 4;
+__global__ void __launch_bounds__(256)
+    awq_delta_rows_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits, int g,
+                          const float* __restrict__ s_table, int n_alpha,
+                          uint16_t* __restrict__ dW) {
+  const int lane = threadIdx.x & 31;
+  const int lg = g >> 3;  // lanes per group
+  const int qmax = (1 << (bits - 1)) - 1;
+  const float fqmax = static_cast<float>(qmax), cmin = static_cast<float>(-qmax - 1),
+              cmax = static_cast<float>(qmax);
+  const float* inv_table = s_table + static_cast<int64_t>(n_alpha) * in;
+  const int64_t slices = (in + 255) / 256;
+  const int64_t rblocks = (out + kRows - 1) / kRows;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t wi = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wi < rblocks * slices; wi += nwarps) {
+    const int64_t rb = wi / slices, sl = wi - rb * slices;
+    const int64_t col = sl * 256 + 8 * lane;
+    const bool act = col < in;  // in % 8 == 0: a lane is wholly in or out
+    const int64_t r0 = rb * kRows;
+    float w[kRows][8];
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      const bool ok = act && r0 + k < out;
+      const float4 a = ok ? __ldg(reinterpret_cast<const float4*>(W + (r0 + k) * in + col))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 b = ok ? __ldg(reinterpret_cast<const float4*>(W + (r0 + k) * in + col + 4))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[k][0] = a.x; w[k][1] = a.y; w[k][2] = a.z; w[k][3] = a.w;
+      w[k][4] = b.x; w[k][5] = b.y; w[k][6] = b.z; w[k][7] = b.w;
+    }
+    for (int al = 0; al < n_alpha; ++al) {
+      float sv[8], iv[8];
+      {
+        const int64_t off = static_cast<int64_t>(al) * in + col;
+        const float4 a = act ? __ldg(reinterpret_cast<const float4*>(s_table + off))
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 b = act ? __ldg(reinterpret_cast<const float4*>(s_table + off + 4))
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 c = act ? __ldg(reinterpret_cast<const float4*>(inv_table + off))
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 d = act ? __ldg(reinterpret_cast<const float4*>(inv_table + off + 4))
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w;
+        sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+        iv[0] = c.x; iv[1] = c.y; iv[2] = c.z; iv[3] = c.w;
+        iv[4] = d.x; iv[5] = d.y; iv[6] = d.z; iv[7] = d.w;
+      }
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        float p[8], m = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = w[k][e] * sv[e];
+          m = fmaxf(m, fabsf(p[e]));
+        }
+        for (int o = 1; o < lg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float scale = __fdiv_rn(m, fqmax);
+        const float rs = scale > 0.f ? __frcp_rn(scale) : 0.f;
+        uint16_t d16[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float q = quant_code_rcp(p[e], scale, rs, cmin, cmax);
+          d16[e] = float_to_bf16_bits(fmaf(-(q * scale), iv[e], w[k][e]));
+        }
+        if (act && r0 + k < out) {
+          uint4 o;
+          o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
+          o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
+          o.z = d16[4] | (static_cast<uint32_t>(d16[5]) << 16);
+          o.w = d16[6] | (static_cast<uint32_t>(d16[7]) << 16);
+          *reinterpret_cast<uint4*>(dW + (static_cast<int64_t>(al) * out + r0 + k) * in + col) = o;
+        }
+      }
+    }
+  }
+}
+
 // codes + fp32 scales of W diag(s_table[sel]) (s_table == NULL: s = 1).
 __global__ void group_quant_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits,
                                    int g, const float* __restrict__ s_table,
@@ -473,7 +570,12 @@ int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,
                      const float* s_table, int n_alpha, uint16_t* dW, cudaStream_t stream) {
   const int64_t warps = out * ceil_div(in, g);
   note_launch();
-  if (g % 4 == 0 && g <= 128)
+  const bool pow2 = g >= 8 && g <= 256 && (g & (g - 1)) == 0;
+  if (pow2 && in % 8 == 0) {
+    const int64_t rwarps = ceil_div(out, kRows) * ceil_div(in, 256);
+    awq_delta_rows_kernel<<<grid_for(rwarps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g,
+                                                                          s_table, n_alpha, dW);
+  } else if (g % 4 == 0 && g <= 128)
     awq_delta_vec_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, out, in, bits, g,
                                                                         s_table, n_alpha, dW);
   else

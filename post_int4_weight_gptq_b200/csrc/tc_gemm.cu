@@ -137,8 +137,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // an earlier step already failed: do nothing (uniform over the CTA)
-  if (status_bad(p.st)) return;
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -166,8 +165,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (p.K + BK - 1) / BK;
+  // inputs come from the previous kernel; an earlier failure skips the work
+  // (uniform over the CTA, which still frees its TMEM below)
+  pdl_wait();
+  const bool skip = status_bad(p.st);
 
-  if (warp == 0) {
+  if (skip) {
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       uint32_t it = 0;
@@ -441,8 +445,10 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
   if (rc != PIQ_OK) return rc;
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
   note_launch();
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(a, b, a2, b2, p);
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, a, b, a2, b2, p) ==
+                 cudaSuccess
+             ? PIQ_OK
+             : PIQ_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
