@@ -38,16 +38,32 @@ constexpr int R = 128;       // rows per CTA, one per thread
 constexpr int LDW = B + 4;   // row-state stride (float4-aligned, conflict-free per 8 lanes)
 constexpr int LDC = B + 4;   // code staging row (bytes)
 constexpr int kSweepSmem = B * B * 4 + B * 4 + R * LDW * 4 + R * LDC;
+constexpr int kQuartersSmem = kSweepSmem + R * 4;
 
 // Per-row state of the column loop.
 struct SweepRow {
   float scale;
+  float rscale;      // 1 / scale (0 when scale is 0)
   int64_t next_gs;   // block-relative column of the next group start
   float fqmax, cmin, cmax;
   int kb;
   int64_t b, in, g, ngroups, row;
   bool valid;
 };
+
+// rint(w / scale) for the IEEE quotient, from w * (1 / scale): the product is
+// within a few units in the last place of the quotient, so it can only round
+// differently within ~1e-6 |w / scale| of a half-integer, where the division
+// itself decides (rare, out of line).
+__device__ __noinline__ float code_by_division(float w, float scale) {
+  return rintf(__fdiv_rn(w, scale));
+}
+__device__ __forceinline__ float code_of(float w, float scale, float rscale) {
+  const float t = w * rscale;
+  const float q = rintf(t);
+  return fabsf(fabsf(t - q) - 0.5f) < 1e-5f * fmaxf(1.f, fabsf(t)) ? code_by_division(w, scale)
+                                                                   : q;
+}
 
 // Group start at block column j (window base c0, jj = j - c0): the scale comes
 // from the current weights of [j, j+g): the window in registers, later block
@@ -76,6 +92,7 @@ __device__ __forceinline__ void group_start(const float (&ws)[SUB], const float 
     for (int64_t c = st.b + st.kb; c < gend; ++c) m = fmaxf(m, fabsf(src[c]));
   }
   st.scale = __fdiv_rn(m, st.fqmax);
+  st.rscale = st.scale > 0.f ? __frcp_rn(st.scale) : 0.f;
   if (st.valid) qscale[st.row * st.ngroups + (st.b + j) / st.g] = st.scale;
   st.next_gs += st.g;
 }
@@ -93,7 +110,7 @@ __device__ __forceinline__ void sweep_col(float (&ws)[SUB], float (&e)[SUB], int
       if (GENERAL && j == st.next_gs) group_start(ws, e, JJ, c0, st, W, Us, wrow, qscale);
       const float wj = ws[JJ];
       const float sc = st.scale;
-      const float q = sc > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(wj, sc)), st.cmin), st.cmax) : 0.f;
+      const float q = sc > 0.f ? fminf(fmaxf(code_of(wj, sc, st.rscale), st.cmin), st.cmax) : 0.f;
       const float err = (wj - q * sc) * inv_u[j];
       code_row[j] = static_cast<int8_t>(q);
       e[JJ] = err;
@@ -184,6 +201,7 @@ __global__ void __launch_bounds__(R, 1)
   const int64_t boff = b % g;
   // a group that started in an earlier block keeps its scale
   rs.scale = (boff != 0 && rs.valid) ? qscale[rs.row * rs.ngroups + b / g] : 0.f;
+  rs.rscale = rs.scale > 0.f ? __frcp_rn(rs.scale) : 0.f;
   rs.next_gs = (boff == 0) ? 0 : g - boff;
 
   float* wrow = Wr + tid * LDW;
@@ -233,6 +251,209 @@ __global__ void __launch_bounds__(R, 1)
   }
 }
 
+// Blocks that hold no group start other than (possibly) their first column,
+// which is every block when g % 128 == 0.  16 warps: warp w owns rows
+// 32 (w % 4) .. + 31 (one per lane) and window q = w / 4 (block columns 32q ..
+// 32q + 31) in registers.  Phase p (0..3): the quarter-p warps apply the errors
+// of window p - 1 to their window and run its serial column loop; the warps of
+// later windows apply the same errors at the same time.  Window errors replace
+// the used columns of the row state in shared memory.
+constexpr int QT = 4 * R;  // threads of the quartered kernel
+
+__global__ void __launch_bounds__(QT, 1)
+    sweep_quarters_kernel(float* __restrict__ W, int64_t out, int64_t in,
+                          const float* __restrict__ U, int64_t b, int kb, int bits, int g,
+                          int8_t* __restrict__ codes, float* __restrict__ qscale,
+                          float* __restrict__ Err, DeviceStatus* st) {
+  extern __shared__ __align__(16) float smem[];
+  float* Us = smem;                     // [B][B], strictly upper part of U[b:e, b:e]
+  float* inv_u = Us + B * B;            // [B], 1 / U[j][j]
+  float* Wr = inv_u + B;                // [R][LDW], row state; errors replace used columns
+  int8_t* Cs = reinterpret_cast<int8_t*>(Wr + R * LDW);  // [R][LDC]
+  float* scale_s = reinterpret_cast<float*>(Cs + R * LDC);  // [R]
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // window q's four warps sit on the four schedulers (warp w issues from w % 4)
+  const int q = warp >> 2;                   // window
+  const int lrow = (warp & 3) * 32 + lane;   // row within the CTA
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
+  const int rows_here = static_cast<int>(std::min<int64_t>(R, out - row0));
+  const bool vec = (b & 3) == 0;  // 16-byte aligned rows at column b (in % 4 == 0 too)
+
+  // U is read before the wait: no kernel that lets its successor start early
+  // (the GEMMs, the factor, the sweep) writes U, so it is complete once this
+  // kernel runs.  The part on and below the diagonal (and past kb) is zeroed in
+  // the same pass.
+  if (vec) {
+    for (int idx = tid; idx < B * (B / 4); idx += QT) {
+      const int r = idx / (B / 4), c = (idx - r * (B / 4)) * 4;
+      float* dst = Us + r * B + c;
+      if (r < kb && c > r && c + 3 < kb) {
+        cp_async16(dst, U + (b + r) * in + b + c);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (r < kb && c + t > r && c + t < kb)
+            cp_async4(dst + t, U + (b + r) * in + b + c + t);
+          else
+            dst[t] = 0.f;
+        }
+      }
+    }
+  } else {
+    for (int idx = tid; idx < B * B; idx += QT) {
+      const int r = idx / B, c = idx - r * B;
+      if (r < kb && c > r && c < kb)
+        cp_async4(Us + idx, U + (b + r) * in + b + c);
+      else
+        Us[idx] = 0.f;
+    }
+  }
+  for (int j = tid; j < B; j += QT) inv_u[j] = (j < kb) ? 1.f / U[(b + j) * in + b + j] : 0.f;
+  pdl_wait();  // W comes from the previous kernels
+  if (status_bad(st)) {
+    cp_async_wait_all();
+    return;
+  }
+  if (vec) {
+    const int kq = (kb + 3) >> 2;
+    for (int idx = tid; idx < R * (B / 4); idx += QT) {
+      const int r = idx / (B / 4), c4 = idx - r * (B / 4);
+      float* dst = Wr + r * LDW + 4 * c4;
+      if (r < rows_here && c4 < kq)
+        cp_async16(dst, W + (row0 + r) * in + b + 4 * c4);  // kb % 4 == 0 or zero-padded below
+      else
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else {
+    for (int idx = tid; idx < R * B; idx += QT) {
+      const int r = idx / B, c = idx - r * B;
+      if (r < rows_here && c < kb)
+        cp_async4(Wr + r * LDW + c, W + (row0 + r) * in + b + c);
+      else
+        Wr[r * LDW + c] = 0.f;
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (vec && (kb & 3) != 0) {  // the last 16-byte chunk of a ragged block read past kb
+    for (int idx = tid; idx < R * 4; idx += QT) {
+      const int r = idx >> 2, c = (kb & ~3) + (idx & 3);
+      if (c >= kb) Wr[r * LDW + c] = 0.f;
+    }
+    __syncthreads();
+  }
+
+  SweepRow rs;
+  const int qmax = (1 << (bits - 1)) - 1;
+  rs.fqmax = static_cast<float>(qmax);
+  rs.cmin = static_cast<float>(-qmax - 1);
+  rs.cmax = static_cast<float>(qmax);
+  rs.kb = kb;
+  rs.b = b;
+  rs.in = in;
+  rs.g = g;
+  rs.ngroups = (in + g - 1) / g;
+  rs.row = row0 + lrow;
+  rs.valid = rs.row < out;
+  rs.next_gs = INT64_MAX;  // no group start inside the window loops
+  float* wrow = Wr + lrow * LDW;
+  int8_t* crow = Cs + lrow * LDC;
+  if (q == 0) {
+    // the row's scale: a group starts here (from the current weights of
+    // [b, b + g), past the block read from W), or it continues from earlier
+    float sc;
+    if (b % g == 0) {
+      const int64_t gend = std::min<int64_t>(b + g, in);
+      float m = 0.f;
+      for (int c4 = 0; c4 < B / 4; ++c4) {  // columns past kb are zero
+        const float4 v = reinterpret_cast<const float4*>(wrow)[c4];
+        m = fmaxf(fmaxf(m, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+      }
+      if (rs.valid)
+        for (int64_t c = b + kb; c < gend; ++c) m = fmaxf(m, fabsf(W[rs.row * in + c]));
+      sc = __fdiv_rn(m, rs.fqmax);
+      if (rs.valid) qscale[rs.row * rs.ngroups + b / g] = sc;
+    } else {
+      sc = rs.valid ? qscale[rs.row * rs.ngroups + b / g] : 0.f;
+    }
+    scale_s[lrow] = sc;
+  }
+  const int c0 = SUB * q;
+  // ws holds the window's weights; a used column's slot then holds its error
+  // (U is zero on and below the diagonal, so later updates leave it unchanged)
+  float ws[SUB];
+#pragma unroll
+  for (int k4 = 0; k4 < SUB / 4; ++k4) {
+    const float4 v = reinterpret_cast<const float4*>(wrow + c0)[k4];
+    ws[4 * k4] = v.x;
+    ws[4 * k4 + 1] = v.y;
+    ws[4 * k4 + 2] = v.z;
+    ws[4 * k4 + 3] = v.w;
+  }
+  __syncthreads();
+  rs.scale = scale_s[lrow];
+  rs.rscale = rs.scale > 0.f ? __frcp_rn(rs.scale) : 0.f;
+
+  for (int p = 0; p < 4; ++p) {
+    if (q >= p && SUB * p < kb) {
+      if (p > 0) {
+        // errors of window p - 1 onto this window
+        const int cp = SUB * (p - 1);
+#pragma unroll 1
+        for (int i4 = 0; i4 < SUB / 4; ++i4) {
+          const float4 e4 = reinterpret_cast<const float4*>(wrow + cp)[i4];
+          const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float4* urow = reinterpret_cast<const float4*>(Us + (cp + 4 * i4 + t) * B + c0);
+#pragma unroll
+            for (int k4 = 0; k4 < SUB / 4; ++k4) {
+              const float4 u = urow[k4];
+              ws[4 * k4 + 0] = fmaf(-ev[t], u.x, ws[4 * k4 + 0]);
+              ws[4 * k4 + 1] = fmaf(-ev[t], u.y, ws[4 * k4 + 1]);
+              ws[4 * k4 + 2] = fmaf(-ev[t], u.z, ws[4 * k4 + 2]);
+              ws[4 * k4 + 3] = fmaf(-ev[t], u.w, ws[4 * k4 + 3]);
+            }
+          }
+        }
+      }
+      if (q == p) {
+        sweep_col<false, 0>(ws, ws, c0, rs, W, Us, inv_u, wrow, crow, qscale);
+#pragma unroll
+        for (int k4 = 0; k4 < SUB / 4; ++k4)
+          reinterpret_cast<float4*>(wrow + c0)[k4] =
+              make_float4(ws[4 * k4], ws[4 * k4 + 1], ws[4 * k4 + 2], ws[4 * k4 + 3]);
+      }
+    }
+    __syncthreads();
+  }
+
+  // coalesced write-out: error rows as float4 (Err rows are 128 floats; the row
+  // state stride LDW = 132 floats keeps 16-byte alignment), codes 4 at a time
+  for (int idx = tid; idx < R * (B / 4); idx += QT) {
+    const int r = idx / (B / 4), c4 = idx - r * (B / 4);
+    if (r < rows_here && 4 * c4 < kb)
+      reinterpret_cast<float4*>(Err + (row0 + r) * B)[c4] =
+          reinterpret_cast<const float4*>(Wr + r * LDW)[c4];
+  }
+  // 4 codes per access: the staging rows (LDC = 132 bytes) are 4-byte aligned
+  const bool cvec = (b & 3) == 0 && (in & 3) == 0 && (kb & 3) == 0;
+  if (cvec) {
+    for (int idx = tid; idx < R * (B / 4); idx += QT) {
+      const int r = idx / (B / 4), c4 = idx - r * (B / 4);
+      if (r < rows_here && 4 * c4 < kb)
+        *reinterpret_cast<uint32_t*>(codes + (row0 + r) * in + b + 4 * c4) =
+            *reinterpret_cast<const uint32_t*>(Cs + r * LDC + 4 * c4);
+    }
+  } else {
+    for (int idx = tid; idx < R * B; idx += QT) {
+      const int r = idx / B, c = idx % B;
+      if (r < rows_here && c < kb) codes[(row0 + r) * in + b + c] = Cs[r * LDC + c];
+    }
+  }
+}
+
 }  // namespace
 
 // Column blocks of width <= 128 where each group start inside a block has its
@@ -257,6 +478,7 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
                    int8_t* codes, float* qscale, float* Err, DeviceStatus* st,
                    cudaStream_t stream) {
   static bool attr_set[64] = {};
+  static bool quarters_attr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   if (dev < 64 && !attr_set[dev]) {
@@ -268,6 +490,14 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
             cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
+  }
+  // with g % 128 == 0 no block holds a group start past its first column
+  const bool quartered = g % B == 0;
+  if (quartered && dev < 64 && !quarters_attr[dev]) {
+    if (cudaFuncSetAttribute(sweep_quarters_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kQuartersSmem) != cudaSuccess)
+      return PIQ_ERR_CUDA;
+    quarters_attr[dev] = true;
   }
   std::vector<std::pair<int64_t, int64_t>> blocks;
   block_partition(in, g, &blocks);
@@ -281,7 +511,9 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
       aligned = aligned && ((gs - b) % SUB == 0);
     note_launch();
     const cudaError_t le =
-        aligned ? launch_pdl(sweep_block_kernel<false>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
+        quartered ? launch_pdl(sweep_quarters_kernel, dim3(grid), dim3(QT), kQuartersSmem, stream,
+                               Wq, out, in, U, b, kb, bits, g, codes, qscale, Err, st)
+        : aligned ? launch_pdl(sweep_block_kernel<false>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
                              out, in, U, b, kb, bits, g, codes, qscale, Err, st)
                 : launch_pdl(sweep_block_kernel<true>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
                              out, in, U, b, kb, bits, g, codes, qscale, Err, st);
