@@ -95,13 +95,17 @@ def _round_clip(v: np.ndarray, qmax: int) -> np.ndarray:
 
 
 def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
-                   force: np.ndarray | None = None, log: bool = True):
+                   force: np.ndarray | None = None, log: bool = True, dtype=np.float64):
     """The listing's column loop on weights already in quantization order.
 
     Returns (codes int16 [out, in], scales [out, ngroups], v, err).
     ``force`` (int array [out, in], NO_FORCE where free) replaces the rounded
-    code at chosen sites: the teacher-forcing hook of the parity comparison."""
-    W = np.array(Wp, dtype=np.float64, copy=True)
+    code at chosen sites: the teacher-forcing hook of the parity comparison.
+    ``dtype`` is the working precision: float64 is the oracle; float32 runs the
+    same loop in the precision the benchmark spec fixes for the sweep, to measure
+    how far that arithmetic alone drifts from float64 (the parity tie window)."""
+    W = np.array(Wp, dtype=dtype, copy=True)
+    U = np.asarray(U, dtype=dtype)
     out, inp = W.shape
     qmax = 2 ** (bits - 1) - 1
     ngroups = -(-inp // g)
@@ -112,15 +116,15 @@ def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
     scale = None
     for j in range(inp):
         if j % g == 0:
-            scale = np.abs(W[:, j:j + g]).max(axis=1) / qmax
+            scale = np.abs(W[:, j:j + g]).max(axis=1) / dtype(qmax)
             scales[:, j // g] = scale
         live = scale > 0
-        v = np.where(live, W[:, j] / np.where(live, scale, 1.0), 0.0)
+        v = np.where(live, W[:, j] / np.where(live, scale, dtype(1.0)), dtype(0.0))
         c = _round_clip(v, qmax)
         if force is not None:
             f = force[:, j]
             c = np.where(f != NO_FORCE, f, c)
-        Q = c * scale
+        Q = c.astype(dtype) * scale
         e = (W[:, j] - Q) / U[j, j]
         W[:, j + 1:] -= np.outer(e, U[j, j + 1:])
         codes[:, j] = c.astype(np.int16)

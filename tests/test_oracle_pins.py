@@ -336,3 +336,23 @@ def test_hessian_sizes_printed_on_the_page():
     assert 28672 * 28672 * 4 == 3_288_334_336 and round(3_288_334_336 / 1e9, 2) == 3.29
     X = bf16_bits_from_f32(np.ones((2, 8), np.float32))
     assert O.hessian_ref(X).astype(np.float32).nbytes == 8 * 8 * 4
+
+
+def test_sweep_working_precision():
+    # float64 is the oracle (the default); the float32 mode runs the same loop in
+    # the sweep precision the benchmark spec fixes, and on the tiny layer it drifts
+    # from float64 by far less than the 1e-4 tie window, deciding every code the
+    # same way away from ties
+    from tests.parity import fp32_drift, tie_distance
+    W, X = make_weight(C1), make_x_bits(C1)
+    perm, U, _ = O.gptq_prepare_ref(O.hessian_ref(X), C1.damp, False)
+    Wp = W.astype(np.float64)[:, perm]
+    ref = O.gptq_sweep_ref(Wp, U, 4, 128)
+    c64 = O.gptq_sweep_ref(Wp, U, 4, 128, dtype=np.float64, log=False)[0]
+    assert np.array_equal(c64, ref[0])
+    c32, s32, v32, _ = O.gptq_sweep_ref(Wp, U, 4, 128, dtype=np.float32)
+    drift = fp32_drift(Wp, U, 4, 128, ref)
+    assert 0.0 < drift < 5e-5
+    for k in np.nonzero((c32 != ref[0]).any(axis=1))[0]:
+        j = int(np.argmax(c32[k] != ref[0][k]))  # first difference of the row: a tie
+        assert tie_distance(ref[2][k, j]) < 2 * drift
