@@ -184,6 +184,12 @@ const char* piq_phase_name(int i);
  * a monotone diagnostic counter. */
 uint64_t piq_kernel_launches(void);
 
+/* The last CUDA runtime error this library saw, as "<error name> in <where>"
+ * ("" if none): what lies behind a PIQ_ERR_CUDA return (a launch the runtime
+ * refused, or a kernel that failed, found when the call synchronized).
+ * Host-side, per process; static storage, overwritten by the next error. */
+const char* piq_last_cuda_error(void);
+
 /* piq_upper_factor without a caller workspace.  (The source pages have no
  * counterpart: this is a deployment variant of the damping + upper-factor step
  * above, same arguments minus the workspace, same results.)

@@ -39,12 +39,14 @@ from .error import x_to_f64
 NO_FORCE = -128  # sentinel in a ``force`` array: "this code is not forced"
 
 
-def hessian_ref(X, chunk: int = 8192) -> np.ndarray:
-    """H = X^T X in float64 (the listing's proxy Hessian), summed over row chunks."""
+def hessian_ref(X, chunk: int = 8192, dtype=np.float64) -> np.ndarray:
+    """H = X^T X (the listing's proxy Hessian), summed over row chunks.  float64
+    is the oracle; dtype=float32 accumulates in the FP32 the pages fix for H
+    (used only to measure that precision's drift, see gptq_sweep_ref)."""
     n, inp = X.shape
-    H = np.zeros((inp, inp), dtype=np.float64)
+    H = np.zeros((inp, inp), dtype=dtype)
     for r0 in range(0, n, chunk):
-        xc = x_to_f64(X[r0:r0 + chunk])
+        xc = x_to_f64(X[r0:r0 + chunk]).astype(dtype)
         H += xc.T @ xc
     return H
 
@@ -55,9 +57,9 @@ def act_order_perm_ref(H: np.ndarray) -> np.ndarray:
 
 
 def damped_ref(H: np.ndarray, damp: float):
-    """H + damp * mean(diag H) * I; returns (H_d, lambda)."""
+    """H + damp * mean(diag H) * I; returns (H_d, lambda), in H's precision."""
     lam = float(damp) * float(np.mean(np.diag(H)))
-    return H + lam * np.eye(H.shape[0]), lam
+    return H + H.dtype.type(lam) * np.eye(H.shape[0], dtype=H.dtype), lam
 
 
 def upper_factor_ref(Hd: np.ndarray) -> np.ndarray:
@@ -81,10 +83,12 @@ class GPTQResult:
     g: int
 
 
-def gptq_prepare_ref(H: np.ndarray, damp: float = 0.01, act_order: bool = False):
-    """Permutation (act-order), damping and the upper factor: (perm, U, lam)."""
+def gptq_prepare_ref(H: np.ndarray, damp: float = 0.01, act_order: bool = False, perm=None):
+    """Permutation (act-order), damping and the upper factor: (perm, U, lam), in
+    H's precision.  ``perm`` given: that quantization order instead."""
     inp = H.shape[0]
-    perm = act_order_perm_ref(H) if act_order else np.arange(inp, dtype=np.int64)
+    if perm is None:
+        perm = act_order_perm_ref(H) if act_order else np.arange(inp, dtype=np.int64)
     Hp = H[np.ix_(perm, perm)]
     Hd, lam = damped_ref(Hp, damp)
     return perm, upper_factor_ref(Hd), lam

@@ -74,6 +74,7 @@ SIGNATURES = {
                                       ctypes.POINTER(_c_int)]),
     "piq_phase_name": (ctypes.c_char_p, [_c_int]),
     "piq_kernel_launches": (ctypes.c_uint64, []),
+    "piq_last_cuda_error": (ctypes.c_char_p, []),
     "piq_upper_factor_noalloc": (_c_int, [_vp, _c_i64, _c_float, _vp, _vp,
                                           ctypes.POINTER(ctypes.c_double), _vp]),
 }
@@ -109,7 +110,14 @@ def status_string(status: int) -> str:
 
 def _check(rc: int, where: str):
     if rc != PIQ_OK:
+        if rc == PIQ_ERR_CUDA:
+            where = f"{where} [{load_library().piq_last_cuda_error().decode()}]"
         raise PiqError(rc, where)
+
+
+def last_cuda_error() -> str:
+    """The last CUDA runtime error the library saw ('' if none)."""
+    return load_library().piq_last_cuda_error().decode()
 
 
 def _stream(stream=None):

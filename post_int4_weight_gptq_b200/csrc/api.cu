@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -37,6 +38,13 @@ int device_info(DeviceInfo* out) {
 
 static std::atomic<uint64_t> g_launches{0};
 void note_launch(int count) { g_launches.fetch_add(static_cast<uint64_t>(count)); }
+
+static std::mutex g_err_mu;
+static char g_err_text[160] = "";
+void note_cuda_error(cudaError_t e, const char* where) {
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  snprintf(g_err_text, sizeof(g_err_text), "%s in %s", cudaGetErrorName(e), where);
+}
 
 namespace {
 
@@ -117,15 +125,20 @@ struct PhaseClock {
   }
 };
 
-int cuda_rc(cudaError_t e) { return e == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA; }
+int cuda_rc(cudaError_t e) {
+  if (e != cudaSuccess) note_cuda_error(e, "runtime call");
+  return e == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
 
 // Read the status word (and optional extra device bytes) after synchronizing.
 int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st) {
   DeviceStatus tmp;
-  if (cudaMemcpyAsync(&tmp, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, stream) !=
-      cudaSuccess)
+  cudaError_t e = cudaMemcpyAsync(&tmp, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    note_cuda_error(e, "stream synchronization (a kernel of this call failed)");
     return PIQ_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return PIQ_ERR_CUDA;
+  }
   if (host_st) *host_st = tmp;
   return tmp.code;
 }
@@ -592,6 +605,11 @@ int piq_last_phase_times(double* ms, int max_phases, int* n_phases) {
 }
 
 uint64_t piq_kernel_launches(void) { return g_launches.load(); }
+
+const char* piq_last_cuda_error(void) {
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  return g_err_text;
+}
 
 const char* piq_phase_name(int i) {
   std::lock_guard<std::mutex> lock(g_timing_mu);

@@ -144,6 +144,15 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// The last CUDA runtime error the library saw (piq_last_cuda_error reports it).
+void note_cuda_error(cudaError_t e, const char* where);
+// cudaGetLastError() == cudaSuccess, recording a failure.
+inline bool launch_ok(const char* where = "kernel launch") {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) note_cuda_error(e, where);
+  return e == cudaSuccess;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args... args) {
@@ -157,7 +166,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) note_cuda_error(e, "kernel launch (dependent)");
+  return e;
 }
 
 // bf16 bit patterns (round to nearest even on the way in)

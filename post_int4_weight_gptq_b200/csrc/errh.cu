@@ -92,14 +92,14 @@ int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uin
   split_vec_kernel<<<grid_1d(out * in / 4), 256, 0, stream>>>(
       reinterpret_cast<const float4*>(D), out * in / 4, reinterpret_cast<uint2*>(d_hi),
       reinterpret_cast<uint2*>(d_lo));
-  if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+  if (!launch_ok()) return PIQ_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in / 4, 256), 16)),
               static_cast<unsigned>(std::min<int64_t>(in, 65535)));
     note_launch();
     split_upper_half_kernel<<<grid, 256, 0, stream>>>(H, in, reinterpret_cast<uint2*>(h_hi),
                                                       reinterpret_cast<uint2*>(h_lo));
-    if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+    if (!launch_ok()) return PIQ_ERR_CUDA;
   }
   int rc = launch_err_dot(d_hi, d_lo, h_hi, h_lo, D, out, in, partials, st, stream);
   if (rc != PIQ_OK) return rc;

@@ -74,13 +74,15 @@ constexpr unsigned FULL = 0xffffffffu;
 // One warp factors a 16 x 16 SPD block, in registers.  Lane i < 16 holds row
 // i: on entry a[k] = A[i][k] (k <= i); on exit a[k] = L[i][k] (k <= i) and
 // rdiag = 1 / L_ii.  Lanes >= 16 carry zeros.  d is pivot J, already
-// broadcast; the next pivot is formed by lane J+1 from its own values and
-// broadcast before the rest of the column update, so the serial chain per
-// pivot is one shuffle, one rsqrt, one multiply and one FMA.  Template
-// recursion keeps register indices compile-time.
+// broadcast.  The next pivot is formed by lane J+1 from its own values and
+// shuffled first (the serial chain per pivot: one shuffle, one rsqrt, a
+// multiply and an FMA); the rest of column J reaches the lanes through shared
+// memory (one store, four broadcast float4 loads, double-buffered by pivot
+// parity) instead of fifteen shuffles.  Template recursion keeps register
+// indices compile-time.
 template <int J>
 __device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lane, bool& ok,
-                                           float d) {
+                                           float d, float* colbuf) {
   if constexpr (J < SP) {
     ok = ok && (d > 0.f);
     const float dd = d > 0.f ? d : 1.f;
@@ -90,13 +92,25 @@ __device__ __forceinline__ void chol16_col(float (&a)[SP], float& rdiag, int lan
     const float lij = (lane > J) ? a[J] * r : (lane == J ? ljj : 0.f);
     a[J] = lij;
     float dn = 0.f;
-    if constexpr (J + 1 < SP) dn = __shfl_sync(FULL, fmaf(-lij, lij, a[J + 1]), J + 1);
+    if constexpr (J + 1 < SP) {
+      dn = __shfl_sync(FULL, fmaf(-lij, lij, a[J + 1]), J + 1);
+      float* col = colbuf + (J & 1) * SP;
+      if (lane < SP) col[lane] = lij;
+      __syncwarp();
+      float lk[SP];
 #pragma unroll
-    for (int k = J + 1; k < SP; ++k) {
-      const float lkj = __shfl_sync(FULL, lij, k);
-      if (k <= lane) a[k] = fmaf(-lij, lkj, a[k]);
+      for (int q = (J + 1) / 4; q < SP / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(col)[q];
+        lk[4 * q] = v.x;
+        lk[4 * q + 1] = v.y;
+        lk[4 * q + 2] = v.z;
+        lk[4 * q + 3] = v.w;
+      }
+#pragma unroll
+      for (int k = J + 1; k < SP; ++k)
+        if (k <= lane) a[k] = fmaf(-lij, lk[k], a[k]);
     }
-    chol16_col<J + 1>(a, rdiag, lane, ok, dn);
+    chol16_col<J + 1>(a, rdiag, lane, ok, dn, colbuf);
   }
 }
 
@@ -174,6 +188,7 @@ __global__ void __launch_bounds__(CI_THREADS)
   float* LT = Xs + NB * SLD;     // [SP][SLD] current panel, transposed
   float* Tm = LT + SP * SLD;     // [64][TLD] merge temp
   float* rinv = Tm + 64 * TLD;   // [NB] reciprocal pivots
+  float* colbuf = rinv + NB;     // [2][SP] pivot-column broadcast (16-byte aligned)
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
@@ -213,7 +228,7 @@ __global__ void __launch_bounds__(CI_THREADS)
 #pragma unroll
         for (int k = 0; k < SP; ++k) a[k] = 0.f;
       }
-      chol16_col<0>(a, rdiag, lane, ok, __shfl_sync(FULL, a[0], 0));
+      chol16_col<0>(a, rdiag, lane, ok, __shfl_sync(FULL, a[0], 0), colbuf);
       if (!ok && lane == 0) {
         bad = 1;
         set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));
@@ -419,7 +434,7 @@ __global__ void identity_perm_kernel(int64_t in, int32_t* perm, int32_t* invperm
   }
 }
 
-constexpr int kCholSmem = (2 * NB * SLD + SP * SLD + 64 * TLD + NB) * sizeof(float);
+constexpr int kCholSmem = (2 * NB * SLD + SP * SLD + 64 * TLD + NB + 2 * SP) * sizeof(float);
 
 // Floats of the pair scratch of the level-by-level inverse: max over levels of
 // (pairs at that level) * s * s.
@@ -464,7 +479,7 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     note_launch();
     build_rev_kernel<<<grid, dim3(32, 8), 0, stream>>>(H, in, perm, lam, P);
   }
-  if (cudaGetLastError() != cudaSuccess) return PIQ_ERR_CUDA;
+  if (!launch_ok()) return PIQ_ERR_CUDA;
 
   // 3. Cholesky, panel by panel; diagonal inverses land in X
   for (int64_t k0 = 0; k0 < in; k0 += NB) {
@@ -525,7 +540,7 @@ int run_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
     else
       extract_u_kernel<<<grid, 256, 0, stream>>>(X, in, U);
   }
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 int launch_act_order_perm(const double* sumsq, int64_t in, int32_t* perm, int32_t* invperm,
@@ -533,14 +548,14 @@ int launch_act_order_perm(const double* sumsq, int64_t in, int32_t* perm, int32_
   note_launch();
   act_order_rank_kernel<<<static_cast<unsigned>(ceil_div(in, 256)), 256, 0, stream>>>(
       sumsq, in, perm, invperm);
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 int launch_identity_perm(int64_t in, int32_t* perm, int32_t* invperm, cudaStream_t stream) {
   note_launch();
   identity_perm_kernel<<<static_cast<unsigned>(ceil_div(in, 256)), 256, 0, stream>>>(in, perm,
                                                                                      invperm);
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 }  // namespace piq

@@ -513,7 +513,7 @@ unsigned grid_for(int64_t work, int threads) {
   return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, 16LL * sms)));
 }
 
-int last_error() { return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA; }
+int last_error() { return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA; }
 
 }  // namespace
 

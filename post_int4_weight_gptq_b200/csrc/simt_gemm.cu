@@ -150,7 +150,7 @@ int launch_one(int M, int N, int K, float alpha, const float* A, int64_t lda, co
   note_launch();
   simt_gemm_kernel<TB, MODE><<<grid, 256, 0, stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C,
                                                        ldc, bt, st);
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 }  // namespace

@@ -120,6 +120,10 @@ constexpr int n_segments() {
   return EPI == EPI_DOT ? 3 : 1;
 }
 
+// One CTA of 320 threads per SM.  Ten warps put three on some schedulers, so a
+// thread gets at most 168 registers (the H build keeps a 128-float running sum
+// per epilogue thread).  Tiles go round-robin, so all CTAs sweep the same sample
+// range at the same time and X streams through L2 once per wave of tiles.
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -435,9 +439,12 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   auto kern = tc_gemm_kernel<A_MN, B_MN, EPI>;
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) {
+      note_cuda_error(e, "tensor-core GEMM shared-memory attribute");
       return PIQ_ERR_CUDA;
+    }
     attr_set[dev] = true;
   }
   DeviceInfo info;
@@ -597,7 +604,7 @@ int launch_reduce_sum(const double* partials, int64_t per, int batch, double* ou
   if (per < 1 || batch < 1) return PIQ_ERR_INVALID_ARG;
   note_launch();
   reduce_partials_kernel<<<batch, RP_THREADS, 0, stream>>>(partials, per, out);
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 int launch_reduce_partials(const double* partials, int64_t n, int64_t rows, int batch,

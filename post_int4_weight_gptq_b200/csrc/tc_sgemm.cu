@@ -473,7 +473,7 @@ int launch_tc_sgemm(int M, int N, int K, float alpha, const float* A, int64_t ld
   if (launch_pdl(tf32x3_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, ma, mb, mc,
                  p) != cudaSuccess)
     return PIQ_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
 int launch_gemm_f32(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
