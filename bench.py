@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one syrk_xtx launch on the
 # 131072 x 4096 workload, from one ncu capture of the current kernel; to be retaken (or set to
 # None) whenever that kernel changes.
-SYRK_TRAFFIC_BYTES = 1.88e9 + 21.69e6
+SYRK_TRAFFIC_BYTES = 1.93e9 + 21.82e6
 
 
 def load_peaks():
@@ -360,7 +360,7 @@ def run_ours(args):
     peak_key = "bf16_tflops_sustained" if capped else "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     ach_h = flops_h / (t_h / 1e3) / 1e12
-    roof = {"kernel": "syrk_xtx (tcgen05 H = X^T X, 4096-sample chunks summed in registers)",
+    roof = {"kernel": "syrk_xtx (tcgen05 H = X^T X, 1024-sample chunks summed in registers)",
             "bound": "tensor", "achieved": ach_h, "peak": peak, "unit": "TFLOP/s",
             "frac": ach_h / peak,
             "traffic": args.traffic if args.traffic is not None else (

@@ -73,7 +73,7 @@ int piq_hessian_bytes(int64_t in, size_t* bytes);
  *   H  device fp32 [in, in] row-major.  Every element on or above the diagonal
  *      is written (H[i][j], j >= i); elements below the diagonal are
  *      unspecified.  BF16 products, FP32 accumulation on the tensor cores in
- *      chunks of 4096 samples; the chunks are added into H in sample order
+ *      chunks of 1024 samples; the chunks are added into H in sample order
  *      (FP32), so the result is deterministic.
  * n >= 1, in >= 8, in % 8 == 0; X and H 16-byte aligned (else
  * PIQ_ERR_INVALID_ARG). */

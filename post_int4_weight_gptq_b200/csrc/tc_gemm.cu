@@ -55,9 +55,9 @@ constexpr int GROUP_M = 16;                     // raster group (err_sumsq)
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 // Samples per TMEM accumulation of H.  The relative error of the tensor-core
 // fp32 sum grows about linearly with the number of MMAs accumulated in place;
-// 4096 samples (256 MMAs of k = 16) keep it near 2e-5 of sqrt(H_ii H_jj)
-// whatever n is.
-constexpr int KC = 4096;
+// 1024 samples (64 MMAs of k = 16) keep it near 5e-6 of sqrt(H_ii H_jj)
+// whatever n is, and the chunks' sum in registers costs the MMAs nothing.
+constexpr int KC = 1024;
 
 enum { EPI_SYRK = 0, EPI_SUMSQ = 1, EPI_DOT = 2 };
 
