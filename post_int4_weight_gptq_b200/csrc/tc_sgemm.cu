@@ -8,7 +8,11 @@
 // top 19 bits of a 32-bit operand, so the TMA-landed tile itself serves as hi
 // and only lo is written; the tile is accumulated in TMEM as
 // A_hi B_hi + A_hi B_lo + A_lo B_hi  (lo is itself cut to 19 bits by the
-// tensor core, and the dropped A_lo B_lo is ~2^-20 of the product).
+// tensor core, and the dropped A_lo B_lo is ~2^-20 of the product).  A_hi B_hi
+// and the two cross terms go to separate accumulators, added in the epilogue:
+// the fp32 TMEM sum truncates relative to its own magnitude, so the small
+// terms would otherwise lose their precision against the large one (this
+// matters over the hundreds of panel updates of a 28672-wide factor).
 //
 // C = alpha A op(B) + beta C, all fp32 row-major: A [M][K] (K-major tiles), B
 // [K][N] (MN-major tiles) or, with trans_b, [N][K] (K-major).  Modes: 0 plain;
@@ -18,7 +22,7 @@
 //
 // Warp roles (320 threads): warp 0 lane 0 issues TMA loads of fp32 tiles into a
 // 3-stage ring; warps 6..9 write the lo part of each landed tile; warp 1 lane 0
-// issues the MMAs; warps 2..5 drain one of two 128-column accumulators.  Every
+// issues the MMAs; warps 2..5 drain one of two accumulator pairs.  Every
 // wait is bounded; no multicast loads.
 #include <cuda.h>
 
@@ -37,7 +41,8 @@ constexpr int STAGES = 3;
 constexpr int TILE_BYTES = BM * BK * 4;      // 16 KB (A and B tiles are the same size)
 constexpr int STAGE_BYTES = 4 * TILE_BYTES;  // A_hi, B_hi, A_lo, B_lo
 constexpr int THREADS = 320;
-constexpr int TMEM_COLS = 2 * BN;
+// two buffers x (hi.hi accumulator, cross-term accumulator) of BN columns
+constexpr int TMEM_COLS = 4 * BN;
 constexpr int TR_BYTES = 4 * 2 * 32 * 32 * 4;  // epilogue staging: 2 per epilogue warp
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + TR_BYTES + 1024 + 256;
 
@@ -248,7 +253,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 13)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        // hi.hi and the cross terms accumulate apart: the small terms then keep
+        // their precision (the fp32 TMEM sum truncates relative to its own size)
+        const uint32_t d_big = tmem_base + static_cast<uint32_t>(buf * 2 * BN);
+        const uint32_t d_small = d_big + BN;
         bool first = true;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int s = it % STAGES;
@@ -276,9 +284,9 @@ __global__ void __launch_bounds__(THREADS, 1)
               bh = smem_desc(b_hi + kk * 1024, BK * 128, 512, kLayoutSw128Base32);
               bl = smem_desc(b_lo + kk * 1024, BK * 128, 512, kLayoutSw128Base32);
             }
-            umma_tf32(d_tmem, al, bh, idesc, first ? 0u : 1u);
-            umma_tf32(d_tmem, ah, bl, idesc, 1u);
-            umma_tf32(d_tmem, ah, bh, idesc, 1u);
+            umma_tf32(d_small, al, bh, idesc, first ? 0u : 1u);
+            umma_tf32(d_small, ah, bl, idesc, 1u);
+            umma_tf32(d_big, ah, bh, idesc, first ? 0u : 1u);
             first = false;
           }
           umma_commit(&empty[s]);
@@ -299,13 +307,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 15)) break;
       tc_fence_after();
       const bool has_k = ti.kb1 > ti.kb0;
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(buf * 2 * BN);
       const int row0 = ti.mt * BM + q * 32;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);  // lane = row, v[i] = column i
+        {
+          float vs[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);         // hi.hi; lane = row, v[i] = column i
+          tmem_ld_32x32b_x32(taddr + BN + c * 32, vs);   // cross terms
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += vs[i];
+        }
         // 32 x 32 staging tile in the TMA 128-byte swizzle: 16-byte chunk k of
         // row r sits at chunk k ^ (r % 8); double-buffered per warp
         float* sb = stg + (chunk & 1) * 1024;
