@@ -16,6 +16,8 @@ Sources (web pages on GPTQ/AWQ; cited by page title and section):
   (uplatz.com), sections 2.1-2.3 and 3.2: the same objective written as
   ||W_q X - W X||_F, group size, act-order, the Babai nearest-plane reading,
   and y = (W s)(X / s).
+* "GPTQ versus AWQ objectives", the serving decision list: AWQ's scaling and
+  GPTQ's rounding compose (``compose.py``).
 
 Every function works in float64 on exact copies of the inputs (bfloat16 X values
 are exact in float64).  Where the pages leave a step open, the reading taken is
@@ -27,11 +29,13 @@ from .gptq import (GPTQResult, act_order_perm_ref, block_partition_ref, damped_r
 from .awq import AWQResult, awq_ref, awq_scales_ref, channel_mean_abs_ref, group_rtn_ref
 from .pack import dequant_ref, g_idx_ref, pack_ref, unpack_ref
 from .error import output_error_ref, x_to_f64
+from .compose import awq_gptq_dequant_ref, awq_gptq_ref, awq_then_gptq_ref, scaled_layer_ref
 
 __all__ = [
     "GPTQResult", "act_order_perm_ref", "block_partition_ref", "damped_ref",
     "gptq_prepare_ref", "gptq_ref", "gptq_ref_blocked", "gptq_sweep_ref", "hessian_ref",
     "rtn_ref", "upper_factor_ref", "AWQResult", "awq_ref", "awq_scales_ref",
     "channel_mean_abs_ref", "group_rtn_ref", "dequant_ref", "g_idx_ref", "pack_ref",
-    "unpack_ref", "output_error_ref", "x_to_f64",
+    "unpack_ref", "output_error_ref", "x_to_f64", "awq_gptq_dequant_ref", "awq_gptq_ref",
+    "awq_then_gptq_ref", "scaled_layer_ref",
 ]
