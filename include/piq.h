@@ -147,6 +147,32 @@ int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
                      float* s, uint32_t* qweight, uint16_t* scales, double* err_per_alpha,
                      void* workspace, size_t ws_bytes, void* stream);
 
+/* AWQ's scaling first, GPTQ's rounding after ("GPTQ versus AWQ objectives",
+ * the serving decision list: at 3 bits or similarly aggressive targets the two
+ * compose; uplatz.com report, section 3.2: y = (W s)(X / s) is the same layer).
+ * GPTQ, exactly as gptq_quantize_layer, of the layer W' = W diag(s) with
+ * calibration inputs X' = X diag(1/s):
+ *   H' = diag(1/s) X^T X diag(1/s) (X is not rescaled or re-rounded: H is
+ *   built from X and scaled in FP64), act-order by decreasing diag(H'),
+ *   damping and factor of H', the sweep over W diag(s) (fp32 products).
+ *   s_ch       device fp32 [in], 16-byte aligned, every s_j finite and > 0
+ *              (typically the s awq_search_layer returned).  A bad s_j is found
+ *              on the device: PIQ_ERR_INVALID_ARG.  Read only.
+ *   qweight/scales quantize W' (as awq_search_layer's do), so the layer's
+ *              weight is code * scale / s_j.
+ *   perm/g_idx as gptq_quantize_layer (perm: order of the scaled layer).
+ *   out_err    host double, may be NULL:
+ *              ||X W^T - X What^T||^2, What = code * fp16(scale) / s_j, taken
+ *              through H' as sum_r D'_r H' D'_r^T with D' = W' - code * fp16(scale)
+ *              (X' D'^T = X (W - What)^T).
+ * Workspace: piq_gptq_workspace_bytes(out, in, n, act_order).  Other
+ * arguments, layout, errors and synchronization as gptq_quantize_layer. */
+int awq_gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
+                            int64_t n, const float* s_ch, int bits, int g, float damp,
+                            int act_order, uint32_t* qweight, uint16_t* scales, int32_t* perm,
+                            int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                            void* stream);
+
 /* Plain group round-to-nearest (the "round-to-nearest" column of the toy table
  * in "GPTQ versus AWQ objectives"): every scale from the original weights, no
  * error feedback.  Same outputs and format as GPTQ with natural order.

@@ -13,6 +13,8 @@ Methods (web pages on the subject, cited by title and section):
   next" (act-order, damping).
 * AWQ  - same page, AWQ paragraph: per-channel scales mean|x_j|^alpha, one
   alpha per layer by grid search on the calibration output error.
+* AWQ then GPTQ - same page, the serving decision list: the two compose, AWQ's
+  scaling first and GPTQ's rounding after (GPTQ on W diag(s), X diag(1/s)).
 """
 from __future__ import annotations
 
@@ -62,6 +64,10 @@ SIGNATURES = {
                                   ctypes.POINTER(ctypes.c_float), _c_int,
                                   ctypes.POINTER(ctypes.c_float), _vp, _vp, _vp,
                                   ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t, _vp]),
+    "awq_gptq_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _vp, _c_int, _c_int,
+                                         _c_float, _c_int, _vp, _vp, _vp, _vp,
+                                         ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
+                                         _vp]),
     "piq_rtn_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_size_p]),
     "piq_rtn_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp,
                                         ctypes.c_size_t, _vp]),
@@ -256,6 +262,42 @@ def awq_search_layer(W, X, bits=4, g=128, alpha_grid=AWQ_DEFAULT_GRID, stream=No
                                 ctypes.byref(best), _ptr(s), _ptr(qweight), _ptr(scales), errs,
                                 _ptr(ws), ws.numel(), _stream(stream)), "awq_search_layer")
     return AWQOutput(best.value, s, qweight, scales, list(errs))
+
+
+def awq_gptq_quantize_layer(W, X, s, bits=4, g=128, damp=0.01, act_order=False,
+                            with_error=True, stream=None, workspace=None, out=None):
+    """GPTQ of the AWQ-scaled layer W diag(s) on inputs X diag(1/s).  The
+    scales quantize W diag(s): the layer's weight is code * scale / s_j."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    _need(X, torch.bfloat16, "X")
+    _need(s, torch.float32, "s")
+    rows, inp = W.shape
+    n = X.shape[0]
+    if X.shape[1] != inp or s.numel() != inp:
+        raise ValueError("W, X and s disagree on the input dimension")
+    dev = W.device
+    if out is None:
+        out = GPTQOutput(torch.empty(rows, inp // 8, dtype=torch.int32, device=dev),
+                         torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev), None)
+    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order), dev, workspace)
+    err = ctypes.c_double(0.0)
+    _check(lib.awq_gptq_quantize_layer(_ptr(W), rows, inp, _ptr(X), n, _ptr(s), bits, g,
+                                       float(damp), int(bool(act_order)), _ptr(out.qweight),
+                                       _ptr(out.scales), _ptr(out.perm), _ptr(out.g_idx),
+                                       ctypes.byref(err) if with_error else None, _ptr(ws),
+                                       ws.numel(), _stream(stream)), "awq_gptq_quantize_layer")
+    return out._replace(err=err.value if with_error else None)
+
+
+def awq_then_gptq_layer(W, X, bits=4, g=128, damp=0.01, act_order=False,
+                        alpha_grid=AWQ_DEFAULT_GRID, stream=None):
+    """AWQ's search picks alpha* and s, then GPTQ rounds W diag(s):
+    (AWQOutput, GPTQOutput); two library calls on the same stream."""
+    a = awq_search_layer(W, X, bits, g, alpha_grid, stream=stream)
+    return a, awq_gptq_quantize_layer(W, X, a.s, bits, g, damp, act_order, stream=stream)
 
 
 def rtn_quantize_layer(W, bits=4, g=128, stream=None, workspace=None):

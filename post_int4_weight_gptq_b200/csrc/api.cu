@@ -293,6 +293,81 @@ int check_ws(void* ws, size_t have, size_t need) {
   return have >= need ? PIQ_OK : PIQ_ERR_WORKSPACE_TOO_SMALL;
 }
 
+size_t gptq_ws_bytes(int64_t out, int64_t in, int64_t n, int act_order) {
+  Carver c(nullptr);
+  carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  return c.bytes();
+}
+
+// GPTQ of one layer; with s_ch, of the scaled layer (W diag(s), X diag(1/s)):
+// H' = diag(1/s) X^T X diag(1/s), the act-order key diag(H'), the sweep over
+// W diag(s), and the error of What = code * scale / s through H' with
+// D' = W diag(s) - code * fp16(scale), since X' D'^T = X (W - What)^T.
+int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
+               const float* s_ch, int bits, int g, float damp, int act_order, uint32_t* qweight,
+               uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err, void* workspace,
+               size_t ws_bytes, cudaStream_t s) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || X == nullptr || qweight == nullptr || scales == nullptr || n < 1 ||
+      !(damp >= 0.f) || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
+    return PIQ_ERR_INVALID_ARG;
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  PIQ_TRY(check_ws(workspace, ws_bytes, gptq_ws_bytes(out, in, n, act_order)));
+  Carver c(workspace);
+  GptqWs w = carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  PhaseClock clk(0, s);
+
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  // 1. H = X^T X on the tensor cores (scaled to H' for the AWQ-scaled layer)
+  PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
+  if (s_ch) PIQ_TRY(launch_scale_upper(w.H, in, s_ch, w.st, s));
+  clk.mark();
+  // 2. quantization order
+  const int32_t* qperm = nullptr;
+  const int32_t* qinv = nullptr;
+  if (act_order) {
+    PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), nullptr, w.sumsq, s));
+    if (s_ch) PIQ_TRY(launch_scale_sumsq(w.sumsq, in, s_ch, s));
+    PIQ_TRY(launch_act_order_perm(w.sumsq, in, w.perm, w.invperm, s));
+    qperm = w.perm;
+    qinv = w.invperm;
+  }
+  if (perm) {
+    if (act_order)
+      PIQ_TRY(cuda_rc(cudaMemcpyAsync(perm, w.perm, sizeof(int32_t) * in, cudaMemcpyDeviceToDevice, s)));
+    else
+      PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
+  }
+  clk.mark();
+  // 3. damping + U (H is kept; U goes over the factor's own scratch)
+  float* U = w.fwork;
+  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, U, w.fwork, w.st, s));
+  clk.mark();
+  // 4. blocked sweep on the permuted (and scaled) copy
+  PIQ_TRY(launch_gather_columns(W, out, in, qperm, s_ch, w.Wq, s));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, w.Err, w.st, s));
+  clk.mark();
+  // 5. pack (+ D = W diag(s) - What' for the error)
+  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, s_ch, qweight, scales,
+                      nullptr, out_err ? w.dW : nullptr, g_idx, s));
+  clk.mark();
+  // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from the H built in step 1
+  //    (scratch: the sweep copy, and the factor's inverse region after U)
+  if (out_err)
+    PIQ_TRY(run_error_via_h(w.dW, out, in, w.H, reinterpret_cast<uint16_t*>(w.Wq),
+                            reinterpret_cast<uint16_t*>(w.fwork + in * in), w.partials, w.err,
+                            w.st, s));
+  clk.mark();
+  double e = 0.0;
+  if (out_err)
+    PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
+  const int rc = finish_call(w.st, s, nullptr);
+  clk.finish();
+  if (out_err) *out_err = e;
+  return rc;
+}
+
 }  // namespace
 }  // namespace piq
 
@@ -385,9 +460,7 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
 
 int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int act_order, size_t* bytes) {
   if (bytes == nullptr || out < 1 || in < 1 || n < 1) return PIQ_ERR_INVALID_ARG;
-  Carver c(nullptr);
-  carve_gptq(c, out, in, n, act_order ? 1 : 0);
-  *bytes = c.bytes();
+  *bytes = gptq_ws_bytes(out, in, n, act_order);
   return PIQ_OK;
 }
 
@@ -395,66 +468,18 @@ int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t*
                         int bits, int g, float damp, int act_order, uint32_t* qweight,
                         uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,
                         void* workspace, size_t ws_bytes, void* stream) {
-  PIQ_TRY(check_layer(out, in, bits, g));
-  if (W == nullptr || X == nullptr || qweight == nullptr || scales == nullptr || n < 1 ||
-      !(damp >= 0.f) || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
-    return PIQ_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  DeviceInfo info;
-  PIQ_TRY(device_info(&info));
-  size_t need = 0;
-  piq_gptq_workspace_bytes(out, in, n, act_order, &need);
-  PIQ_TRY(check_ws(workspace, ws_bytes, need));
-  Carver c(workspace);
-  GptqWs w = carve_gptq(c, out, in, n, act_order ? 1 : 0);
-  PhaseClock clk(0, s);
+  return gptq_layer(W, out, in, X, n, nullptr, bits, g, damp, act_order, qweight, scales, perm,
+                    g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
 
-  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
-  // 1. H = X^T X on the tensor cores
-  PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
-  clk.mark();
-  // 2. quantization order
-  const int32_t* qperm = nullptr;
-  const int32_t* qinv = nullptr;
-  if (act_order) {
-    PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), nullptr, w.sumsq, s));
-    PIQ_TRY(launch_act_order_perm(w.sumsq, in, w.perm, w.invperm, s));
-    qperm = w.perm;
-    qinv = w.invperm;
-  }
-  if (perm) {
-    if (act_order)
-      PIQ_TRY(cuda_rc(cudaMemcpyAsync(perm, w.perm, sizeof(int32_t) * in, cudaMemcpyDeviceToDevice, s)));
-    else
-      PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
-  }
-  clk.mark();
-  // 3. damping + U (H is kept; U goes over the factor's own scratch)
-  float* U = w.fwork;
-  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, U, w.fwork, w.st, s));
-  clk.mark();
-  // 4. blocked sweep on the permuted copy
-  PIQ_TRY(launch_gather_columns(W, out, in, qperm, w.Wq, s));
-  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, w.Err, w.st, s));
-  clk.mark();
-  // 5. pack (+ D = W - What for the error)
-  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, qweight, scales, nullptr,
-                      out_err ? w.dW : nullptr, g_idx, s));
-  clk.mark();
-  // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from the H built in step 1
-  //    (scratch: the sweep copy, and the factor's inverse region after U)
-  if (out_err)
-    PIQ_TRY(run_error_via_h(w.dW, out, in, w.H, reinterpret_cast<uint16_t*>(w.Wq),
-                            reinterpret_cast<uint16_t*>(w.fwork + in * in), w.partials, w.err,
-                            w.st, s));
-  clk.mark();
-  double e = 0.0;
-  if (out_err)
-    PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
-  const int rc = finish_call(w.st, s, nullptr);
-  clk.finish();
-  if (out_err) *out_err = e;
-  return rc;
+int awq_gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
+                            int64_t n, const float* s_ch, int bits, int g, float damp,
+                            int act_order, uint32_t* qweight, uint16_t* scales, int32_t* perm,
+                            int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  if (s_ch == nullptr || !aligned16(s_ch)) return PIQ_ERR_INVALID_ARG;
+  return gptq_layer(W, out, in, X, n, s_ch, bits, g, damp, act_order, qweight, scales, perm,
+                    g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int piq_awq_workspace_bytes(int64_t out, int64_t in, int64_t n, int n_alpha, size_t* bytes) {
@@ -504,8 +529,8 @@ int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
   // 4. first minimum, re-quantize at it, pack
   PIQ_TRY(launch_argmin(w.err, n_alpha, w.alphas, w.best, w.best_alpha, s));
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, w.s_table, w.best, w.codes, w.qscale, s_out, s));
-  PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
-                      nullptr, nullptr, nullptr, s));
+  PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
+                      scales, nullptr, nullptr, nullptr, s));
   clk.mark();
   double errs[64];
   float ba = 0.f;
@@ -542,8 +567,8 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
   Carver c(workspace);
   RtnWs w = carve_rtn(c, out, in);
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, nullptr, nullptr, w.codes, w.qscale, nullptr, s));
-  return launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, qweight, scales,
-                     nullptr, nullptr, nullptr, s);
+  return launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
+                     scales, nullptr, nullptr, nullptr, s);
 }
 
 int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t* bytes) {

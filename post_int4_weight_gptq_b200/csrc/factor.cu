@@ -400,16 +400,22 @@ __global__ void extract_u_vec_kernel(const float* X, int64_t in, float* U) {
 
 // rank of each column by decreasing sumsq (exact FP64 column sums of squares,
 // i.e. diag(X^T X)); equal values keep index order.
+// A NaN key (NaN or infinite inputs) ranks as -inf, so that (key, index) stays
+// a strict total order and perm is always a permutation of 0..in-1.
+__device__ __forceinline__ double rank_key(double x) {
+  return x == x ? x : __longlong_as_double(static_cast<long long>(0xfff0000000000000ULL));
+}
+
 __global__ void act_order_rank_kernel(const double* d, int64_t in, int32_t* perm,
                                       int32_t* invperm) {
   __shared__ double tile[1024];
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const double di = i < in ? d[i] : 0.0;
+  const double di = i < in ? rank_key(d[i]) : 0.0;
   int64_t rank = 0;
   for (int64_t j0 = 0; j0 < in; j0 += 1024) {
     __syncthreads();
     for (int t = threadIdx.x; t < 1024; t += blockDim.x)
-      tile[t] = (j0 + t < in) ? d[j0 + t] : 0.0;
+      tile[t] = (j0 + t < in) ? rank_key(d[j0 + t]) : 0.0;
     __syncthreads();
     const int lim = static_cast<int>(std::min<int64_t>(1024, in - j0));
     if (i < in) {

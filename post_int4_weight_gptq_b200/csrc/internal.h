@@ -106,13 +106,21 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
 int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, int splits,
                     double* mean_abs, double* sumsq, cudaStream_t stream);
 int colstats_splits(int64_t n, int64_t in);
+// Wq[r][p] = W[r][perm[p]] * cs[perm[p]]; perm and cs may be NULL.
 int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
-                          float* Wq, cudaStream_t stream);
-// dW (bf16) and dW32 (fp32), when given, receive W0 - code * fp16(scale).
+                          const float* cs, float* Wq, cudaStream_t stream);
+// dW (bf16) and dW32 (fp32), when given, receive W0 diag(cs) - code * fp16(scale)
+// (cs == NULL: W0 - code * fp16(scale)).
 int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
-                int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
+                int64_t in, int bits, int g, const float* W0, const float* cs, uint32_t* qweight,
                 uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
                 cudaStream_t stream);
+// H = diag(1/s) H diag(1/s) on the upper triangle, in place; a non-finite or
+// non-positive s_k sets PIQ_ERR_INVALID_ARG (where = k) in st.
+int launch_scale_upper(float* H, int64_t in, const float* s, DeviceStatus* st,
+                       cudaStream_t stream);
+// sumsq[j] /= s_j^2 (FP64).
+int launch_scale_sumsq(double* sumsq, int64_t in, const float* s, cudaStream_t stream);
 int launch_awq_scale_table(const double* mean_abs, int64_t in, const float* alphas_dev,
                            int n_alpha, float* s_table, cudaStream_t stream);
 int launch_awq_delta(const float* W, int64_t out, int64_t in, int bits, int g,

@@ -12,6 +12,10 @@
 //   pack          codes -> uint32 nibbles, fp32 -> fp16 scales, act-order
 //                 column un-permutation and g_idx, and D = W - code * fp16(scale)
 //                 (bf16) for the output-error GEMM, in one pass.
+//   scale_upper   H' = diag(1/s) H diag(1/s) in place, the proxy Hessian of the
+//                 AWQ-scaled inputs X diag(1/s) (AWQ's scaling first, GPTQ's
+//                 rounding after: the serving decision list of "GPTQ versus AWQ
+//                 objectives"); also checks s.
 #include <algorithm>
 
 #include "internal.h"
@@ -96,35 +100,87 @@ __global__ void colstats_finish_kernel(const double* __restrict__ part, int64_t 
 }
 
 // --------------------------------------------------------------------- gather
-// Wq[r][p] = W[r][perm[p]] (perm == NULL: a copy), four positions per thread
-// (in % 4 == 0 and 16-byte aligned rows; the launcher checks).
+// Wq[r][p] = W[r][perm[p]] * cs[perm[p]] (perm == NULL: identity; cs == NULL:
+// no scaling), four positions per thread (in % 4 == 0 and 16-byte aligned
+// rows, perm and cs; the launcher checks).  The product is the same fp32
+// multiply pack_kernel makes, so both see the same W diag(s).
 __global__ void gather_columns_kernel(const float* __restrict__ W, int64_t out, int64_t in,
-                                      const int32_t* __restrict__ perm, float* __restrict__ Wq) {
+                                      const int32_t* __restrict__ perm,
+                                      const float* __restrict__ cs, float* __restrict__ Wq) {
   const int64_t total4 = out * in / 4;
   const int64_t in4 = in / 4;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total4;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     float4 v;
+    const int64_t r = idx / in4, p = (idx - r * in4) * 4;
+    int4 c = make_int4(static_cast<int>(p), static_cast<int>(p + 1), static_cast<int>(p + 2),
+                       static_cast<int>(p + 3));
     if (perm == nullptr) {
       v = __ldg(reinterpret_cast<const float4*>(W) + idx);
     } else {
-      const int64_t r = idx / in4, p = (idx - r * in4) * 4;
-      const int4 c = __ldg(reinterpret_cast<const int4*>(perm + p));
+      c = __ldg(reinterpret_cast<const int4*>(perm + p));
       const float* wr = W + r * in;
       v = make_float4(__ldg(wr + c.x), __ldg(wr + c.y), __ldg(wr + c.z), __ldg(wr + c.w));
+    }
+    if (cs != nullptr) {
+      if (perm == nullptr) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(cs + p));
+        v = make_float4(v.x * t.x, v.y * t.y, v.z * t.z, v.w * t.w);
+      } else {
+        v = make_float4(v.x * __ldg(cs + c.x), v.y * __ldg(cs + c.y), v.z * __ldg(cs + c.z),
+                        v.w * __ldg(cs + c.w));
+      }
     }
     reinterpret_cast<float4*>(Wq)[idx] = v;
   }
 }
 
+// -------------------------------------------------------------- scale_upper
+// H[k][j] /= s_k s_j for the 4-column chunks that hold j >= k (the valid upper
+// triangle; the rest is never read), one rounding from FP64.  A block with
+// blockIdx.x == 0 checks s_k (finite, > 0) for each of its rows.
+__global__ void scale_upper_kernel(float* __restrict__ H, int64_t in, const float* __restrict__ s,
+                                   DeviceStatus* st) {
+  const int64_t in4 = in >> 2;
+  for (int64_t k = blockIdx.y; k < in; k += gridDim.y) {
+    const float sk = s[k];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && !(sk > 0.f && sk <= 3.4028235e38f))
+      set_status(st, PIQ_ERR_INVALID_ARG, static_cast<int>(k));
+    const double rk = 1.0 / static_cast<double>(sk);
+    float4* row = reinterpret_cast<float4*>(H + k * in);
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    for (int64_t t = (k >> 2) + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+         t < in4; t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const float4 h = row[t];
+      const float4 sj = __ldg(s4 + t);
+      row[t] = make_float4(static_cast<float>(static_cast<double>(h.x) * rk / sj.x),
+                           static_cast<float>(static_cast<double>(h.y) * rk / sj.y),
+                           static_cast<float>(static_cast<double>(h.z) * rk / sj.z),
+                           static_cast<float>(static_cast<double>(h.w) * rk / sj.w));
+    }
+  }
+}
+
+// sumsq[j] /= s_j^2 in FP64 (s_j^2 is exact there): diag of the scaled Hessian,
+// the act-order key of the scaled layer.
+__global__ void scale_sumsq_kernel(double* __restrict__ sumsq, int64_t in,
+                                   const float* __restrict__ s) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j < in) {
+    const double sj = static_cast<double>(s[j]);
+    sumsq[j] = sumsq[j] / (sj * sj);
+  }
+}
+
 // ----------------------------------------------------------------------- pack
-// One thread per uint32 word (8 memory-order columns).
+// One thread per uint32 word (8 memory-order columns).  With cs, the delta is
+// taken against W0[r][c] * cs[c] (the scaled layer the codes belong to).
 __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __restrict__ qscale,
                             const int32_t* __restrict__ invperm, int64_t out, int64_t in,
                             int bits, int g, const float* __restrict__ W0,
-                            uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales16,
-                            uint16_t* __restrict__ dW, float* __restrict__ dW32,
-                            int32_t* __restrict__ g_idx) {
+                            const float* __restrict__ cs, uint32_t* __restrict__ qweight,
+                            uint16_t* __restrict__ scales16, uint16_t* __restrict__ dW,
+                            float* __restrict__ dW32, int32_t* __restrict__ g_idx) {
   const int64_t words = in / 8;
   const int64_t ngroups = (in + g - 1) / g;
   const int64_t total = out * words;
@@ -143,6 +199,12 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
       const float4 b = *reinterpret_cast<const float4*>(W0 + r * in + wd * 8 + 4);
       w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w;
       w0[4] = b.x; w0[5] = b.y; w0[6] = b.z; w0[7] = b.w;
+      if (cs != nullptr) {
+        const float4 sa = __ldg(reinterpret_cast<const float4*>(cs + wd * 8));
+        const float4 sb = __ldg(reinterpret_cast<const float4*>(cs + wd * 8 + 4));
+        w0[0] *= sa.x; w0[1] *= sa.y; w0[2] *= sa.z; w0[3] *= sa.w;
+        w0[4] *= sb.x; w0[5] *= sb.y; w0[6] *= sb.z; w0[7] *= sb.w;
+      }
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -537,23 +599,45 @@ int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, 
 }
 
 int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
-                          float* Wq, cudaStream_t stream) {
+                          const float* cs, float* Wq, cudaStream_t stream) {
   if (in % 4 != 0 || (reinterpret_cast<uintptr_t>(W) & 15u) != 0 ||
-      (reinterpret_cast<uintptr_t>(Wq) & 15u) != 0 || (reinterpret_cast<uintptr_t>(perm) & 15u) != 0)
+      (reinterpret_cast<uintptr_t>(Wq) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(perm) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cs) & 15u) != 0)
     return PIQ_ERR_INVALID_ARG;
   note_launch();
-  gather_columns_kernel<<<grid_for(out * in / 4, 256), 256, 0, stream>>>(W, out, in, perm, Wq);
+  gather_columns_kernel<<<grid_for(out * in / 4, 256), 256, 0, stream>>>(W, out, in, perm, cs,
+                                                                         Wq);
+  return last_error();
+}
+
+int launch_scale_upper(float* H, int64_t in, const float* s, DeviceStatus* st,
+                       cudaStream_t stream) {
+  if (in % 4 != 0 || (reinterpret_cast<uintptr_t>(H) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(s) & 15u) != 0 || s == nullptr)
+    return PIQ_ERR_INVALID_ARG;
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in / 4, 256), 16)),
+            static_cast<unsigned>(std::min<int64_t>(in, 65535)));
+  note_launch();
+  scale_upper_kernel<<<grid, 256, 0, stream>>>(H, in, s, st);
+  return last_error();
+}
+
+int launch_scale_sumsq(double* sumsq, int64_t in, const float* s, cudaStream_t stream) {
+  note_launch();
+  scale_sumsq_kernel<<<static_cast<unsigned>(ceil_div(in, 256)), 256, 0, stream>>>(sumsq, in, s);
   return last_error();
 }
 
 int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
-                int64_t in, int bits, int g, const float* W0, uint32_t* qweight,
+                int64_t in, int bits, int g, const float* W0, const float* cs, uint32_t* qweight,
                 uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
                 cudaStream_t stream) {
   if ((dW != nullptr || dW32 != nullptr) && W0 == nullptr) return PIQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cs) & 15u) != 0) return PIQ_ERR_INVALID_ARG;
   note_launch();
   pack_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
-      codes, qscale, invperm, out, in, bits, g, W0, qweight, scales16, dW, dW32, g_idx);
+      codes, qscale, invperm, out, in, bits, g, W0, cs, qweight, scales16, dW, dW32, g_idx);
   return last_error();
 }
 

@@ -85,6 +85,14 @@ def make_weight(spec: LayerSpec, seed: int | None = None) -> np.ndarray:
     return (rng.standard_normal((spec.out, spec.inp)) * spec.w_std).astype(np.float32)
 
 
+def make_channel_scales(inp: int, seed: int, sigma: float = 0.5) -> np.ndarray:
+    """A positive per-input-channel vector s ~ LogNormal(0, sigma), float32 [in]
+    (a stand-in for a searched channel scaling, so that a scaled layer can be
+    tested without running the search)."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 4]))
+    return rng.lognormal(0.0, sigma, inp).astype(np.float32)
+
+
 def channel_gains(spec: LayerSpec, seed: int | None = None,
                   permute_seed: int | None = None) -> np.ndarray:
     """Per-channel multiplier sigma_j * (outlier gain), float32 [in].
