@@ -27,6 +27,15 @@ Readings where the pages are silent (each listed in the design notes):
   diagonal (the listing's order of operations).
 * Codes are returned in quantization order; ``perm[p]`` is the memory column
   quantized at position p.
+* Asymmetric groups (``sym=False``): the uplatz.com report, section "Key
+  Parameters" (Group Size), gives each group "a scale and zero-point" and no
+  formula.  Read as min/max affine rounding of the group's current weights with
+  the range widened to hold 0: lo = min(0, min w), hi = max(0, max w),
+  scale = (hi - lo) / (2^bits - 1), zero = round(-lo / scale), stored code
+  u = clip(round(w / scale) + zero, 0, 2^bits - 1), What = (u - zero) * scale.
+  Widening to 0 keeps the zero-point a valid code (0 <= zero <= 2^bits - 1,
+  stored like the weights) and reconstructs a zero weight exactly.  Codes are
+  returned signed, c = u - zero, so What = c * scale as in the symmetric case.
 """
 from __future__ import annotations
 
@@ -71,7 +80,7 @@ def upper_factor_ref(Hd: np.ndarray) -> np.ndarray:
 
 @dataclasses.dataclass
 class GPTQResult:
-    codes: np.ndarray        # int16 [out, in], quantization order
+    codes: np.ndarray        # int16 [out, in], quantization order (signed: What = code * scale)
     scales: np.ndarray       # float64 [out, ngroups], group of position p is p // g
     perm: np.ndarray         # int64 [in]
     g_idx: np.ndarray        # int64 [in], group of each memory-order column
@@ -81,6 +90,7 @@ class GPTQResult:
     lam: float
     bits: int
     g: int
+    zeros: np.ndarray | None = None  # int16 [out, ngroups] zero-points (asymmetric groups)
 
 
 def gptq_prepare_ref(H: np.ndarray, damp: float = 0.01, act_order: bool = False, perm=None):
@@ -98,33 +108,57 @@ def _round_clip(v: np.ndarray, qmax: int) -> np.ndarray:
     return np.clip(np.round(v), -qmax - 1, qmax)
 
 
-def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
-                   force: np.ndarray | None = None, log: bool = True, dtype=np.float64):
-    """The listing's column loop on weights already in quantization order.
+def group_quantizer_ref(Wg: np.ndarray, bits: int, sym: bool = True, dtype=np.float64,
+                        force_zero=None):
+    """Per-row quantizer of one group from its current weights Wg [out, <= g]:
+    (scale, zero, zv, cmin, cmax); signed codes are clip(round(w / scale),
+    cmin, cmax) and What = code * scale.
 
-    Returns (codes int16 [out, in], scales [out, ngroups], v, err).
-    ``force`` (int array [out, in], NO_FORCE where free) replaces the rounded
-    code at chosen sites: the teacher-forcing hook of the parity comparison.
-    ``dtype`` is the working precision: float64 is the oracle; float32 runs the
-    same loop in the precision the north star fixes for the sweep, to measure
-    how far that arithmetic alone drifts from float64 (the parity tie window)."""
+    sym: scale = max|w| / qmax, zero 0, codes in [-qmax - 1, qmax] (the listing).
+    asym: lo = min(0, min w), hi = max(0, max w), scale = (hi - lo) / (2^bits - 1),
+    zv = -lo / scale, zero = round(zv), codes in [-zero, 2^bits - 1 - zero].
+    A row whose group is all zero gets scale 0 and zero 0.  ``force_zero``
+    (int [out], NO_FORCE where free) overrides the rounded zero-point."""
+    out = Wg.shape[0]
+    if sym:
+        qmax = 2 ** (bits - 1) - 1
+        scale = np.abs(Wg).max(axis=1) / dtype(qmax)
+        zero = np.zeros(out)
+        return (scale, zero, zero.copy(), np.full(out, -qmax - 1.0), np.full(out, float(qmax)))
+    maxq = 2 ** bits - 1
+    lo = np.minimum(Wg.min(axis=1), dtype(0.0))
+    hi = np.maximum(Wg.max(axis=1), dtype(0.0))
+    scale = (hi - lo) / dtype(maxq)
+    live = scale > 0
+    zv = np.where(live, -lo / np.where(live, scale, dtype(1.0)), dtype(0.0))
+    zero = np.round(zv)
+    if force_zero is not None:
+        zero = np.where(force_zero != NO_FORCE, force_zero, zero)
+    return scale, zero, zv, -zero, maxq - zero
+
+
+def _sweep(Wp, U, bits, g, sym, force, force_zero, log, dtype):
     W = np.array(Wp, dtype=dtype, copy=True)
     U = np.asarray(U, dtype=dtype)
     out, inp = W.shape
-    qmax = 2 ** (bits - 1) - 1
     ngroups = -(-inp // g)
     codes = np.zeros((out, inp), dtype=np.int16)
     scales = np.zeros((out, ngroups), dtype=np.float64)
+    zeros = np.zeros((out, ngroups), dtype=np.int16)
+    zvlog = np.zeros((out, ngroups))
     vlog = np.zeros((out, inp)) if log else None
     elog = np.zeros((out, inp)) if log else None
-    scale = None
+    scale = cmin = cmax = None
     for j in range(inp):
         if j % g == 0:
-            scale = np.abs(W[:, j:j + g]).max(axis=1) / dtype(qmax)
+            fz = None if force_zero is None else force_zero[:, j // g]
+            scale, zero, zv, cmin, cmax = group_quantizer_ref(W[:, j:j + g], bits, sym, dtype, fz)
             scales[:, j // g] = scale
+            zeros[:, j // g] = zero.astype(np.int16)
+            zvlog[:, j // g] = zv
         live = scale > 0
         v = np.where(live, W[:, j] / np.where(live, scale, dtype(1.0)), dtype(0.0))
-        c = _round_clip(v, qmax)
+        c = np.clip(np.round(v), cmin, cmax)
         if force is not None:
             f = force[:, j]
             c = np.where(f != NO_FORCE, f, c)
@@ -135,7 +169,32 @@ def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
         if log:
             vlog[:, j] = v
             elog[:, j] = e
+    return codes, scales, zeros, zvlog, vlog, elog
+
+
+def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
+                   force: np.ndarray | None = None, log: bool = True, dtype=np.float64):
+    """The listing's column loop on weights already in quantization order.
+
+    Returns (codes int16 [out, in], scales [out, ngroups], v, err).
+    ``force`` (int array [out, in], NO_FORCE where free) replaces the rounded
+    code at chosen sites: the teacher-forcing hook of the parity comparison.
+    ``dtype`` is the working precision: float64 is the oracle; float32 runs the
+    same loop in the precision the north star fixes for the sweep, to measure
+    how far that arithmetic alone drifts from float64 (the parity tie window)."""
+    codes, scales, _, _, vlog, elog = _sweep(Wp, U, bits, g, True, force, None, log, dtype)
     return codes, scales, vlog, elog
+
+
+def gptq_sweep_asym_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
+                        force: np.ndarray | None = None, force_zero: np.ndarray | None = None,
+                        log: bool = True, dtype=np.float64):
+    """The same loop with a scale and zero-point per group (asymmetric groups,
+    see the module notes).  Returns (codes, scales, zeros, zv, v, err): signed
+    codes (stored u = code + zero), zero-points int16 [out, ngroups] and their
+    unrounded values zv = -lo / scale.  ``force_zero`` [out, ngroups] overrides
+    rounded zero-points (teacher forcing)."""
+    return _sweep(Wp, U, bits, g, False, force, force_zero, log, dtype)
 
 
 def g_idx_from_perm(perm: np.ndarray, g: int) -> np.ndarray:
@@ -145,14 +204,17 @@ def g_idx_from_perm(perm: np.ndarray, g: int) -> np.ndarray:
 
 
 def gptq_ref(W, X=None, *, H=None, bits: int = 4, g: int = 128, damp: float = 0.01,
-             act_order: bool = False, force=None, log: bool = True) -> GPTQResult:
-    """GPTQ of one layer, literally (one column at a time)."""
+             act_order: bool = False, force=None, log: bool = True,
+             sym: bool = True) -> GPTQResult:
+    """GPTQ of one layer, literally (one column at a time); ``sym=False``: a
+    scale and zero-point per group."""
     if H is None:
         H = hessian_ref(X)
     perm, U, lam = gptq_prepare_ref(H, damp, act_order)
     Wp = np.asarray(W, dtype=np.float64)[:, perm]
-    codes, scales, v, e = gptq_sweep_ref(Wp, U, bits, g, force=force, log=log)
-    return GPTQResult(codes, scales, perm, g_idx_from_perm(perm, g), v, e, U, lam, bits, g)
+    codes, scales, zeros, _, v, e = _sweep(Wp, U, bits, g, sym, force, None, log, np.float64)
+    return GPTQResult(codes, scales, perm, g_idx_from_perm(perm, g), v, e, U, lam, bits, g,
+                      None if sym else zeros)
 
 
 def block_partition_ref(inp: int, g: int, block: int = 128):
@@ -175,27 +237,24 @@ def block_partition_ref(inp: int, g: int, block: int = 128):
     return blocks
 
 
-def gptq_sweep_blocked_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
-                           block: int = 128):
-    """The same loop with updates deferred per column block: inside a block the
-    error goes to the block's later columns; after the block one product
-    Err[:, b:e] @ U[b:e, e:] updates every column past it."""
+def _sweep_blocked(Wp, U, bits, g, block, sym):
     W = np.array(Wp, dtype=np.float64, copy=True)
     out, inp = W.shape
-    qmax = 2 ** (bits - 1) - 1
     codes = np.zeros((out, inp), dtype=np.int16)
     scales = np.zeros((out, -(-inp // g)), dtype=np.float64)
+    zeros = np.zeros((out, -(-inp // g)), dtype=np.int16)
     vlog = np.zeros((out, inp))
-    scale = None
+    scale = cmin = cmax = None
     for b, e in block_partition_ref(inp, g, block):
         Err = np.zeros((out, e - b))
         for j in range(b, e):
             if j % g == 0:
-                scale = np.abs(W[:, j:j + g]).max(axis=1) / qmax
+                scale, zero, _, cmin, cmax = group_quantizer_ref(W[:, j:j + g], bits, sym)
                 scales[:, j // g] = scale
+                zeros[:, j // g] = zero.astype(np.int16)
             live = scale > 0
             v = np.where(live, W[:, j] / np.where(live, scale, 1.0), 0.0)
-            c = _round_clip(v, qmax)
+            c = np.clip(np.round(v), cmin, cmax)
             err = (W[:, j] - c * scale) / U[j, j]
             W[:, j + 1:e] -= np.outer(err, U[j, j + 1:e])
             Err[:, j - b] = err
@@ -203,18 +262,34 @@ def gptq_sweep_blocked_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int 
             vlog[:, j] = v
         if e < inp:
             W[:, e:] -= Err @ U[b:e, e:]
+    return codes, scales, zeros, vlog
+
+
+def gptq_sweep_blocked_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
+                           block: int = 128):
+    """The same loop with updates deferred per column block: inside a block the
+    error goes to the block's later columns; after the block one product
+    Err[:, b:e] @ U[b:e, e:] updates every column past it.  (codes, scales, v)."""
+    codes, scales, _, vlog = _sweep_blocked(Wp, U, bits, g, block, True)
     return codes, scales, vlog
 
 
+def gptq_sweep_blocked_asym_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
+                                block: int = 128):
+    """Blocked sweep with asymmetric groups: (codes, scales, zeros, v)."""
+    return _sweep_blocked(Wp, U, bits, g, block, False)
+
+
 def gptq_ref_blocked(W, X=None, *, H=None, bits: int = 4, g: int = 128, damp: float = 0.01,
-                     act_order: bool = False, block: int = 128) -> GPTQResult:
+                     act_order: bool = False, block: int = 128, sym: bool = True) -> GPTQResult:
     """GPTQ with block-deferred updates (same arithmetic, faster on large layers)."""
     if H is None:
         H = hessian_ref(X)
     perm, U, lam = gptq_prepare_ref(H, damp, act_order)
     Wp = np.asarray(W, dtype=np.float64)[:, perm]
-    codes, scales, v = gptq_sweep_blocked_ref(Wp, U, bits, g, block)
-    return GPTQResult(codes, scales, perm, g_idx_from_perm(perm, g), v, None, U, lam, bits, g)
+    codes, scales, zeros, v = _sweep_blocked(Wp, U, bits, g, block, sym)
+    return GPTQResult(codes, scales, perm, g_idx_from_perm(perm, g), v, None, U, lam, bits, g,
+                      None if sym else zeros)
 
 
 def rtn_ref(W, bits: int = 4, g: int = 128):
@@ -233,3 +308,23 @@ def rtn_ref(W, bits: int = 4, g: int = 128):
         codes[:, s:s + g] = _round_clip(v, qmax).astype(np.int16)
         scales[:, s // g] = sc
     return codes, scales
+
+
+def rtn_asym_ref(W, bits: int = 4, g: int = 128):
+    """Group round-to-nearest with a scale and zero-point per group (the
+    asymmetric quantizer of the module notes, no error feedback).  Returns
+    (signed codes, scales, zeros); the stored code is code + zero."""
+    W = np.asarray(W, dtype=np.float64)
+    out, inp = W.shape
+    codes = np.zeros((out, inp), dtype=np.int16)
+    scales = np.zeros((out, -(-inp // g)))
+    zeros = np.zeros((out, -(-inp // g)), dtype=np.int16)
+    for s0 in range(0, inp, g):
+        blk = W[:, s0:s0 + g]
+        sc, z, _, cmin, cmax = group_quantizer_ref(blk, bits, sym=False)
+        live = sc > 0
+        v = np.where(live[:, None], blk / np.where(live, sc, 1.0)[:, None], 0.0)
+        codes[:, s0:s0 + g] = np.clip(np.round(v), cmin[:, None], cmax[:, None]).astype(np.int16)
+        scales[:, s0 // g] = sc
+        zeros[:, s0 // g] = z.astype(np.int16)
+    return codes, scales, zeros

@@ -6,6 +6,8 @@ act-order needs a group index per column (same section).  The byte layout is
 this library's own: code c of memory column k is stored as u = c + 2^(bits-1)
 in nibble k % 8 (bits 4(k%8) .. 4(k%8)+3) of uint32 word k // 8 of its row;
 scales are FP16 (round to nearest even) of the scale the quantizer used.
+With a zero-point per group (asymmetric groups) the stored code is
+u = c + zero instead, and the zero-points are one byte each, [out, ngroups].
 """
 from __future__ import annotations
 
@@ -58,3 +60,14 @@ def dequant_ref(codes_q: np.ndarray, scales: np.ndarray, perm: np.ndarray, g: in
     cols = np.arange(codes_q.shape[1]) // g
     What_q = codes_q.astype(np.float64) * sc[:, cols]
     return to_memory_order(What_q, np.asarray(perm))
+
+
+def pack_asym_ref(codes_mem: np.ndarray, zeros: np.ndarray, g_idx: np.ndarray,
+                  bits: int) -> np.ndarray:
+    """Asymmetric groups: stored code u = code + zero of the column's group
+    (0 <= u <= 2^bits - 1), packed like pack_ref's words."""
+    c = np.asarray(codes_mem, dtype=np.int64)
+    z = np.asarray(zeros, dtype=np.int64)[:, np.asarray(g_idx)]
+    u = c + z
+    assert u.min() >= 0 and u.max() <= 2 ** bits - 1
+    return pack_ref(u - 2 ** (bits - 1), bits)
