@@ -378,6 +378,9 @@ def run_ours(args):
     awq = None
     if args.awq and rank == 0:
         awq = run_awq(dev)
+    variants = None
+    if args.variants and rank == 0:
+        variants = run_variants(dev, Wg, Xg)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -387,7 +390,7 @@ def run_ours(args):
                 "config": workload_config(C2, n), "xtx_tflops": ach_h,
                 "phases_ms": ph, "roofline": roof,
                 "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
-                "awq": awq, "shift_error": e2, "calib_error": o.err}
+                "awq": awq, "variants": variants, "shift_error": e2, "calib_error": o.err}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -425,6 +428,49 @@ def run_awq(dev, steps=3, warmup=1):
             "phases_ms": ph, "error_gemm_tflops": flops / (ph["error_gemm"] / 1e3) / 1e12}
 
 
+def run_variants(dev, Wg, Xg, steps=5, warmup=3):
+    """The q_proj layer through plain GPTQ, AWQ-scaled GPTQ (s from AWQ's
+    20-point search, run once untimed) and GPTQ with asymmetric groups, timed
+    interleaved step by step so that all three see the same clocks: ms per layer
+    (median) and each one's output error."""
+    import torch
+    import post_int4_weight_gptq_b200 as piq
+    from workloads import AWQ_GRID, C2
+    out_rows, inp = Wg.shape
+    n = Xg.shape[0]
+    a = piq.awq_search_layer(Wg, Xg, C2.bits, C2.g, AWQ_GRID)
+    ws = torch.empty(piq.gptq_workspace_bytes(out_rows, inp, n), dtype=torch.uint8, device=dev)
+    calls = {
+        "gptq": lambda: piq.gptq_quantize_layer(Wg, Xg, C2.bits, C2.g, C2.damp, workspace=ws),
+        "awq_then_gptq": lambda: piq.awq_gptq_quantize_layer(Wg, Xg, a.s, C2.bits, C2.g,
+                                                             C2.damp, workspace=ws),
+        "gptq_asym": lambda: piq.gptq_quantize_layer(Wg, Xg, C2.bits, C2.g, C2.damp,
+                                                     workspace=ws, sym=False),
+    }
+    for _ in range(warmup):
+        for f in calls.values():
+            f()
+    times = {k: [] for k in calls}
+    errs = {}
+    for _ in range(steps):
+        for k, f in calls.items():
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            r = f()
+            e1.record()
+            torch.cuda.synchronize()
+            times[k].append(e0.elapsed_time(e1))
+            errs[k] = r.err
+    res = {"workload": "q_proj 4096x4096, X 131072x4096, 4-bit g128: three GPTQ variants "
+                       "timed interleaved", "awq_alpha": a.best_alpha,
+           "awq_error": a.err_per_alpha[int(np.argmin([abs(x - a.best_alpha) for x in AWQ_GRID]))]}
+    for k in calls:
+        ms = statistics.median(times[k])
+        res[k] = {"ms_per_layer": ms, "mweights_per_s": out_rows * inp / (ms / 1e3) / 1e6,
+                  "error": errs[k]}
+    return res
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,6 +480,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--awq", action="store_true", help="also time the AWQ search (8192^2 layer)")
+    ap.add_argument("--variants", action="store_true",
+                    help="also time plain, AWQ-scaled and asymmetric-group GPTQ on the same "
+                         "layer, interleaved")
     ap.add_argument("--samples", type=int, default=None,
                     help="calibration rows per layer (default: the workload's 131072); a smaller "
                          "value is for profiler captures, not for reported numbers")

@@ -38,7 +38,9 @@
  *    row (qweight is [out, in/8]).  scales is [out, ceil(in/g)] IEEE fp16 bit
  *    patterns, round-to-nearest-even of the fp32 scale the quantizer used.
  *    The dequantized weight is code * scale[row, group(k)] (GPTQ, RTN) and
- *    code * scale[row, group(k)] / s[k] (AWQ).
+ *    code * scale[row, group(k)] / s[k] (AWQ).  With a zero-point per group
+ *    (gptq_quantize_layer_asym) the nibble holds u = c + zero[row, group(k)]
+ *    instead, zeros being uint8 [out, ceil(in/g)].
  */
 #ifndef PIQ_H_
 #define PIQ_H_
@@ -129,6 +131,25 @@ int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t*
                         uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* GPTQ with a scale and a zero-point per group (the uplatz.com report, GPTQ's
+ * key parameters, Group Size).  The pages give no formula; the quantizer is
+ * min/max affine rounding of the group's current weights over a range widened
+ * to hold 0, taken at each group start like the symmetric scale:
+ *   lo = min(0, min w), hi = max(0, max w),  scale = (hi - lo) / (2^bits - 1),
+ *   zero = rint(-lo / scale)  (0 <= zero <= 2^bits - 1; 0 when scale is 0),
+ *   u = clip(rint(w / scale) + zero, 0, 2^bits - 1),  What = (u - zero) * scale.
+ *   qweight  as gptq_quantize_layer, but nibble = u (the stored code itself).
+ *   zeros    device uint8 [out, ceil(in/g)], required: the zero-points, groups
+ *            in quantization order like scales.
+ *   out_err  What = (u - zero) * fp16(scale).
+ * Workspace: piq_gptq_workspace_bytes.  Everything else as gptq_quantize_layer
+ * (the error feedback, blocking, act-order and factor are unchanged). */
+int gptq_quantize_layer_asym(const float* W, int64_t out, int64_t in, const uint16_t* X,
+                             int64_t n, int bits, int g, float damp, int act_order,
+                             uint32_t* qweight, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                             int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                             void* stream);
+
 /* AWQ scale search of one layer.
  *   alpha_grid     host float [n_alpha], 1 <= n_alpha <= 64 (e.g. k/20, k = 0..19).
  *   best_alpha     host float, may be NULL: the grid value with the smallest
@@ -185,7 +206,9 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
 /* Output error of a packed layer on inputs X (the shared objective, "How to
  * approach it"; e.g. a held-out or shifted X'):
  *   ||X W^T - X What^T||_F^2,  What[r, k] = code * fp16(scale[r, grp(k)]) / s[k]
- * grp(k) = g_idx[k] (or k / g when g_idx == NULL); s == NULL means s = 1.
+ * grp(k) = g_idx[k] (or k / g when g_idx == NULL); s == NULL means s = 1;
+ * code = u - zeros[r, grp(k)] (uint8 [out, ceil(in/g)], asymmetric groups) or
+ * u - 2^(bits-1) when zeros == NULL.
  * Two exact routes, picked from (out, in, n) alone so the workspace size is
  * fixed by them: directly, a BF16 tensor-core product X D^T (D = W - What
  * rounded to bf16) squared and summed; or, when n is large against out and in
@@ -194,9 +217,9 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
  * All pointers device except out_err (host).  Synchronizes `stream`. */
 int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t* bytes);
 int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
-                           const uint16_t* scales, const int32_t* g_idx, const float* s,
-                           int bits, int g, const uint16_t* X, int64_t n, double* out_err,
-                           void* workspace, size_t ws_bytes, void* stream);
+                           const uint16_t* scales, const uint8_t* zeros, const int32_t* g_idx,
+                           const float* s, int bits, int g, const uint16_t* X, int64_t n,
+                           double* out_err, void* workspace, size_t ws_bytes, void* stream);
 
 /* Per-phase timing (diagnostics).  When enabled, gptq_quantize_layer and
  * awq_search_layer record CUDA events around their phases; the times of the

@@ -59,6 +59,10 @@ SIGNATURES = {
                                      _c_int, _vp, _vp, _vp, _vp,
                                      ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
                                      _vp]),
+    "gptq_quantize_layer_asym": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int,
+                                          _c_float, _c_int, _vp, _vp, _vp, _vp, _vp,
+                                          ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
+                                          _vp]),
     "piq_awq_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_size_p]),
     "awq_search_layer": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int,
                                   ctypes.POINTER(ctypes.c_float), _c_int,
@@ -72,8 +76,8 @@ SIGNATURES = {
     "piq_rtn_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp,
                                         ctypes.c_size_t, _vp]),
     "piq_output_error_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_size_p]),
-    "piq_layer_output_error": (_c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _c_int, _c_int,
-                                        _vp, _c_i64, ctypes.POINTER(ctypes.c_double), _vp,
+    "piq_layer_output_error": (_c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                        _c_int, _vp, _c_i64, ctypes.POINTER(ctypes.c_double), _vp,
                                         ctypes.c_size_t, _vp]),
     "piq_set_timing": (_c_int, [_c_int]),
     "piq_last_phase_times": (_c_int, [ctypes.POINTER(ctypes.c_double), _c_int,
@@ -203,7 +207,8 @@ def gptq_sweep(Wp, U, bits=4, g=128, stream=None, workspace=None):
     return codes, qscale
 
 
-GPTQOutput = collections.namedtuple("GPTQOutput", "qweight scales perm g_idx err")
+GPTQOutput = collections.namedtuple("GPTQOutput", "qweight scales perm g_idx err zeros",
+                                    defaults=(None,))
 AWQOutput = collections.namedtuple("AWQOutput", "best_alpha s qweight scales err_per_alpha")
 
 
@@ -212,8 +217,10 @@ def gptq_workspace_bytes(out, inp, n, act_order=False) -> int:
 
 
 def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_error=True,
-                        stream=None, workspace=None, out=None):
-    """GPTQ of one layer W [out, in] (fp32) on calibration X [n, in] (bf16)."""
+                        stream=None, workspace=None, out=None, sym=True):
+    """GPTQ of one layer W [out, in] (fp32) on calibration X [n, in] (bf16).
+    sym=False: a scale and a zero-point per group (gptq_quantize_layer_asym);
+    the zero-points come back in ``zeros`` (uint8 [out, ceil(in/g)])."""
     lib = load_library()
     _need(W, torch.float32, "W")
     _need(X, torch.bfloat16, "X")
@@ -222,18 +229,30 @@ def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_er
     if X.shape[1] != inp:
         raise ValueError("W and X disagree on the input dimension")
     dev = W.device
+    ng = -(-inp // g)
     if out is None:
         out = GPTQOutput(torch.empty(rows, inp // 8, dtype=torch.int32, device=dev),
-                         torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev),
+                         torch.empty(rows, ng, dtype=torch.float16, device=dev),
                          torch.empty(inp, dtype=torch.int32, device=dev),
-                         torch.empty(inp, dtype=torch.int32, device=dev), None)
+                         torch.empty(inp, dtype=torch.int32, device=dev), None,
+                         None if sym else torch.empty(rows, ng, dtype=torch.uint8, device=dev))
     ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order), dev, workspace)
     err = ctypes.c_double(0.0)
-    _check(lib.gptq_quantize_layer(_ptr(W), rows, inp, _ptr(X), n, bits, g, float(damp),
-                                   int(bool(act_order)), _ptr(out.qweight), _ptr(out.scales),
-                                   _ptr(out.perm), _ptr(out.g_idx),
-                                   ctypes.byref(err) if with_error else None, _ptr(ws),
-                                   ws.numel(), _stream(stream)), "gptq_quantize_layer")
+    eptr = ctypes.byref(err) if with_error else None
+    if sym:
+        rc = lib.gptq_quantize_layer(_ptr(W), rows, inp, _ptr(X), n, bits, g, float(damp),
+                                     int(bool(act_order)), _ptr(out.qweight), _ptr(out.scales),
+                                     _ptr(out.perm), _ptr(out.g_idx), eptr, _ptr(ws),
+                                     ws.numel(), _stream(stream))
+        _check(rc, "gptq_quantize_layer")
+    else:
+        _need(out.zeros, torch.uint8, "zeros")
+        rc = lib.gptq_quantize_layer_asym(_ptr(W), rows, inp, _ptr(X), n, bits, g, float(damp),
+                                          int(bool(act_order)), _ptr(out.qweight),
+                                          _ptr(out.scales), _ptr(out.zeros), _ptr(out.perm),
+                                          _ptr(out.g_idx), eptr, _ptr(ws), ws.numel(),
+                                          _stream(stream))
+        _check(rc, "gptq_quantize_layer_asym")
     return out._replace(err=err.value if with_error else None)
 
 
@@ -320,7 +339,7 @@ def output_error_workspace_bytes(out, inp, n) -> int:
 
 
 def layer_output_error(W, qweight, scales, X, bits=4, g=128, g_idx=None, s=None, stream=None,
-                       workspace=None) -> float:
+                       workspace=None, zeros=None) -> float:
     """||X W^T - X What^T||^2 of a packed layer on inputs X."""
     lib = load_library()
     _need(W, torch.float32, "W")
@@ -331,8 +350,8 @@ def layer_output_error(W, qweight, scales, X, bits=4, g=128, g_idx=None, s=None,
                     workspace)
     e = ctypes.c_double(0.0)
     _check(lib.piq_layer_output_error(_ptr(W), rows, inp, _ptr(qweight), _ptr(scales),
-                                      _ptr(g_idx), _ptr(s), bits, g, _ptr(X), n, ctypes.byref(e),
-                                      _ptr(ws), ws.numel(), _stream(stream)),
+                                      _ptr(zeros), _ptr(g_idx), _ptr(s), bits, g, _ptr(X), n,
+                                      ctypes.byref(e), _ptr(ws), ws.numel(), _stream(stream)),
            "piq_layer_output_error")
     return e.value
 

@@ -303,10 +303,12 @@ size_t gptq_ws_bytes(int64_t out, int64_t in, int64_t n, int act_order) {
 // H' = diag(1/s) X^T X diag(1/s), the act-order key diag(H'), the sweep over
 // W diag(s), and the error of What = code * scale / s through H' with
 // D' = W diag(s) - code * fp16(scale), since X' D'^T = X (W - What)^T.
+// With zeros, every group gets a scale and a zero-point (asymmetric groups):
+// the sweep writes the zero-points there and the pack stores code + zero.
 int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
                const float* s_ch, int bits, int g, float damp, int act_order, uint32_t* qweight,
-               uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err, void* workspace,
-               size_t ws_bytes, cudaStream_t s) {
+               uint16_t* scales, uint8_t* zeros, int32_t* perm, int32_t* g_idx, double* out_err,
+               void* workspace, size_t ws_bytes, cudaStream_t s) {
   PIQ_TRY(check_layer(out, in, bits, g));
   if (W == nullptr || X == nullptr || qweight == nullptr || scales == nullptr || n < 1 ||
       !(damp >= 0.f) || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
@@ -346,10 +348,10 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
   clk.mark();
   // 4. blocked sweep on the permuted (and scaled) copy
   PIQ_TRY(launch_gather_columns(W, out, in, qperm, s_ch, w.Wq, s));
-  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, w.Err, w.st, s));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, zeros, w.Err, w.st, s));
   clk.mark();
   // 5. pack (+ D = W diag(s) - What' for the error)
-  PIQ_TRY(launch_pack(w.codes, w.qscale, qinv, out, in, bits, g, W, s_ch, qweight, scales,
+  PIQ_TRY(launch_pack(w.codes, w.qscale, zeros, qinv, out, in, bits, g, W, s_ch, qweight, scales,
                       nullptr, out_err ? w.dW : nullptr, g_idx, s));
   clk.mark();
   // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from the H built in step 1
@@ -454,7 +456,7 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
   SweepWs w = carve_sweep(c, out, in);
   PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
   PIQ_TRY(cuda_rc(cudaMemcpyAsync(w.Wq, Wp, sizeof(float) * out * in, cudaMemcpyDeviceToDevice, s)));
-  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, codes, qscale, w.Err, w.st, s));
+  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, codes, qscale, nullptr, w.Err, w.st, s));
   return finish_call(w.st, s, nullptr);
 }
 
@@ -468,8 +470,18 @@ int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t*
                         int bits, int g, float damp, int act_order, uint32_t* qweight,
                         uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,
                         void* workspace, size_t ws_bytes, void* stream) {
-  return gptq_layer(W, out, in, X, n, nullptr, bits, g, damp, act_order, qweight, scales, perm,
-                    g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+  return gptq_layer(W, out, in, X, n, nullptr, bits, g, damp, act_order, qweight, scales, nullptr,
+                    perm, g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int gptq_quantize_layer_asym(const float* W, int64_t out, int64_t in, const uint16_t* X,
+                             int64_t n, int bits, int g, float damp, int act_order,
+                             uint32_t* qweight, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                             int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (zeros == nullptr) return PIQ_ERR_INVALID_ARG;
+  return gptq_layer(W, out, in, X, n, nullptr, bits, g, damp, act_order, qweight, scales, zeros,
+                    perm, g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int awq_gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
@@ -478,8 +490,8 @@ int awq_gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint1
                             int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
                             void* stream) {
   if (s_ch == nullptr || !aligned16(s_ch)) return PIQ_ERR_INVALID_ARG;
-  return gptq_layer(W, out, in, X, n, s_ch, bits, g, damp, act_order, qweight, scales, perm,
-                    g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+  return gptq_layer(W, out, in, X, n, s_ch, bits, g, damp, act_order, qweight, scales, nullptr,
+                    perm, g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int piq_awq_workspace_bytes(int64_t out, int64_t in, int64_t n, int n_alpha, size_t* bytes) {
@@ -529,7 +541,7 @@ int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
   // 4. first minimum, re-quantize at it, pack
   PIQ_TRY(launch_argmin(w.err, n_alpha, w.alphas, w.best, w.best_alpha, s));
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, w.s_table, w.best, w.codes, w.qscale, s_out, s));
-  PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
+  PIQ_TRY(launch_pack(w.codes, w.qscale, nullptr, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
                       scales, nullptr, nullptr, nullptr, s));
   clk.mark();
   double errs[64];
@@ -567,7 +579,7 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
   Carver c(workspace);
   RtnWs w = carve_rtn(c, out, in);
   PIQ_TRY(launch_group_quant(W, out, in, bits, g, nullptr, nullptr, w.codes, w.qscale, nullptr, s));
-  return launch_pack(w.codes, w.qscale, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
+  return launch_pack(w.codes, w.qscale, nullptr, nullptr, out, in, bits, g, nullptr, nullptr, qweight,
                      scales, nullptr, nullptr, nullptr, s);
 }
 
@@ -580,9 +592,9 @@ int piq_output_error_workspace_bytes(int64_t out, int64_t in, int64_t n, size_t*
 }
 
 int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
-                           const uint16_t* scales, const int32_t* g_idx, const float* s_ch,
-                           int bits, int g, const uint16_t* X, int64_t n, double* out_err,
-                           void* workspace, size_t ws_bytes, void* stream) {
+                           const uint16_t* scales, const uint8_t* zeros, const int32_t* g_idx,
+                           const float* s_ch, int bits, int g, const uint16_t* X, int64_t n,
+                           double* out_err, void* workspace, size_t ws_bytes, void* stream) {
   PIQ_TRY(check_layer(out, in, bits, g));
   if (W == nullptr || qweight == nullptr || scales == nullptr || X == nullptr ||
       out_err == nullptr || n < 1 || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
@@ -597,13 +609,13 @@ int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32
   ErrWs w = carve_err(c, out, in, n);
   PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
   if (error_route_h(out, in, n)) {
-    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, nullptr,
-                                 w.dW32, w.st, s));
+    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, zeros, g_idx, s_ch, bits, g,
+                                 nullptr, w.dW32, w.st, s));
     PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
     PIQ_TRY(run_error_via_h(w.dW32, out, in, w.H, w.dsplit, w.hsplit, w.partials, w.err, w.st,
                             s));
   } else {
-    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, g_idx, s_ch, bits, g, w.dW,
+    PIQ_TRY(launch_dequant_delta(W, out, in, qweight, scales, zeros, g_idx, s_ch, bits, g, w.dW,
                                  nullptr, w.st, s));
     PIQ_TRY(launch_err_sumsq(X, n, in, w.dW, out, 1, w.partials, w.st, s));
     PIQ_TRY(launch_reduce_partials(w.partials, n, out, 1, w.err, s));

@@ -98,8 +98,10 @@ int launch_identity_perm(int64_t in, int32_t* perm, int32_t* invperm, cudaStream
 // ---------------------------------------------------------------- sweep (sweep.cu)
 constexpr int kSweepB = 128;
 // Full blocked sweep over quantization-order weights Wq (updated in place).
+// qzero != NULL: asymmetric groups, zero-points written to qzero [out, ngroups]
+// (signed codes c = u - zero, What = c * scale either way).
 int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits, int g,
-                   int8_t* codes, float* qscale, float* Err, DeviceStatus* st,
+                   int8_t* codes, float* qscale, uint8_t* qzero, float* Err, DeviceStatus* st,
                    cudaStream_t stream);
 
 // ------------------------------------------------- quantize / pack / stats (quant.cu)
@@ -110,11 +112,12 @@ int colstats_splits(int64_t n, int64_t in);
 int launch_gather_columns(const float* W, int64_t out, int64_t in, const int32_t* perm,
                           const float* cs, float* Wq, cudaStream_t stream);
 // dW (bf16) and dW32 (fp32), when given, receive W0 diag(cs) - code * fp16(scale)
-// (cs == NULL: W0 - code * fp16(scale)).
-int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
-                int64_t in, int bits, int g, const float* W0, const float* cs, uint32_t* qweight,
-                uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
-                cudaStream_t stream);
+// (cs == NULL: W0 - code * fp16(scale)).  qzero != NULL: stored code
+// u = code + zero of the (row, quantization-order group), else code + 2^(bits-1).
+int launch_pack(const int8_t* codes, const float* qscale, const uint8_t* qzero,
+                const int32_t* invperm, int64_t out, int64_t in, int bits, int g,
+                const float* W0, const float* cs, uint32_t* qweight, uint16_t* scales16,
+                uint16_t* dW, float* dW32, int32_t* g_idx, cudaStream_t stream);
 // H = diag(1/s) H diag(1/s) on the upper triangle, in place; a non-finite or
 // non-positive s_k sets PIQ_ERR_INVALID_ARG (where = k) in st.
 int launch_scale_upper(float* H, int64_t in, const float* s, DeviceStatus* st,
@@ -130,10 +133,11 @@ int launch_group_quant(const float* W, int64_t out, int64_t in, int bits, int g,
                        float* s_out, cudaStream_t stream);
 int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_idx,
                   float* best_alpha, cudaStream_t stream);
-// W - What from a packed layer, into dW (bf16) or dW32 (fp32), whichever is given.
+// W - What from a packed layer, into dW (bf16) or dW32 (fp32), whichever is given;
+// zeros != NULL: code = u - zeros[r][grp], else u - 2^(bits-1).
 int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
-                         const uint16_t* scales16, const int32_t* g_idx, const float* s,
-                         int bits, int g, uint16_t* dW, float* dW32, DeviceStatus* st,
-                         cudaStream_t stream);
+                         const uint16_t* scales16, const uint8_t* zeros, const int32_t* g_idx,
+                         const float* s, int bits, int g, uint16_t* dW, float* dW32,
+                         DeviceStatus* st, cudaStream_t stream);
 
 }  // namespace piq

@@ -176,6 +176,7 @@ __global__ void scale_sumsq_kernel(double* __restrict__ sumsq, int64_t in,
 // One thread per uint32 word (8 memory-order columns).  With cs, the delta is
 // taken against W0[r][c] * cs[c] (the scaled layer the codes belong to).
 __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __restrict__ qscale,
+                            const uint8_t* __restrict__ qzero,
                             const int32_t* __restrict__ invperm, int64_t out, int64_t in,
                             int bits, int g, const float* __restrict__ W0,
                             const float* __restrict__ cs, uint32_t* __restrict__ qweight,
@@ -211,7 +212,8 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
       const int64_t c = wd * 8 + k;
       const int64_t p = invperm ? invperm[c] : c;
       const int code = crow[p];
-      word |= static_cast<uint32_t>(code + off) << (4 * k);
+      const int zp = qzero ? static_cast<int>(qzero[r * ngroups + p / g]) : off;
+      word |= static_cast<uint32_t>(code + zp) << (4 * k);
       if (delta) {
         const float s16 = __half2float(__float2half_rn(srow[p / g]));
         d32[k] = w0[k] - static_cast<float>(code) * s16;
@@ -494,10 +496,12 @@ __global__ void argmin_kernel(const double* err, int n, const float* alphas, int
   if (best_alpha) *best_alpha = alphas[b];
 }
 
-// D = W - code * fp16(scale) / s, from the packed format; one thread per word.
+// D = W - code * fp16(scale) / s, from the packed format (code = u - zero with
+// zero-points, else u - 2^(bits-1)); one thread per word.
 __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, int64_t in,
                                      const uint32_t* __restrict__ qweight,
                                      const uint16_t* __restrict__ scales16,
+                                     const uint8_t* __restrict__ zeros,
                                      const int32_t* __restrict__ g_idx,
                                      const float* __restrict__ s, int bits, int g,
                                      uint16_t* __restrict__ dW, float* __restrict__ dW32,
@@ -539,12 +543,13 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int64_t c = wd * 8 + k;
-      const int code = static_cast<int>((word >> (4 * k)) & 0xFu) - off;
       int64_t grp = gi[k];
       if (grp < 0 || grp >= ngroups) {  // caller's group index out of range
         set_status(st, PIQ_ERR_INVALID_ARG, static_cast<int>(c));
         grp = 0;
       }
+      const int zp = zeros ? static_cast<int>(zeros[r * ngroups + grp]) : off;
+      const int code = static_cast<int>((word >> (4 * k)) & 0xFu) - zp;
       const float sc = __half2float(__ushort_as_half(scales16[r * ngroups + grp]));
       float what = static_cast<float>(code) * sc;
       if (s) what = __fdiv_rn(what, sv[k]);
@@ -629,15 +634,16 @@ int launch_scale_sumsq(double* sumsq, int64_t in, const float* s, cudaStream_t s
   return last_error();
 }
 
-int launch_pack(const int8_t* codes, const float* qscale, const int32_t* invperm, int64_t out,
-                int64_t in, int bits, int g, const float* W0, const float* cs, uint32_t* qweight,
-                uint16_t* scales16, uint16_t* dW, float* dW32, int32_t* g_idx,
-                cudaStream_t stream) {
+int launch_pack(const int8_t* codes, const float* qscale, const uint8_t* qzero,
+                const int32_t* invperm, int64_t out, int64_t in, int bits, int g,
+                const float* W0, const float* cs, uint32_t* qweight, uint16_t* scales16,
+                uint16_t* dW, float* dW32, int32_t* g_idx, cudaStream_t stream) {
   if ((dW != nullptr || dW32 != nullptr) && W0 == nullptr) return PIQ_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(cs) & 15u) != 0) return PIQ_ERR_INVALID_ARG;
   note_launch();
   pack_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
-      codes, qscale, invperm, out, in, bits, g, W0, cs, qweight, scales16, dW, dW32, g_idx);
+      codes, qscale, qzero, invperm, out, in, bits, g, W0, cs, qweight, scales16, dW, dW32,
+      g_idx);
   return last_error();
 }
 
@@ -686,13 +692,13 @@ int launch_argmin(const double* err, int n, const float* alphas_dev, int* best_i
 }
 
 int launch_dequant_delta(const float* W, int64_t out, int64_t in, const uint32_t* qweight,
-                         const uint16_t* scales16, const int32_t* g_idx, const float* s,
-                         int bits, int g, uint16_t* dW, float* dW32, DeviceStatus* st,
-                         cudaStream_t stream) {
+                         const uint16_t* scales16, const uint8_t* zeros, const int32_t* g_idx,
+                         const float* s, int bits, int g, uint16_t* dW, float* dW32,
+                         DeviceStatus* st, cudaStream_t stream) {
   if ((dW == nullptr) == (dW32 == nullptr)) return PIQ_ERR_INVALID_ARG;
   note_launch();
   dequant_delta_kernel<<<grid_for(out * (in / 8), 256), 256, 0, stream>>>(
-      W, out, in, qweight, scales16, g_idx, s, bits, g, dW, dW32, st);
+      W, out, in, qweight, scales16, zeros, g_idx, s, bits, g, dW, dW32, st);
   return last_error();
 }
 

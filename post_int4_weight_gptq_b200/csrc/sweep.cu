@@ -23,6 +23,14 @@
 // instruction cache: only the 32-column window is unrolled.  W/scale is an IEEE
 // round-to-nearest division and rintf rounds half to even (the listing's
 // np.round); the error uses the reciprocal of U[j, j].
+//
+// Asymmetric groups (qzero != NULL; a scale and zero-point per group, the
+// uplatz.com report's Group Size paragraph, formula read as min/max affine
+// rounding over a range widened to hold 0): at a group start
+// scale = (max(0, max w) - min(0, min w)) / (2^bits - 1) and
+// zero = rint(-min(0, min w) / scale); the signed code is clipped to
+// [-zero, 2^bits - 1 - zero] instead of [-qmax - 1, qmax], and zero is stored as
+// one byte per (row, group).  Everything else is the symmetric loop.
 #include <algorithm>
 #include <vector>
 
@@ -38,14 +46,15 @@ constexpr int R = 128;       // rows per CTA, one per thread
 constexpr int LDW = B + 4;   // row-state stride (float4-aligned, conflict-free per 8 lanes)
 constexpr int LDC = B + 4;   // code staging row (bytes)
 constexpr int kSweepSmem = B * B * 4 + B * 4 + R * LDW * 4 + R * LDC;
-constexpr int kQuartersSmem = kSweepSmem + R * 4;
+constexpr int kQuartersSmem = kSweepSmem + 2 * R * 4;
 
 // Per-row state of the column loop.
 struct SweepRow {
   float scale;
   float rscale;      // 1 / scale (0 when scale is 0)
   int64_t next_gs;   // block-relative column of the next group start
-  float fqmax, cmin, cmax;
+  float fqmax;       // qmax (symmetric) or 2^bits - 1 (asymmetric)
+  float cmin, cmax;  // signed code range of the current group
   int kb;
   int64_t b, in, g, ngroups, row;
   bool valid;
@@ -65,35 +74,61 @@ __device__ __forceinline__ float code_of(float w, float scale, float rscale) {
                                                                    : q;
 }
 
+// Scale, zero-point and code range of an asymmetric group from the extremes of
+// its current weights (mx = max(0, max w), mn = min(0, min w)).
+__device__ __forceinline__ void asym_params(float mx, float mn, SweepRow& st,
+                                            uint8_t* __restrict__ qzero, int64_t grp) {
+  st.scale = __fdiv_rn(mx - mn, st.fqmax);
+  float z = st.scale > 0.f ? rintf(__fdiv_rn(-mn, st.scale)) : 0.f;
+  z = fminf(fmaxf(z, 0.f), st.fqmax);
+  st.cmin = -z;
+  st.cmax = st.fqmax - z;
+  if (st.valid) qzero[st.row * st.ngroups + grp] = static_cast<uint8_t>(z);
+}
+
 // Group start at block column j (window base c0, jj = j - c0): the scale comes
 // from the current weights of [j, j+g): the window in registers, later block
 // columns in shared memory minus the updates still pending from window columns
 // before j, and (only when j is the block start) columns past the block in W.
+// Symmetric: m = max|w|.  Asymmetric: m = max(0, max w), mn = min(0, min w).
 __device__ __forceinline__ void group_start(const float (&ws)[SUB], const float (&e)[SUB], int jj,
                                             int c0, SweepRow& st, const float* __restrict__ W,
                                             const float* Us, const float* wrow,
-                                            float* __restrict__ qscale) {
+                                            float* __restrict__ qscale,
+                                            uint8_t* __restrict__ qzero) {
   const int j = c0 + jj;
   const int64_t gend = std::min<int64_t>(st.b + j + st.g, st.in);
   const int jend = static_cast<int>(std::min<int64_t>(gend - st.b, st.kb));
-  float m = 0.f;
+  const bool asym = qzero != nullptr;
+  float m = 0.f, mn = 0.f;
 #pragma unroll
   for (int k = 0; k < SUB; ++k)
-    if (k >= jj && c0 + k < jend) m = fmaxf(m, fabsf(ws[k]));
+    if (k >= jj && c0 + k < jend) {
+      m = fmaxf(m, asym ? ws[k] : fabsf(ws[k]));
+      mn = fminf(mn, ws[k]);
+    }
   for (int c = c0 + SUB; c < jend; ++c) {
     float v = wrow[c];
 #pragma unroll
     for (int p = 0; p < SUB; ++p)
       if (p < jj) v = fmaf(-e[p], Us[(c0 + p) * B + c], v);
-    m = fmaxf(m, fabsf(v));
+    m = fmaxf(m, asym ? v : fabsf(v));
+    mn = fminf(mn, v);
   }
   if (gend > st.b + st.kb && st.valid) {
     const float* src = W + st.row * st.in;
-    for (int64_t c = st.b + st.kb; c < gend; ++c) m = fmaxf(m, fabsf(src[c]));
+    for (int64_t c = st.b + st.kb; c < gend; ++c) {
+      m = fmaxf(m, asym ? src[c] : fabsf(src[c]));
+      mn = fminf(mn, src[c]);
+    }
   }
-  st.scale = __fdiv_rn(m, st.fqmax);
+  const int64_t grp = (st.b + j) / st.g;
+  if (asym)
+    asym_params(m, mn, st, qzero, grp);
+  else
+    st.scale = __fdiv_rn(m, st.fqmax);
   st.rscale = st.scale > 0.f ? __frcp_rn(st.scale) : 0.f;
-  if (st.valid) qscale[st.row * st.ngroups + (st.b + j) / st.g] = st.scale;
+  if (st.valid) qscale[st.row * st.ngroups + grp] = st.scale;
   st.next_gs += st.g;
 }
 
@@ -103,11 +138,13 @@ template <bool GENERAL, int JJ>
 __device__ __forceinline__ void sweep_col(float (&ws)[SUB], float (&e)[SUB], int c0, SweepRow& st,
                                           const float* __restrict__ W, const float* Us,
                                           const float* inv_u, const float* wrow, int8_t* code_row,
-                                          float* __restrict__ qscale) {
+                                          float* __restrict__ qscale,
+                                          uint8_t* __restrict__ qzero) {
   if constexpr (JJ < SUB) {
     const int j = c0 + JJ;
     if (j < st.kb) {
-      if (GENERAL && j == st.next_gs) group_start(ws, e, JJ, c0, st, W, Us, wrow, qscale);
+      if (GENERAL && j == st.next_gs)
+        group_start(ws, e, JJ, c0, st, W, Us, wrow, qscale, qzero);
       const float wj = ws[JJ];
       const float sc = st.scale;
       const float q = sc > 0.f ? fminf(fmaxf(code_of(wj, sc, st.rscale), st.cmin), st.cmax) : 0.f;
@@ -126,7 +163,7 @@ __device__ __forceinline__ void sweep_col(float (&ws)[SUB], float (&e)[SUB], int
     } else {
       e[JJ] = 0.f;
     }
-    sweep_col<GENERAL, JJ + 1>(ws, e, c0, st, W, Us, inv_u, wrow, code_row, qscale);
+    sweep_col<GENERAL, JJ + 1>(ws, e, c0, st, W, Us, inv_u, wrow, code_row, qscale, qzero);
   }
 }
 
@@ -138,7 +175,7 @@ __global__ void __launch_bounds__(R, 1)
     sweep_block_kernel(float* __restrict__ W, int64_t out, int64_t in,
                        const float* __restrict__ U, int64_t b, int kb, int bits, int g,
                        int8_t* __restrict__ codes, float* __restrict__ qscale,
-                       float* __restrict__ Err, DeviceStatus* st) {
+                       uint8_t* __restrict__ qzero, float* __restrict__ Err, DeviceStatus* st) {
   extern __shared__ __align__(16) float smem[];
   float* Us = smem;                     // [B][B], strictly upper part of U[b:e, b:e]
   float* inv_u = Us + B * B;            // [B], 1 / U[j][j]
@@ -188,7 +225,7 @@ __global__ void __launch_bounds__(R, 1)
 
   SweepRow rs;
   const int qmax = (1 << (bits - 1)) - 1;
-  rs.fqmax = static_cast<float>(qmax);
+  rs.fqmax = qzero ? static_cast<float>((1 << bits) - 1) : static_cast<float>(qmax);
   rs.cmin = static_cast<float>(-qmax - 1);
   rs.cmax = static_cast<float>(qmax);
   rs.kb = kb;
@@ -199,9 +236,14 @@ __global__ void __launch_bounds__(R, 1)
   rs.row = row0 + tid;
   rs.valid = rs.row < out;
   const int64_t boff = b % g;
-  // a group that started in an earlier block keeps its scale
+  // a group that started in an earlier block keeps its scale (and zero-point)
   rs.scale = (boff != 0 && rs.valid) ? qscale[rs.row * rs.ngroups + b / g] : 0.f;
   rs.rscale = rs.scale > 0.f ? __frcp_rn(rs.scale) : 0.f;
+  if (qzero && boff != 0) {
+    const float z = rs.valid ? static_cast<float>(qzero[rs.row * rs.ngroups + b / g]) : 0.f;
+    rs.cmin = -z;
+    rs.cmax = rs.fqmax - z;
+  }
   rs.next_gs = (boff == 0) ? 0 : g - boff;
 
   float* wrow = Wr + tid * LDW;
@@ -219,9 +261,9 @@ __global__ void __launch_bounds__(R, 1)
     if (!GENERAL && c0 == rs.next_gs) {
 #pragma unroll
       for (int p = 0; p < SUB; ++p) e[p] = 0.f;
-      group_start(ws, e, 0, c0, rs, W, Us, wrow, qscale);
+      group_start(ws, e, 0, c0, rs, W, Us, wrow, qscale, qzero);
     }
-    sweep_col<GENERAL, 0>(ws, e, c0, rs, W, Us, inv_u, wrow, crow, qscale);
+    sweep_col<GENERAL, 0>(ws, e, c0, rs, W, Us, inv_u, wrow, crow, qscale, qzero);
 #pragma unroll
     for (int k4 = 0; k4 < SUB / 4; ++k4)
       reinterpret_cast<float4*>(wrow + c0)[k4] =
@@ -264,13 +306,15 @@ __global__ void __launch_bounds__(QT, 1)
     sweep_quarters_kernel(float* __restrict__ W, int64_t out, int64_t in,
                           const float* __restrict__ U, int64_t b, int kb, int bits, int g,
                           int8_t* __restrict__ codes, float* __restrict__ qscale,
-                          float* __restrict__ Err, DeviceStatus* st) {
+                          uint8_t* __restrict__ qzero, float* __restrict__ Err,
+                          DeviceStatus* st) {
   extern __shared__ __align__(16) float smem[];
   float* Us = smem;                     // [B][B], strictly upper part of U[b:e, b:e]
   float* inv_u = Us + B * B;            // [B], 1 / U[j][j]
   float* Wr = inv_u + B;                // [R][LDW], row state; errors replace used columns
   int8_t* Cs = reinterpret_cast<int8_t*>(Wr + R * LDW);  // [R][LDC]
   float* scale_s = reinterpret_cast<float*>(Cs + R * LDC);  // [R]
+  float* zero_s = scale_s + R;                              // [R] (asymmetric groups)
   pdl_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // window q's four warps sit on the four schedulers (warp w issues from w % 4)
@@ -346,7 +390,7 @@ __global__ void __launch_bounds__(QT, 1)
 
   SweepRow rs;
   const int qmax = (1 << (bits - 1)) - 1;
-  rs.fqmax = static_cast<float>(qmax);
+  rs.fqmax = qzero ? static_cast<float>((1 << bits) - 1) : static_cast<float>(qmax);
   rs.cmin = static_cast<float>(-qmax - 1);
   rs.cmax = static_cast<float>(qmax);
   rs.kb = kb;
@@ -362,22 +406,42 @@ __global__ void __launch_bounds__(QT, 1)
   if (q == 0) {
     // the row's scale: a group starts here (from the current weights of
     // [b, b + g), past the block read from W), or it continues from earlier
-    float sc;
+    float sc, z = 0.f;
     if (b % g == 0) {
       const int64_t gend = std::min<int64_t>(b + g, in);
       float m = 0.f;
-      for (int c4 = 0; c4 < B / 4; ++c4) {  // columns past kb are zero
-        const float4 v = reinterpret_cast<const float4*>(wrow)[c4];
-        m = fmaxf(fmaxf(m, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+      if (qzero == nullptr) {
+        for (int c4 = 0; c4 < B / 4; ++c4) {  // columns past kb are zero
+          const float4 v = reinterpret_cast<const float4*>(wrow)[c4];
+          m = fmaxf(fmaxf(m, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+        }
+        if (rs.valid)
+          for (int64_t c = b + kb; c < gend; ++c) m = fmaxf(m, fabsf(W[rs.row * in + c]));
+        sc = __fdiv_rn(m, rs.fqmax);
+      } else {
+        // max(0, max w) and min(0, min w); zero columns past kb change neither
+        float mn = 0.f;
+        for (int c4 = 0; c4 < B / 4; ++c4) {
+          const float4 v = reinterpret_cast<const float4*>(wrow)[c4];
+          m = fmaxf(fmaxf(m, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+          mn = fminf(fminf(mn, fminf(v.x, v.y)), fminf(v.z, v.w));
+        }
+        if (rs.valid)
+          for (int64_t c = b + kb; c < gend; ++c) {
+            m = fmaxf(m, W[rs.row * in + c]);
+            mn = fminf(mn, W[rs.row * in + c]);
+          }
+        asym_params(m, mn, rs, qzero, b / g);
+        sc = rs.scale;
+        z = -rs.cmin;
       }
-      if (rs.valid)
-        for (int64_t c = b + kb; c < gend; ++c) m = fmaxf(m, fabsf(W[rs.row * in + c]));
-      sc = __fdiv_rn(m, rs.fqmax);
       if (rs.valid) qscale[rs.row * rs.ngroups + b / g] = sc;
     } else {
       sc = rs.valid ? qscale[rs.row * rs.ngroups + b / g] : 0.f;
+      if (qzero && rs.valid) z = static_cast<float>(qzero[rs.row * rs.ngroups + b / g]);
     }
     scale_s[lrow] = sc;
+    zero_s[lrow] = z;
   }
   const int c0 = SUB * q;
   // ws holds the window's weights; a used column's slot then holds its error
@@ -394,6 +458,10 @@ __global__ void __launch_bounds__(QT, 1)
   __syncthreads();
   rs.scale = scale_s[lrow];
   rs.rscale = rs.scale > 0.f ? __frcp_rn(rs.scale) : 0.f;
+  if (qzero) {
+    rs.cmin = -zero_s[lrow];
+    rs.cmax = rs.fqmax - zero_s[lrow];
+  }
 
   for (int p = 0; p < 4; ++p) {
     if (q >= p && SUB * p < kb) {
@@ -419,7 +487,7 @@ __global__ void __launch_bounds__(QT, 1)
         }
       }
       if (q == p) {
-        sweep_col<false, 0>(ws, ws, c0, rs, W, Us, inv_u, wrow, crow, qscale);
+        sweep_col<false, 0>(ws, ws, c0, rs, W, Us, inv_u, wrow, crow, qscale, qzero);
 #pragma unroll
         for (int k4 = 0; k4 < SUB / 4; ++k4)
           reinterpret_cast<float4*>(wrow + c0)[k4] =
@@ -475,7 +543,7 @@ static void block_partition(int64_t in, int g, std::vector<std::pair<int64_t, in
 }
 
 int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits, int g,
-                   int8_t* codes, float* qscale, float* Err, DeviceStatus* st,
+                   int8_t* codes, float* qscale, uint8_t* qzero, float* Err, DeviceStatus* st,
                    cudaStream_t stream) {
   static bool attr_set[64] = {};
   static bool quarters_attr[64] = {};
@@ -512,11 +580,11 @@ int run_gptq_sweep(float* Wq, int64_t out, int64_t in, const float* U, int bits,
     note_launch();
     const cudaError_t le =
         quartered ? launch_pdl(sweep_quarters_kernel, dim3(grid), dim3(QT), kQuartersSmem, stream,
-                               Wq, out, in, U, b, kb, bits, g, codes, qscale, Err, st)
+                               Wq, out, in, U, b, kb, bits, g, codes, qscale, qzero, Err, st)
         : aligned ? launch_pdl(sweep_block_kernel<false>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
-                             out, in, U, b, kb, bits, g, codes, qscale, Err, st)
+                             out, in, U, b, kb, bits, g, codes, qscale, qzero, Err, st)
                 : launch_pdl(sweep_block_kernel<true>, dim3(grid), dim3(R), kSweepSmem, stream, Wq,
-                             out, in, U, b, kb, bits, g, codes, qscale, Err, st);
+                             out, in, U, b, kb, bits, g, codes, qscale, qzero, Err, st);
     if (le != cudaSuccess) return PIQ_ERR_CUDA;
     if (e < in) {
       // W[:, e:] -= Err[:, :kb] U[b:e, e:]

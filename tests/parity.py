@@ -55,32 +55,67 @@ def fp32_drift(Wp: np.ndarray, U: np.ndarray, bits: int, g: int, ref) -> float:
     return drift
 
 
+def _sweep(Wr, U, bits, g, asym, force=None, force_zero=None):
+    """(codes, scales, zeros, zv, v) of the oracle's literal loop."""
+    if asym:
+        c, s, z, zv, v, _ = O.gptq_sweep_asym_ref(Wr, U, bits, g, force=force,
+                                                  force_zero=force_zero)
+        return c, s, z, zv, v
+    c, s, v, _ = O.gptq_sweep_ref(Wr, U, bits, g, force=force)
+    return c, s, None, None, v
+
+
 def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray, bits: int,
-                           g: int, ref=None, max_iters: int = 64, tie_tol: float = TIE_TOL):
-    """gpu_codes, Wp in quantization order.  Returns (stats, forced oracle run on
-    all rows) and raises AssertionError on a contract violation."""
+                           g: int, ref=None, max_iters: int = 64, tie_tol: float = TIE_TOL,
+                           gpu_zeros: np.ndarray | None = None):
+    """gpu_codes (signed), Wp in quantization order.  Returns (stats, codes,
+    scales) of the forced oracle run on all rows, plus its zero-points when
+    ``gpu_zeros`` ([out, ngroups], asymmetric groups) is given; raises
+    AssertionError on a contract violation.  A zero-point is a rounded value
+    too (-lo / scale): where the GPU's differs, the oracle's unrounded value
+    must be within the tie window of a half-integer, and it is forced like a
+    code."""
+    asym = gpu_zeros is not None
     gpu_codes = np.asarray(gpu_codes, dtype=np.int16)
     if ref is None:
-        ref = O.gptq_sweep_ref(Wp, U, bits, g)
-    codes0, scales0, v0, _ = ref
+        codes0, scales0, zeros0, _, _ = _sweep(Wp, U, bits, g, asym)
+    else:
+        codes0, scales0 = ref[0], ref[1]
+        zeros0 = None
     mism0 = gpu_codes != codes0
+    zmism0 = (gpu_zeros != zeros0) if asym else np.zeros((Wp.shape[0], 1), dtype=bool)
     n0 = int(mism0.sum())
     total = gpu_codes.size
-    stats = {"mismatches": n0, "total": total, "frac": n0 / total, "forced": 0, "iters": 0}
+    stats = {"mismatches": n0, "total": total, "frac": n0 / total, "forced": 0, "iters": 0,
+             "forced_zeros": 0}
     codes, scales = codes0.copy(), scales0.copy()
-    rows = np.unique(np.nonzero(mism0)[0])
+    zeros = zeros0.copy() if asym else None
+    rows = np.unique(np.concatenate([np.nonzero(mism0)[0], np.nonzero(zmism0)[0]]))
     if rows.size:
         force = np.full((rows.size, gpu_codes.shape[1]), NO_FORCE, dtype=np.int16)
+        fz = np.full((rows.size, scales0.shape[1]), NO_FORCE, dtype=np.int16) if asym else None
         Wr = Wp[rows]
         for it in range(max_iters):
-            c, s, v, _ = O.gptq_sweep_ref(Wr, U, bits, g, force=force)
+            c, s, z, zv, v = _sweep(Wr, U, bits, g, asym, force, fz)
             d = c != gpu_codes[rows]
+            dz = (z != gpu_zeros[rows]) if asym else np.zeros((rows.size, 1), dtype=bool)
             stats["iters"] = it + 1
-            if not d.any():
+            if not d.any() and not dz.any():
                 codes[rows], scales[rows] = c, s
+                if asym:
+                    zeros[rows] = z
                 break
-            for k in np.nonzero(d.any(axis=1))[0]:
-                j = int(np.argmax(d[k]))           # first mismatch of the row
+            for k in np.nonzero(d.any(axis=1) | dz.any(axis=1))[0]:
+                j = int(np.argmax(d[k])) if d[k].any() else gpu_codes.shape[1]
+                jz = int(np.argmax(dz[k])) if dz[k].any() else None
+                if jz is not None and jz * g <= j:   # the group's zero-point differs first
+                    td = float(tie_distance(zv[k, jz]))
+                    assert td < tie_tol, (
+                        f"row {rows[k]} group {jz}: GPU zero-point {gpu_zeros[rows[k], jz]} vs "
+                        f"oracle {z[k, jz]} at -lo/scale = {zv[k, jz]!r} (tie distance {td:.3g})")
+                    fz[k, jz] = gpu_zeros[rows[k], jz]
+                    stats["forced_zeros"] += 1
+                    continue
                 td = float(tie_distance(v[k, j]))
                 assert td < tie_tol, (
                     f"row {rows[k]} col {j}: GPU code {gpu_codes[rows[k], j]} vs oracle "
@@ -89,8 +124,10 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
                 stats["forced"] += 1
         else:
             raise AssertionError("teacher forcing did not converge")
-    assert stats["forced"] <= MAX_MISMATCH_FRAC * total, (
+    assert stats["forced"] + stats["forced_zeros"] <= MAX_MISMATCH_FRAC * total, (
         f"{stats['forced']} of {total} codes decided differently")
+    if asym:
+        return stats, codes, scales, zeros
     return stats, codes, scales
 
 
