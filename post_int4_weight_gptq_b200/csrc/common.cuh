@@ -178,6 +178,12 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// Two floats to bf16 (round to nearest even) in one conversion: a in the low
+// half, b in the high half of the word.
+__device__ __forceinline__ uint32_t floats_to_bf16x2_bits(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
 
 // generic-proxy writes to shared memory become visible to the async proxy (TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -226,14 +226,11 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
       dst[1] = make_float4(d32[4], d32[5], d32[6], d32[7]);
     }
     if (dW) {
-      uint16_t d16[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) d16[k] = float_to_bf16_bits(d32[k]);
       uint4 o;
-      o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
-      o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
-      o.z = d16[4] | (static_cast<uint32_t>(d16[5]) << 16);
-      o.w = d16[6] | (static_cast<uint32_t>(d16[7]) << 16);
+      o.x = floats_to_bf16x2_bits(d32[0], d32[1]);
+      o.y = floats_to_bf16x2_bits(d32[2], d32[3]);
+      o.z = floats_to_bf16x2_bits(d32[4], d32[5]);
+      o.w = floats_to_bf16x2_bits(d32[6], d32[7]);
       *reinterpret_cast<uint4*>(dW + r * in + wd * 8) = o;
     }
   }
@@ -561,14 +558,11 @@ __global__ void dequant_delta_kernel(const float* __restrict__ W, int64_t out, i
       dst[1] = make_float4(d32[4], d32[5], d32[6], d32[7]);
       continue;
     }
-    uint16_t d16[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) d16[k] = float_to_bf16_bits(d32[k]);
     uint4 o;
-    o.x = d16[0] | (static_cast<uint32_t>(d16[1]) << 16);
-    o.y = d16[2] | (static_cast<uint32_t>(d16[3]) << 16);
-    o.z = d16[4] | (static_cast<uint32_t>(d16[5]) << 16);
-    o.w = d16[6] | (static_cast<uint32_t>(d16[7]) << 16);
+    o.x = floats_to_bf16x2_bits(d32[0], d32[1]);
+    o.y = floats_to_bf16x2_bits(d32[2], d32[3]);
+    o.z = floats_to_bf16x2_bits(d32[4], d32[5]);
+    o.w = floats_to_bf16x2_bits(d32[6], d32[7]);
     *reinterpret_cast<uint4*>(dW + r * in + wd * 8) = o;
   }
 }
