@@ -398,6 +398,22 @@ def run_ours(args):
     return 0
 
 
+def hbm_phase_rates(phases_ms, n, inp, out, n_alpha, hbm_peak_gbs):
+    """Achieved HBM rate of AWQ's bandwidth-bound phases: algorithmic bytes
+    (X read once for mean|x|: n*in*2; W read once and the n_alpha bf16 deltas
+    written: out*in*4 + n_alpha*out*in*2) over the phase's measured time.  A
+    phase time also holds its small launches (the grid copy, the finishing
+    sums, the scale table), so these are lower bounds on the kernels' own."""
+    algo = {"colstats": n * inp * 2, "quant_delta": out * inp * 4 + n_alpha * out * inp * 2}
+    res = {}
+    for k, b in algo.items():
+        ms = phases_ms.get(k)
+        if ms:
+            gbs = b / (ms / 1e3) / 1e9
+            res[k] = {"bytes": b, "gb_per_s": gbs, "frac": gbs / hbm_peak_gbs}
+    return res
+
+
 def run_awq(dev, steps=3, warmup=1):
     """AWQ alpha search (20-point grid) on the 8192x8192 layer: ms per layer."""
     import torch
@@ -423,9 +439,12 @@ def run_awq(dev, steps=3, warmup=1):
     piq.set_timing(False)
     ph = {k: statistics.mean(v) for k, v in ph.items()}
     flops = 2.0 * C5.n * C5.inp * C5.out * len(AWQ_GRID)
+    peaks, src = load_peaks()
     return {"workload": "AWQ 20-point alpha search: W 8192x8192, X 16384x8192",
             "ms_per_layer": statistics.median(times), "best_alpha": r.best_alpha,
-            "phases_ms": ph, "error_gemm_tflops": flops / (ph["error_gemm"] / 1e3) / 1e12}
+            "phases_ms": ph, "error_gemm_tflops": flops / (ph["error_gemm"] / 1e3) / 1e12,
+            "hbm": hbm_phase_rates(ph, C5.n, C5.inp, C5.out, len(AWQ_GRID), peaks["hbm_gbs"]),
+            "hbm_peak_source": f"{src} hbm_gbs"}
 
 
 def run_variants(dev, Wg, Xg, steps=5, warmup=3):

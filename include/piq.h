@@ -20,6 +20,11 @@
  *           W diag(s) rounded to nearest, one alpha per layer chosen by grid
  *           search on the calibration output error ||X W^T - X What^T||^2.
  *
+ * Two widenings of GPTQ: AWQ's scaling first and GPTQ's rounding after (the
+ * same page's serving decision list: the two compose; awq_gptq_quantize_layer),
+ * and a scale plus a zero-point per group (the uplatz.com report, GPTQ's key
+ * parameters, Group Size; gptq_quantize_layer_asym).
+ *
  * Conventions for every entry point:
  *  - Pointers marked "device" are CUDA device pointers of the current device;
  *    "host" pointers are ordinary host memory.  The caller owns every buffer.

@@ -75,3 +75,32 @@ def test_bad_arguments_rejected_before_any_device_work(lib):
 def test_library_is_sm100a_only(lib):
     # every kernel was compiled for sm_100a alone
     assert "-gencode" in piq_build.ARCH and "arch=compute_100a,code=sm_100a" in piq_build.ARCH
+
+
+def test_widened_entries_reject_missing_buffers(lib):
+    # the zero-point buffer of the asymmetric entry and the channel scales of
+    # the composed entry are required; a misaligned s is refused (the pointer
+    # is only checked, never read)
+    null = None
+    err = ctypes.c_double()
+    rc = lib.gptq_quantize_layer_asym(null, 16, 64, null, 64, 4, 32, 0.01, 0, null, null, null,
+                                      null, null, ctypes.byref(err), null, 0, null)
+    assert rc == piq.PIQ_ERR_INVALID_ARG
+    for s_ptr in (None, ctypes.c_void_p(4)):
+        rc = lib.awq_gptq_quantize_layer(null, 16, 64, null, 64, s_ptr, 4, 32, 0.01, 0, null,
+                                         null, null, null, ctypes.byref(err), null, 0, null)
+        assert rc == piq.PIQ_ERR_INVALID_ARG
+    rc = lib.piq_layer_output_error(null, 16, 64, null, null, null, null, null, 7, 32, null, 64,
+                                    ctypes.byref(err), null, 0, null)
+    assert rc == piq.PIQ_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    W = torch.zeros(16, 64)
+    X = torch.zeros(64, 64, dtype=torch.bfloat16)
+    s = torch.ones(64)
+    with pytest.raises(TypeError):
+        piq.gptq_quantize_layer(W, X, sym=False)
+    with pytest.raises(TypeError):
+        piq.awq_gptq_quantize_layer(W, X, s)
