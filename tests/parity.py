@@ -76,6 +76,8 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
     must be within the tie window of a half-integer, and it is forced like a
     code."""
     asym = gpu_zeros is not None
+    if asym and ref is not None:
+        raise ValueError("a precomputed ref carries no zero-points; pass ref=None")
     gpu_codes = np.asarray(gpu_codes, dtype=np.int16)
     if ref is None:
         codes0, scales0, zeros0, _, _ = _sweep(Wp, U, bits, g, asym)
