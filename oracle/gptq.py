@@ -180,8 +180,9 @@ def gptq_sweep_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
     ``force`` (int array [out, in], NO_FORCE where free) replaces the rounded
     code at chosen sites: the teacher-forcing hook of the parity comparison.
     ``dtype`` is the working precision: float64 is the oracle; float32 runs the
-    same loop in the precision the benchmark spec fixes for the sweep, to measure
-    how far that arithmetic alone drifts from float64 (the parity tie window)."""
+    same loop in float32, the working precision of the GPU sweep and its block
+    updates, to measure how far that arithmetic alone drifts from float64 (the
+    parity tie window)."""
     codes, scales, _, _, vlog, elog = _sweep(Wp, U, bits, g, True, force, None, log, dtype)
     return codes, scales, vlog, elog
 

@@ -9,7 +9,7 @@ on the affected rows with the GPU's code forced at the first mismatching site
 mismatches.  Scales and output errors then agree within 1e-3 relative.
 
 The tie window is 1e-4, or twice the drift of the same loop run in float32 (the
-precision the benchmark spec fixes for the sweep) when that is larger: over tens of
+working precision of the GPU sweep and its block updates) when that is larger: over tens of
 thousands of columns float32 arithmetic alone moves w/scale by up to ~2e-4 from
 float64, so closer decisions are not fixed by the method at that precision.
 """

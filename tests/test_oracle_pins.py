@@ -364,7 +364,7 @@ def test_hessian_sizes_printed_on_the_page():
 
 def test_sweep_working_precision():
     # float64 is the oracle (the default); the float32 mode runs the same loop in
-    # the sweep precision the benchmark spec fixes, and on the tiny layer it drifts
+    # the GPU sweep's working precision, and on the tiny layer it drifts
     # from float64 by far less than the 1e-4 tie window, deciding every code the
     # same way away from ties
     from tests.parity import fp32_drift, tie_distance
