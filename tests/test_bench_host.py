@@ -21,3 +21,31 @@ def test_awq_hbm_phase_rates():
 
 def test_awq_hbm_phase_rates_skip_missing_phases():
     assert bench.hbm_phase_rates({}, 16, 8, 8, 1, 1000.0) == {}
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    # the oracle arm's JSON line, with the timed oracle sample stubbed (its real
+    # run takes about ten seconds a step)
+    import json
+    import numpy as np
+    monkeypatch.setattr(bench, "make_inputs",
+                        lambda rank, n=None: (np.zeros((8, 8), np.float32),
+                                              np.zeros((4, 8), np.uint16),
+                                              np.zeros((4, 8), np.uint16)))
+    monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: (2.0, "stub sample"))
+    assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] == pytest.approx(4096 * 4096 / 2.0 / 1e6)
+    assert line["higher_is_better"] is True and line["steps"] == 2 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["sample"] == "stub sample"
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "workload" in line["config"] and "model" not in line["config"]
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
