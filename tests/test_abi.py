@@ -104,3 +104,23 @@ def test_binding_refuses_host_tensors(lib):
         piq.gptq_quantize_layer(W, X, sym=False)
     with pytest.raises(TypeError):
         piq.awq_gptq_quantize_layer(W, X, s)
+
+
+def test_empty_and_oversized_layers_rejected(lib):
+    # empty layers (no rows, no inputs, no samples) and sizes past the supported
+    # maximum are refused before any device work; the fake buffer address is
+    # aligned and never read
+    fake = ctypes.c_void_p(1 << 12)
+    err = ctypes.c_double()
+    out = ctypes.c_size_t()
+    for rows, inp, n in ((0, 64, 64), (16, 0, 64), (16, 64, 0), ((1 << 24) + 1, 64, 64),
+                         (16, (1 << 20) + 8, 64)):
+        rc = lib.gptq_quantize_layer(fake, rows, inp, fake, n, 4, 32, 0.01, 0, fake, fake, None,
+                                     None, ctypes.byref(err), fake, 1 << 30, None)
+        assert rc == piq.PIQ_ERR_INVALID_ARG, (rows, inp, n)
+        grid = (ctypes.c_float * 2)(0.0, 0.5)
+        rc = lib.awq_search_layer(fake, rows, inp, fake, n, 4, 32, grid, 2, None, fake, fake,
+                                  fake, None, fake, 1 << 30, None)
+        assert rc == piq.PIQ_ERR_INVALID_ARG, (rows, inp, n)
+    for args in ((0, 64, 64, 0), (16, 0, 64, 0), (16, 64, 0, 0)):
+        assert lib.piq_gptq_workspace_bytes(*args, ctypes.byref(out)) == piq.PIQ_ERR_INVALID_ARG
