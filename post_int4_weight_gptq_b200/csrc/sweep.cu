@@ -7,7 +7,9 @@
 // gets W[:, k] -= err * U[j, k].  The remark after the listing batches the
 // updates over column blocks: inside a block the updates are applied at once
 // (here, in registers), and the block's errors update all later columns with
-// one GEMM, W[:, e:] -= Err[:, b:e] U[b:e, e:] (simt_gemm.cu).
+// one GEMM, W[:, e:] -= Err[:, b:e] U[b:e, e:] (FP32-accurate: three TF32
+// tensor-core passes, tc_sgemm.cu; the SIMT kernel of simt_gemm.cu where the
+// operands do not suit TMA).
 //
 // Blocks are at most 128 wide and are cut so that every group start is either
 // a block start or has its whole group inside its block; a group scale then
