@@ -82,6 +82,9 @@ def test_zero_inputs_not_positive_definite():
     with pytest.raises(piq.PiqError) as e:
         piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X))
     assert e.value.status == piq.PIQ_ERR_NOT_PD
+    # the status is per call: the next call on the same context succeeds
+    out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(make_x_bits(C1)))
+    assert np.isfinite(out.err) and out.err > 0
 
 
 def test_workspace_too_small():
