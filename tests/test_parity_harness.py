@@ -44,8 +44,9 @@ def test_planted_code_error_is_rejected():
 
 
 def test_planted_tie_flip_is_accepted_and_counted():
-    # flip the code at the row's closest tie (made exact: w/scale on the tie),
-    # then let the loop continue from the flipped code: a legal tie decision
+    # flip the code at the row's closest tie and let the loop continue from the
+    # flipped code; with a window just wide enough to hold that tie the
+    # comparison must accept it as one forced decision
     Wp, U = _layer(4, 128, 13)
     c, s, v, _ = O.gptq_sweep_ref(Wp, U, 4, 128)
     row = 7
