@@ -1,0 +1,100 @@
+"""Oracle invariants over many small random layers (hypothesis, derandomized).
+
+Each property is one the pages and the mathematics fix, checked on layers the
+fixed pins do not cover (odd widths, group sizes, bit widths, both quantizers):
+the factorisation's error identity, blocked = literal, a diagonal Hessian
+reducing to rounding, and s = 1 reducing the composition to plain GPTQ.
+"""
+import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle as O
+from oracle.gptq import gptq_sweep_asym_ref, gptq_sweep_blocked_asym_ref
+from oracle.pack import to_memory_order
+from workloads import bf16_bits_from_f32
+
+SETTINGS = settings(derandomize=True, max_examples=60, deadline=None)
+
+
+def _layer(seed, out, inp, n, corr):
+    rng = np.random.default_rng(seed)
+    Z = rng.standard_normal((n, inp))
+    X = Z + corr * np.roll(Z, 1, axis=1)
+    X *= rng.lognormal(0, 0.6, inp)
+    W = rng.standard_normal((out, inp)) * 0.02 + 0.005 * rng.standard_normal((out, 1))
+    return W.astype(np.float32), bf16_bits_from_f32(X.astype(np.float32))
+
+
+layers = st.fixed_dictionaries({
+    "seed": st.integers(0, 10_000),
+    "out": st.integers(1, 6),
+    "inp": st.sampled_from([8, 16, 24, 40, 64, 96]),
+    "g": st.sampled_from([4, 8, 12, 16, 32, 1000]),
+    "bits": st.sampled_from([2, 3, 4]),
+    "act": st.booleans(),
+    "sym": st.booleans(),
+    "corr": st.floats(0.0, 0.9),
+})
+
+
+@SETTINGS
+@given(layers)
+def test_error_identity(p):
+    # sum err^2 = tr(dW H_d dW^T) = ||X dW^T||^2 + lam ||dW||^2 for every layer
+    W, X = _layer(p["seed"], p["out"], p["inp"], 4 * p["inp"], p["corr"])
+    g = min(p["g"], p["inp"])
+    r = O.gptq_ref(W, X, bits=p["bits"], g=g, act_order=p["act"], sym=p["sym"])
+    Q_q = r.codes * r.scales[:, np.arange(p["inp"]) // g]
+    dW = W.astype(np.float64) - to_memory_order(Q_q, r.perm)
+    lhs = float(np.sum(r.err ** 2)) - r.lam * float(np.sum(dW ** 2))
+    rhs = O.output_error_ref(W, W.astype(np.float64) - dW, X)
+    assert abs(lhs - rhs) <= 1e-9 * max(abs(rhs), 1e-30) + 1e-18
+
+
+@SETTINGS
+@given(layers)
+def test_blocked_equals_literal(p):
+    W, X = _layer(p["seed"], p["out"], p["inp"], 4 * p["inp"], p["corr"])
+    _, U, _ = O.gptq_prepare_ref(O.hessian_ref(X), 0.01, False)
+    Wp = W.astype(np.float64)
+    g, bits = p["g"], p["bits"]
+    if p["sym"]:
+        c1, s1, _, _ = O.gptq_sweep_ref(Wp, U, bits, g)
+        c2, s2, _ = O.gptq.gptq_sweep_blocked_ref(Wp, U, bits, g, block=16)
+        z1 = z2 = None
+    else:
+        c1, s1, z1, _, _, _ = gptq_sweep_asym_ref(Wp, U, bits, g)
+        c2, s2, z2, _ = gptq_sweep_blocked_asym_ref(Wp, U, bits, g, block=16)
+    assert np.array_equal(c1, c2)
+    assert np.allclose(s1, s2, rtol=1e-12, atol=0)
+    if z1 is not None:
+        assert np.array_equal(z1, z2)
+
+
+@SETTINGS
+@given(layers)
+def test_diagonal_hessian_is_rounding(p):
+    rng = np.random.default_rng(p["seed"])
+    inp, n = p["inp"], 8 * p["inp"]
+    Xf = np.zeros((n, inp), dtype=np.float32)
+    Xf[np.arange(n), rng.integers(0, inp, n)] = rng.standard_normal(n).astype(np.float32)
+    X = bf16_bits_from_f32(Xf)
+    W, _ = _layer(p["seed"], p["out"], inp, 4, 0.0)
+    r = O.gptq_ref(W, X, bits=p["bits"], g=p["g"], sym=p["sym"])
+    if p["sym"]:
+        c, s = O.rtn_ref(W, p["bits"], p["g"])
+    else:
+        c, s, z = O.rtn_asym_ref(W, p["bits"], p["g"])
+        assert np.array_equal(r.zeros, z)
+    assert np.array_equal(r.codes, c) and np.array_equal(r.scales, s)
+
+
+@SETTINGS
+@given(layers)
+def test_unit_scales_compose_to_plain_gptq(p):
+    W, X = _layer(p["seed"], p["out"], p["inp"], 4 * p["inp"], p["corr"])
+    a = O.awq_gptq_ref(W, X, np.ones(p["inp"]), bits=p["bits"], g=p["g"], act_order=p["act"])
+    b = O.gptq_ref(W, X, bits=p["bits"], g=p["g"], act_order=p["act"])
+    assert np.array_equal(a.perm, b.perm) and np.array_equal(a.codes, b.codes)
+    assert np.array_equal(a.scales, b.scales)
