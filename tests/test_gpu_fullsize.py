@@ -94,3 +94,64 @@ def test_awq_8192_full():
     srt = np.sort(ref.err)
     if (srt[1] - srt[0]) / srt[0] >= 1e-4:
         assert res.best_alpha == np.float32(ref.best_alpha)
+
+
+def _widened_full(spec, s=None, sym=True, sample_rows=48):
+    """Full-size parity of the AWQ-scaled call (channel scales s) or of
+    asymmetric groups (sym=False) on one layer, as _gptq_full does for plain
+    GPTQ.  The oracle's Hessian is that of X diag(1/s), summed over row chunks."""
+    from oracle.gptq import gptq_sweep_asym_ref, gptq_sweep_blocked_asym_ref
+    W, X = make_weight(spec), make_x_bits(spec)
+    Wg, Xg = to_gpu_w(W), to_gpu_x(X)
+    if s is not None:
+        import torch
+        out = piq.awq_gptq_quantize_layer(Wg, Xg, torch.from_numpy(s).cuda(), spec.bits, spec.g,
+                                          spec.damp, spec.act_order)
+    else:
+        out = piq.gptq_quantize_layer(Wg, Xg, spec.bits, spec.g, spec.damp, spec.act_order,
+                                      sym=sym)
+    bits, g = spec.bits, spec.g
+    s64 = np.ones(W.shape[1]) if s is None else s.astype(np.float64)
+    H = np.zeros((W.shape[1], W.shape[1]))
+    for r0 in range(0, X.shape[0], 8192):
+        xc = O.x_to_f64(X[r0:r0 + 8192]) / s64[None, :]
+        H += xc.T @ xc
+    perm, U, _ = O.gptq_prepare_ref(H, spec.damp, spec.act_order)
+    del H
+    assert np.array_equal(out.perm.cpu().numpy(), perm)
+    Wp = (W.astype(np.float64) * s64[None, :])[:, perm]
+    rows = np.sort(np.random.default_rng(123).choice(W.shape[0], sample_rows, replace=False))
+    g_idx = O.g_idx_ref(perm, g)
+    if sym:
+        codes_q = unpack_gpu(out.qweight, bits)[rows][:, perm]
+        stats, _, s_ref = teacher_forced_compare(codes_q, Wp[rows], U, bits, g)
+    else:
+        z_gpu = out.zeros.cpu().numpy().astype(np.int16)
+        u = unpack_gpu(out.qweight, bits) + 2 ** (bits - 1)
+        codes_q = (u - z_gpu[:, g_idx])[rows][:, perm]
+        stats, _, s_ref, _ = teacher_forced_compare(codes_q, Wp[rows], U, bits, g,
+                                                    gpu_zeros=z_gpu[rows])
+    sc_gpu = out.scales.cpu().numpy().astype(np.float64)[rows]
+    s16 = s_ref.astype(np.float16).astype(np.float64)
+    live = s16 > 0
+    assert (np.abs(sc_gpu[live] - s16[live]) / s16[live]).max() < REL_TOL
+    if sym:
+        c_all, sc_all, _ = gptq_sweep_blocked_ref(Wp, U, bits, g)
+    else:
+        c_all, sc_all, _, _ = gptq_sweep_blocked_asym_ref(Wp, U, bits, g)
+    What = dequant_ref(c_all, sc_all, perm, g) / s64[None, :]
+    e_ref = O.output_error_ref(W, What, X)
+    assert rel(out.err, e_ref) < REL_TOL, (out.err, e_ref)
+    return stats
+
+
+@pytest.mark.skipif(not SLOW, reason="minutes of host float64; PIQ_FULLSIZE_SLOW=1")
+def test_q_proj_7b_awq_scaled_full():
+    # the q_proj layer through awq_gptq_quantize_layer with seeded channel scales
+    from workloads import make_channel_scales
+    _widened_full(C2, s=make_channel_scales(C2.inp, 7, 0.5))
+
+
+@pytest.mark.skipif(not SLOW, reason="minutes of host float64; PIQ_FULLSIZE_SLOW=1")
+def test_q_proj_7b_asym_full():
+    _widened_full(C2, sym=False)
