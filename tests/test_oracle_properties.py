@@ -98,3 +98,34 @@ def test_unit_scales_compose_to_plain_gptq(p):
     b = O.gptq_ref(W, X, bits=p["bits"], g=p["g"], act_order=p["act"])
     assert np.array_equal(a.perm, b.perm) and np.array_equal(a.codes, b.codes)
     assert np.array_equal(a.scales, b.scales)
+
+
+awq_layers = st.fixed_dictionaries({
+    "seed": st.integers(0, 10_000),
+    "out": st.integers(1, 6),
+    "inp": st.sampled_from([16, 32, 64, 96]),
+    "g": st.sampled_from([8, 16, 32, 1000]),
+    "bits": st.sampled_from([2, 3, 4]),
+    "k": st.integers(-3, 3),
+})
+
+
+@settings(derandomize=True, max_examples=40, deadline=None)
+@given(awq_layers)
+def test_awq_search_properties(p):
+    # alpha = 0 is plain group rounding; the chosen alpha is the first minimum
+    # of the scored errors; s -> 2^k s keeps the codes (scales x 2^k)
+    from oracle.awq import awq_dequant_ref
+    W, X = _layer(p["seed"], p["out"], p["inp"], 4 * p["inp"], 0.5)
+    grid = [0.0, 0.25, 0.5, 0.75]
+    a = O.awq_ref(W, X, p["bits"], p["g"], grid)
+    c, s = O.rtn_ref(W, p["bits"], p["g"])
+    g = min(p["g"], p["inp"])
+    e_rtn = O.output_error_ref(W, awq_dequant_ref(c, s, np.ones(p["inp"]), g), X)
+    assert abs(a.err[0] - e_rtn) <= 1e-12 * max(e_rtn, 1e-300)
+    assert a.best_index == int(np.flatnonzero(a.err == a.err.min())[0])
+    s_best = O.awq_scales_ref(a.m, grid[a.best_index])
+    c1, sc1 = O.group_rtn_ref(W * s_best[None, :], p["bits"], p["g"])
+    c2, sc2 = O.group_rtn_ref(W * (2.0 ** p["k"] * s_best)[None, :], p["bits"], p["g"])
+    assert np.array_equal(c1, a.codes) and np.array_equal(c1, c2)
+    assert np.array_equal(sc2, 2.0 ** p["k"] * sc1)
