@@ -238,6 +238,13 @@ const char* piq_phase_name(int i);
  * a monotone diagnostic counter. */
 uint64_t piq_kernel_launches(void);
 
+/* Number of FP32-accurate GEMMs (the factor's panel updates and the sweep's
+ * trailing updates) that ran on the SIMT FP32 kernel instead of the tensor
+ * cores because an operand's base or row stride was not 16-byte aligned, as a
+ * tensor-memory-accelerator copy requires.  Process-wide, monotone; both paths
+ * give FP32-accurate results, the SIMT one more slowly. */
+uint64_t piq_simt_gemm_fallbacks(void);
+
 /* The last CUDA runtime error this library saw, as "<error name> in <where>"
  * ("" if none): what lies behind a PIQ_ERR_CUDA return (a launch the runtime
  * refused, or a kernel that failed, found when the call synchronized).
@@ -255,10 +262,18 @@ const char* piq_last_cuda_error(void);
  * region inside this library (a file-scope __device__ array of about 2.4 MB
  * that every GPU which loads the library keeps until the process exits).
  *   - in <= PIQ_NOALLOC_MAX_IN (512); a larger in returns PIQ_ERR_INVALID_ARG
- *     and does nothing.  No device memory is allocated or freed.
- *   - The first call on a device looks up the region's device address for that
- *     device (cudaGetSymbolAddress, with that device current); make that first
- *     call before capturing any stream.
+ *     and does nothing.  The call itself allocates and frees nothing.
+ *   - The region is created by the CUDA driver when it loads this library's
+ *     code onto a device.  With lazy module loading (CUDA's default) that
+ *     happens at the first use on the device, which may be this entry's first
+ *     call; a caller that must see no allocation at call time makes one
+ *     warm-up call at initialisation (or sets CUDA_MODULE_LOADING=EAGER).
+ *   - The first call on a device also looks up the region's device address
+ *     for that device (cudaGetSymbolAddress, with that device current); make
+ *     that first call before capturing any stream.
+ *   - Errors: PIQ_ERR_INVALID_ARG for bad arguments, PIQ_ERR_NOT_PD as for
+ *     piq_upper_factor, PIQ_ERR_CUDA for a failed runtime call (its name is
+ *     then reported by piq_last_cuda_error).
  *   - All calls on a device share the one region, which keeps the last call's
  *     contents (the status word is cleared on every call).  Calls that overlap
  *     on the GPU (different streams or threads) race on it: serialise them.

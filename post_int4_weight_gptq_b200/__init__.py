@@ -84,6 +84,7 @@ SIGNATURES = {
                                       ctypes.POINTER(_c_int)]),
     "piq_phase_name": (ctypes.c_char_p, [_c_int]),
     "piq_kernel_launches": (ctypes.c_uint64, []),
+    "piq_simt_gemm_fallbacks": (ctypes.c_uint64, []),
     "piq_last_cuda_error": (ctypes.c_char_p, []),
     "piq_upper_factor_noalloc": (_c_int, [_vp, _c_i64, _c_float, _vp, _vp,
                                           ctypes.POINTER(ctypes.c_double), _vp]),
@@ -371,6 +372,12 @@ def last_phase_times() -> dict:
 def kernel_launches() -> int:
     """Kernels launched by libpiq in this process so far."""
     return int(load_library().piq_kernel_launches())
+
+
+def simt_gemm_fallbacks() -> int:
+    """FP32-accurate GEMMs that ran on the SIMT kernel instead of the tensor
+    cores (an operand not 16-byte aligned), in this process so far."""
+    return int(load_library().piq_simt_gemm_fallbacks())
 
 
 NOALLOC_MAX_IN = 512

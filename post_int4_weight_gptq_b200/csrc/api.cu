@@ -33,7 +33,8 @@ int device_info(DeviceInfo* out) {
     have[dev] = true;
   }
   *out = cache[dev];
-  return cache[dev].major == 10 ? PIQ_OK : PIQ_ERR_UNSUPPORTED_DEVICE;
+  // the library holds sm_100a code only: compute capability 10.0 exactly
+  return (cache[dev].major == 10 && cache[dev].minor == 0) ? PIQ_OK : PIQ_ERR_UNSUPPORTED_DEVICE;
 }
 
 static std::atomic<uint64_t> g_launches{0};
@@ -44,6 +45,24 @@ static char g_err_text[160] = "";
 void note_cuda_error(cudaError_t e, const char* where) {
   std::lock_guard<std::mutex> lock(g_err_mu);
   snprintf(g_err_text, sizeof(g_err_text), "%s in %s", cudaGetErrorName(e), where);
+}
+
+int cuda_rc(cudaError_t e) {
+  if (e != cudaSuccess) note_cuda_error(e, "runtime call");
+  return e == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+// Read the status word (and optional extra device bytes) after synchronizing.
+int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st) {
+  DeviceStatus tmp;
+  cudaError_t e = cudaMemcpyAsync(&tmp, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    note_cuda_error(e, "stream synchronization (a kernel of this call failed)");
+    return PIQ_ERR_CUDA;
+  }
+  if (host_st) *host_st = tmp;
+  return tmp.code;
 }
 
 namespace {
@@ -124,24 +143,6 @@ struct PhaseClock {
     g_timing.last_kind = g_timing.kind;
   }
 };
-
-int cuda_rc(cudaError_t e) {
-  if (e != cudaSuccess) note_cuda_error(e, "runtime call");
-  return e == cudaSuccess ? PIQ_OK : PIQ_ERR_CUDA;
-}
-
-// Read the status word (and optional extra device bytes) after synchronizing.
-int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st) {
-  DeviceStatus tmp;
-  cudaError_t e = cudaMemcpyAsync(&tmp, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) {
-    note_cuda_error(e, "stream synchronization (a kernel of this call failed)");
-    return PIQ_ERR_CUDA;
-  }
-  if (host_st) *host_st = tmp;
-  return tmp.code;
-}
 
 #define PIQ_TRY(expr)             \
   do {                            \
@@ -642,6 +643,8 @@ int piq_last_phase_times(double* ms, int max_phases, int* n_phases) {
 }
 
 uint64_t piq_kernel_launches(void) { return g_launches.load(); }
+
+uint64_t piq_simt_gemm_fallbacks(void) { return simt_gemm_fallbacks(); }
 
 const char* piq_last_cuda_error(void) {
   std::lock_guard<std::mutex> lock(g_err_mu);

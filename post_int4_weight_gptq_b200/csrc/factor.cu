@@ -13,7 +13,8 @@
 //   3. right-looking blocked Cholesky, 128-wide panels: each diagonal block is
 //      factored and inverted in shared memory (chol_inv_kernel), the panel
 //      below is L21 = A21 inv(L11)^T and the trailing matrix A22 -= L21 L21^T
-//      (FP32 SIMT GEMMs that skip the zero triangles)
+//      (FP32-accurate tensor-core GEMMs, three TF32 passes, that skip the zero
+//      triangles)
 //   4. X = inv(L) from the diagonal inverses, merging pairs of s-blocks level by
 //      level (s = 128, 256, ...): X21 = -X22 (L21 X11), every pair of a level in
 //      one batched launch

@@ -19,6 +19,14 @@ int device_info(DeviceInfo* out);  // PIQ_OK / PIQ_ERR_CUDA / PIQ_ERR_UNSUPPORTE
 // Count one kernel launch (piq_kernel_launches).
 void note_launch(int count = 1);
 
+// PIQ_OK for cudaSuccess, else PIQ_ERR_CUDA with the error recorded for
+// piq_last_cuda_error.
+int cuda_rc(cudaError_t e);
+// Copy the status word back, synchronize `stream` and return the status code
+// (PIQ_ERR_CUDA, recorded, when the copy or a kernel of the call failed).
+// host_st, when given, receives the whole status word.
+int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st);
+
 // ------------------------------------------------------ tensor-core GEMMs (tc_gemm.cu)
 // H (+)= X^T X: upper-triangle tiles of a [in, in] fp32 matrix (row-major).
 int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
@@ -83,6 +91,8 @@ int launch_tc_sgemm(int M, int N, int K, float alpha, const float* A, int64_t ld
 int launch_gemm_f32(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
                     int64_t ldb, bool trans_b, float beta, float* C, int64_t ldc, int mode,
                     DeviceStatus* st, cudaStream_t stream, const GemmBatch& bt = GemmBatch());
+// Number of launch_gemm_f32 calls that ran on the SIMT kernel (process-wide).
+uint64_t simt_gemm_fallbacks();
 
 // ------------------------------------------------------------- factor (factor.cu)
 constexpr int kFactorNB = 128;  // panel width of the blocked Cholesky / inverse

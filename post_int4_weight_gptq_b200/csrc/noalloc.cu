@@ -37,8 +37,12 @@ int scratch_for_current_device(void** out) {
   std::lock_guard<std::mutex> lock(g_addr_mu);
   if (!g_addr[dev].ready) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_factor_scratch) != cudaSuccess || p == nullptr)
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_factor_scratch);
+    if (e != cudaSuccess) {
+      note_cuda_error(e, "cudaGetSymbolAddress of the fixed factor region");
       return PIQ_ERR_CUDA;
+    }
+    if (p == nullptr) return PIQ_ERR_CUDA;
     g_addr[dev].ptr = p;
     g_addr[dev].ready = true;
   }
@@ -69,13 +73,12 @@ extern "C" int piq_upper_factor_noalloc(const float* H, int64_t in, float damp,
   float* work = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + 256);
   // the region keeps the previous call's contents: only the status word must
   // start at zero (every other byte is written before it is read)
-  if (cudaMemsetAsync(st, 0, sizeof(DeviceStatus), s) != cudaSuccess) return PIQ_ERR_CUDA;
+  rc = cuda_rc(cudaMemsetAsync(st, 0, sizeof(DeviceStatus), s));
+  if (rc != PIQ_OK) return rc;
   rc = run_upper_factor(H, in, damp, perm, U, work, st, s);
   if (rc != PIQ_OK) return rc;
   DeviceStatus hs;
-  if (cudaMemcpyAsync(&hs, st, sizeof(DeviceStatus), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return PIQ_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return PIQ_ERR_CUDA;
-  if (lambda_out) *lambda_out = hs.lambda;
-  return hs.code;
+  rc = finish_call(st, s, &hs);
+  if (rc == PIQ_OK && lambda_out) *lambda_out = hs.lambda;
+  return rc;
 }

@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "internal.h"
 
@@ -490,12 +491,19 @@ int launch_tc_sgemm(int M, int N, int K, float alpha, const float* A, int64_t ld
   return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
+static std::atomic<uint64_t> g_simt_fallbacks{0};
+
+uint64_t simt_gemm_fallbacks() { return g_simt_fallbacks.load(); }
+
 int launch_gemm_f32(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
                     int64_t ldb, bool trans_b, float beta, float* C, int64_t ldc, int mode,
                     DeviceStatus* st, cudaStream_t stream, const GemmBatch& bt) {
   const int rc = launch_tc_sgemm(M, N, K, alpha, A, lda, B, ldb, trans_b, beta, C, ldc, mode,
                                  st, stream, bt);
   if (rc != PIQ_ERR_INVALID_ARG) return rc;
+  // an operand the tensor maps cannot describe (a base or row stride that is
+  // not 16-byte aligned): counted, so callers can see which path ran
+  g_simt_fallbacks.fetch_add(1);
   return launch_simt_gemm(M, N, K, alpha, A, lda, B, ldb, trans_b, beta, C, ldc, mode, st,
                           stream, bt);
 }
