@@ -251,6 +251,27 @@ uint64_t piq_simt_gemm_fallbacks(void);
  * Host-side, per process; static storage, overwritten by the next error. */
 const char* piq_last_cuda_error(void);
 
+/* Self-test of the bounded device waits (no counterpart on the source pages:
+ * part of this library's failure detection).  Every in-kernel wait of the
+ * library gives up after a time limit (2 s in the compute calls), records
+ * PIQ_ERR_TIMEOUT in the call's status word and lets its kernel return, so a
+ * lost producer never hangs the GPU.  This call launches one block that waits,
+ * through the same code, on a barrier nothing ever completes, with the limit
+ * set to wait_ns; it returns PIQ_ERR_TIMEOUT (and the wait's site number in
+ * *where_out, host, may be NULL) and leaves the context usable.
+ *   wait_ns    1e3 .. 1e10 (else PIQ_ERR_INVALID_ARG)
+ *   workspace  device, >= 256 bytes, 256-byte aligned (the status word)
+ *   Synchronizes `stream` once.
+ *
+ * Host-side fault injection, for testing callers' error handling: with the
+ * environment variable PIQ_FAULT set to "notpd", "timeout" or "oom", every
+ * compute entry point (all but this one) returns PIQ_ERR_NOT_PD,
+ * PIQ_ERR_TIMEOUT or PIQ_ERR_CUDA (reported by piq_last_cuda_error as an
+ * injected cudaErrorMemoryAllocation) after checking its arguments and before
+ * any device work.  Read at every call; unset or any other value: no effect. */
+int piq_wait_selftest(uint64_t wait_ns, int* where_out, void* workspace, size_t ws_bytes,
+                      void* stream);
+
 /* piq_upper_factor without a caller workspace.  (The source pages have no
  * counterpart: this is a deployment variant of the damping + upper-factor step
  * above, same arguments minus the workspace, same results.)

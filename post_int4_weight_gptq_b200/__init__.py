@@ -86,6 +86,8 @@ SIGNATURES = {
     "piq_kernel_launches": (ctypes.c_uint64, []),
     "piq_simt_gemm_fallbacks": (ctypes.c_uint64, []),
     "piq_last_cuda_error": (ctypes.c_char_p, []),
+    "piq_wait_selftest": (_c_int, [ctypes.c_uint64, ctypes.POINTER(_c_int), _vp, ctypes.c_size_t,
+                                   _vp]),
     "piq_upper_factor_noalloc": (_c_int, [_vp, _c_i64, _c_float, _vp, _vp,
                                           ctypes.POINTER(ctypes.c_double), _vp]),
 }
@@ -378,6 +380,19 @@ def simt_gemm_fallbacks() -> int:
     """FP32-accurate GEMMs that ran on the SIMT kernel instead of the tensor
     cores (an operand not 16-byte aligned), in this process so far."""
     return int(load_library().piq_simt_gemm_fallbacks())
+
+
+def wait_selftest(wait_ns=1_000_000, stream=None, workspace=None):
+    """Run out one bounded device wait (a barrier nothing completes) with the
+    given limit.  Returns (status, where): PIQ_ERR_TIMEOUT is the expected
+    status.  Does not raise for it."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = _workspace(256, dev, workspace)
+    where = ctypes.c_int(0)
+    rc = lib.piq_wait_selftest(int(wait_ns), ctypes.byref(where), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    return rc, where.value
 
 
 NOALLOC_MAX_IN = 512

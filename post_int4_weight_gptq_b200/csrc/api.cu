@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -45,6 +46,18 @@ static char g_err_text[160] = "";
 void note_cuda_error(cudaError_t e, const char* where) {
   std::lock_guard<std::mutex> lock(g_err_mu);
   snprintf(g_err_text, sizeof(g_err_text), "%s in %s", cudaGetErrorName(e), where);
+}
+
+int injected_fault() {
+  const char* f = std::getenv("PIQ_FAULT");
+  if (f == nullptr || *f == 0) return PIQ_OK;
+  if (std::strcmp(f, "notpd") == 0) return PIQ_ERR_NOT_PD;
+  if (std::strcmp(f, "timeout") == 0) return PIQ_ERR_TIMEOUT;
+  if (std::strcmp(f, "oom") == 0) {
+    note_cuda_error(cudaErrorMemoryAllocation, "PIQ_FAULT=oom (injected)");
+    return PIQ_ERR_CUDA;
+  }
+  return PIQ_OK;
 }
 
 int cuda_rc(cudaError_t e) {
@@ -314,6 +327,7 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
   if (W == nullptr || X == nullptr || qweight == nullptr || scales == nullptr || n < 1 ||
       !(damp >= 0.f) || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
     return PIQ_ERR_INVALID_ARG;
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   PIQ_TRY(check_ws(workspace, ws_bytes, gptq_ws_bytes(out, in, n, act_order)));
@@ -401,6 +415,7 @@ int piq_hessian(const uint16_t* X, int64_t n, int64_t in, float* H, int accumula
                 void* stream) {
   if (X == nullptr || H == nullptr || !aligned16(X) || !aligned16(H)) return PIQ_ERR_INVALID_ARG;
   if (n < 1 || in < 8 || in % 8 != 0) return PIQ_ERR_INVALID_ARG;
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   return launch_syrk_xtx(X, n, in, H, accumulate, nullptr, static_cast<cudaStream_t>(stream));
@@ -418,6 +433,7 @@ int piq_upper_factor(const float* H, int64_t in, float damp, const int32_t* perm
                      double* lambda_out, void* workspace, size_t ws_bytes, void* stream) {
   if (H == nullptr || U == nullptr || in < 1 || !(damp >= 0.f)) return PIQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   size_t need = 0;
@@ -448,6 +464,7 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
   if (Wp == nullptr || U == nullptr || codes == nullptr || qscale == nullptr)
     return PIQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   size_t need = 0;
@@ -516,6 +533,7 @@ int awq_search_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,
   for (int a = 0; a < n_alpha; ++a)
     if (!(alpha_grid[a] == alpha_grid[a])) return PIQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   size_t need = 0;
@@ -572,6 +590,7 @@ int piq_rtn_quantize_layer(const float* W, int64_t out, int64_t in, int bits, in
       !aligned16(qweight))
     return PIQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   size_t need = 0;
@@ -601,6 +620,7 @@ int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32
       out_err == nullptr || n < 1 || !aligned16(W) || !aligned16(X) || !aligned16(qweight))
     return PIQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
   size_t need = 0;

@@ -20,6 +20,7 @@ struct DeviceStatus {
   int where;         // kernel-specific detail (e.g. failing pivot index)
   double lambda;     // damping actually added
   double aux[6];
+  uint64_t wait_ns;  // limit of every bounded wait of the call; 0 = kWaitLimitNs
 };
 
 __device__ __forceinline__ void set_status(DeviceStatus* st, int code, int where) {
@@ -78,18 +79,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase of `bar` with the given parity has completed.  Bounded:
-// after kWaitLimitNs it records PIQ_ERR_TIMEOUT (detail = `where`) and returns
-// false; callers then stop issuing work.  A status set by an earlier kernel is
+// after st->wait_ns (kWaitLimitNs when that is 0 or st is NULL) it records
+// PIQ_ERR_TIMEOUT (detail = `where`) and returns false; callers then stop
+// issuing work.  A status set by an earlier kernel is
 // checked once at kernel entry, not here, so no wait gives up while copies it
 // issued are still in flight.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DeviceStatus* st,
                                           int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint64_t lim = (st != nullptr && st->wait_ns != 0) ? st->wait_ns : kWaitLimitNs;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > lim) {
         set_status(st, PIQ_ERR_TIMEOUT, where);
         return false;
       }

@@ -19,6 +19,13 @@ int device_info(DeviceInfo* out);  // PIQ_OK / PIQ_ERR_CUDA / PIQ_ERR_UNSUPPORTE
 // Count one kernel launch (piq_kernel_launches).
 void note_launch(int count = 1);
 
+// Host-side fault injection for testing callers' error handling: with the
+// environment variable PIQ_FAULT set to notpd, timeout or oom, every compute
+// entry point returns PIQ_ERR_NOT_PD, PIQ_ERR_TIMEOUT or PIQ_ERR_CUDA (recorded
+// as cudaErrorMemoryAllocation) after checking its arguments and before any
+// device work; unset or any other value: PIQ_OK.
+int injected_fault();
+
 // PIQ_OK for cudaSuccess, else PIQ_ERR_CUDA with the error recorded for
 // piq_last_cuda_error.
 int cuda_rc(cudaError_t e);

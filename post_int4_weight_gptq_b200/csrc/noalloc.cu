@@ -62,8 +62,10 @@ extern "C" int piq_upper_factor_noalloc(const float* H, int64_t in, float damp,
   if (in > kNoAllocMaxIn) return PIQ_ERR_INVALID_ARG;  // larger than the fixed region
   if (256 + static_cast<size_t>(factor_workspace_floats(in)) * 4 > kNoAllocBytes)
     return PIQ_ERR_INVALID_ARG;
+  int rc = injected_fault();
+  if (rc != PIQ_OK) return rc;
   DeviceInfo info;
-  int rc = device_info(&info);
+  rc = device_info(&info);
   if (rc != PIQ_OK) return rc;
   void* base = nullptr;
   rc = scratch_for_current_device(&base);
