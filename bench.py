@@ -1,14 +1,22 @@
 #!/usr/bin/env python
-"""Throughput of one-layer GPTQ (INT4, g128) on a Llama-7B-shaped q_proj.
+"""Throughput of one-layer GPTQ (INT4, g128) on a Llama-70B-shaped down_proj,
+plus the AWQ alpha search and a 7B-shaped q_proj layer.
 
-One step = the whole quantization of one layer through the C ABI:
-gptq_quantize_layer (H = X^T X, damping, upper factor, blocked sweep with
-trailing GEMMs, packing, output error on the calibration X) plus the output
-error on the shifted X' (piq_layer_output_error) that the workload asks for.
-Workload: W 4096x4096 fp32 ~N(0, 0.02^2); X 131072x4096 bf16 with per-channel
-std ~LogNormal(0, 1) and 41 channels x30; X' a fresh draw with the channel stds
-reshuffled; bits 4, g 128, damp 0.01.  Inputs are synthetic and seeded
-(workloads/), X is larger than L2 so no flush is needed between steps.
+One step = the whole quantization of one layer through the C ABI
+(gptq_quantize_layer: H = X^T X, damping, the FP64-grade factor, the blocked
+sweep with its block updates, packing, output error on the calibration X).
+Default workload (the largest single-GPU one): W 8192x28672 fp32 ~N(0, 0.01^2),
+X 32768x28672 bf16 ~N(0, 1) with 143 channels x40; bits 4, g 128, damp 0.01.
+``--workload q_proj_7b`` times W 4096^2 with X 131072x4096 (lognormal channel
+stds, 41 channels x30) plus the error on the shifted X' instead.  Inputs are
+synthetic and seeded (workloads/); X is larger than L2, so no flush is needed
+between steps.
+
+The JSON line also carries, unless switched off: the AWQ 20-point alpha search
+on the 8192^2 layer (ms per layer, phases, their rooflines), the q_proj_7b
+layer as a second record, per-phase roofline fractions of the headline layer,
+and the FP64 oracle timed on the host cores (exactly on the tiny 256x512
+layer; on a bounded sample of the headline layer, every scaled term labelled).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -38,10 +46,6 @@ METRIC = "GPTQ INT4 sec/layer & Mweights/s; XᵀX TFLOPS; AWQ α-search ms/layer
 UNIT = "Mweights/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one syrk_xtx launch on the
-# 131072 x 4096 workload, from one ncu capture of the current kernel; to be retaken (or set to
-# None) whenever that kernel changes.
-SYRK_TRAFFIC_BYTES = 1.93e9 + 21.82e6
 
 
 def load_peaks():
@@ -156,6 +160,14 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ------------------------------------------------------------- workload
+WORKLOADS = ("down_proj_70b", "q_proj_7b")
+
+
+def spec_of(name):
+    from workloads import C2, C4
+    return {"down_proj_70b": C4, "q_proj_7b": C2}[name]
+
+
 def to_gpu_w(W, dev):
     import torch
     return torch.from_numpy(np.ascontiguousarray(W, dtype=np.float32)).to(dev)
@@ -167,58 +179,62 @@ def to_gpu_x(Xbits, dev):
         torch.bfloat16)
 
 
-def make_inputs(rank: int, n=None):
-    from workloads import C2, make_weight, make_x_bits
-    seed = C2.seed + rank               # each rank quantizes its own layer
-    W = make_weight(C2, seed=seed)
-    X = make_x_bits(C2, n=n, seed=seed)
-    X2 = make_x_bits(C2, n=n, seed=seed + 1, permute_seed=seed + 1)
+def make_inputs(rank: int, n=None, workload="down_proj_70b"):
+    """(W, X, X') of one rank's layer; X' (the shifted inputs) only for q_proj_7b."""
+    from workloads import make_weight, make_x_bits
+    spec = spec_of(workload)
+    seed = spec.seed + rank               # each rank quantizes its own layer
+    W = make_weight(spec, seed=seed)
+    X = make_x_bits(spec, n=n, seed=seed)
+    X2 = None
+    if workload == "q_proj_7b":
+        X2 = make_x_bits(spec, n=n, seed=seed + 1, permute_seed=seed + 1)
     return W, X, X2
 
 
-def workload_config(spec, n):
-    return {"workload": f"q_proj_7b GPTQ: W {spec.out}x{spec.inp} fp32, X {n}x{spec.inp} bf16 "
-                        f"(+ error on shifted X'), bits {spec.bits}, g {spec.g}, damp {spec.damp}",
+def workload_config(spec, n, workload="down_proj_70b"):
+    shifted = " (+ error on shifted X')" if workload == "q_proj_7b" else ""
+    gb = n * spec.inp * 2 / 1e9
+    return {"workload": f"{workload} GPTQ: W {spec.out}x{spec.inp} fp32, X {n}x{spec.inp} bf16"
+                        f"{shifted}, bits {spec.bits}, g {spec.g}, damp {spec.damp}",
             "out": spec.out, "in": spec.inp, "samples": n, "bits": spec.bits, "g": spec.g,
-            "l2_flush": "not needed: inputs larger than L2 (X 1.07 GB per step)"}
+            "l2_flush": f"not needed: inputs larger than L2 (X {gb:.2f} GB per step)"}
+
+
+# ------------------------------------------------------------ roofline arithmetic
+# Digits per operand of the FP64-grade products (library constants: factor 6,
+# block updates 5) and the nominal INT8 : BF16 dense tensor ratio.
+FACTOR_PAIRS = 6 * 7 // 2
+SWEEP_PAIRS = 5 * 6 // 2
+INT8_PER_BF16 = 2.0
+
+
+def phase_rooflines(ph, out, inp, n, bf16_peak, hbm_peak):
+    """Per-phase achieved rate and fraction of its roofline, from the phase
+    times (ms) of one gptq_quantize_layer call.  Algorithmic work:
+    hessian n in (in+1) bf16 flop (upper triangle); factor in^3 / 3 FP64 flop
+    (Cholesky of the damped H), bound by the INT8 tensor rate over the 21 digit
+    products of each FP64-grade product; sweep out in^2 FP64 flop of block
+    updates (15 digit products); pack out in (1 + 4 + 4 + 1/2) bytes (codes and
+    W read, D written, nibbles written); error 3 out in (in + 256) bf16 flop."""
+    res = {}
+    int8_peak = INT8_PER_BF16 * bf16_peak
+
+    def put(k, work, unit, peak, scale):
+        ms = ph.get(k)
+        if ms:
+            a = work / (ms / 1e3) / scale
+            res[k] = {"ms": ms, "achieved": a, "unit": unit, "peak": peak, "frac": a / peak}
+
+    put("hessian", float(n) * inp * (inp + 1), "TFLOP/s", bf16_peak, 1e12)
+    put("factor", inp ** 3 / 3.0, "TFLOP/s (FP64-grade)", int8_peak / FACTOR_PAIRS, 1e12)
+    put("sweep", float(out) * inp * inp, "TFLOP/s (FP64-grade)", int8_peak / SWEEP_PAIRS, 1e12)
+    put("pack", out * inp * 9.5, "GB/s", hbm_peak, 1e9)
+    put("error", 3.0 * out * inp * (inp + 256), "TFLOP/s", bf16_peak, 1e12)
+    return res
 
 
 # ---------------------------------------------------------- oracle baseline
-def oracle_sample(W, X, X2, n_full, n_rows=4096, w_rows=256):
-    """Oracle on a bounded sample, scaled to one full layer of n_full samples.
-    Returns (seconds per full layer, description)."""
-    import oracle as O
-    from workloads import C2
-    n, inp = n_full, X.shape[1]
-    out = W.shape[0]
-    t0 = time.perf_counter()
-    H = O.hessian_ref(X[:n_rows])
-    t_h = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    perm, U, lam = O.gptq_prepare_ref(H, C2.damp, False)
-    t_f = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    from oracle.gptq import gptq_sweep_blocked_ref
-    codes, scales, _ = gptq_sweep_blocked_ref(W[:w_rows].astype(np.float64)[:, perm], U, C2.bits,
-                                              C2.g)
-    t_s = time.perf_counter() - t0
-    from oracle.pack import dequant_ref
-    What = dequant_ref(codes, scales, perm, C2.g)
-    t0 = time.perf_counter()
-    O.output_error_ref(W[:w_rows], What, X[:n_rows])
-    t_e1 = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    O.output_error_ref(W[:w_rows], What, X2[:n_rows])
-    t_e2 = time.perf_counter() - t0
-    # H and error scale with samples; sweep and error with rows; factor is whole
-    total = (t_h * n / n_rows + t_f + t_s * out / w_rows
-             + (t_e1 + t_e2) * (n / n_rows) * (out / w_rows))
-    desc = (f"H on {n_rows}/{n} samples (x{n // n_rows}); factor of the full {inp}x{inp} H; "
-            f"sweep on {w_rows}/{out} rows (x{out // w_rows}); errors on {n_rows} samples x "
-            f"{w_rows} rows (x{(n // n_rows) * (out // w_rows)}); float64 NumPy/OpenBLAS")
-    return total, desc
-
-
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -226,23 +242,81 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def oracle_sample(W, X, X2, n_full, n_rows=1024, w_rows=64, sub_in=4096):
+    """The FP64 oracle on a bounded sample of one layer, scaled to the full
+    layer.  Returns (seconds per full layer, description).  Every scaled term
+    is named in the description:
+      H on n_rows of n_full samples, scaled by samples;
+      factor (damping, inv, cholesky) of the leading sub_in x sub_in block of
+        that H, scaled by (in / sub_in)^3 when in > sub_in;
+      blocked sweep of w_rows rows over the leading sub_in columns, scaled by
+        rows and by (in / sub_in)^2;
+      output errors on n_rows samples x w_rows rows, scaled by samples x rows."""
+    import oracle as O
+    from oracle.gptq import gptq_sweep_blocked_ref
+    from oracle.pack import dequant_ref
+    n, inp = n_full, X.shape[1]
+    out = W.shape[0]
+    si = min(sub_in, inp)
+    t0 = time.perf_counter()
+    H = O.hessian_ref(X[:n_rows])
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    perm, U, lam = O.gptq_prepare_ref(H[:si, :si], 0.01, False)
+    t_f = time.perf_counter() - t0
+    Ws = W[:w_rows, :si].astype(np.float64)
+    t0 = time.perf_counter()
+    codes, scales, _ = gptq_sweep_blocked_ref(Ws[:, perm], U, 4, 128)
+    t_s = time.perf_counter() - t0
+    What = dequant_ref(codes, scales, perm, 128)
+    t0 = time.perf_counter()
+    O.output_error_ref(W[:w_rows, :si], What, X[:n_rows, :si])
+    t_e = (time.perf_counter() - t0) * (inp / si)
+    n_err = 2 if X2 is not None else 1
+    fs = (inp / si) ** 3
+    total = (t_h * n / n_rows + t_f * fs + t_s * (out / w_rows) * (inp / si) ** 2
+             + n_err * t_e * (n / n_rows) * (out / w_rows))
+    desc = (f"measured: H on {n_rows}/{n} samples (scaled x{n / n_rows:g}); factor of the "
+            f"{si}x{si} leading block (scaled x{fs:g}); blocked sweep of {w_rows}/{out} rows "
+            f"over {si}/{inp} columns (scaled x{(out / w_rows) * (inp / si) ** 2:g}); "
+            f"{n_err} output error(s) on {n_rows} samples x {w_rows} rows x {si} columns "
+            f"(scaled x{(n / n_rows) * (out / w_rows) * (inp / si):g}); "
+            f"float64 NumPy/OpenBLAS")
+    return total, desc
+
+
+def oracle_tiny_exact():
+    """The oracle's literal loop on the whole tiny layer (W 256x512, X 2048x512,
+    4-bit g128): seconds, measured, nothing scaled."""
+    import oracle as O
+    from workloads import C1, make_weight, make_x_bits
+    W, X = make_weight(C1), make_x_bits(C1)
+    t0 = time.perf_counter()
+    r = O.gptq_ref(W, X, bits=4, g=128, log=False)
+    from oracle.pack import dequant_ref
+    O.output_error_ref(W, dequant_ref(r.codes, r.scales, r.perm, 128), X)
+    return time.perf_counter() - t0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from workloads import C2
-    n_sample = 4096
-    W, X, X2 = make_inputs(0, n=n_sample)
+    spec = spec_of(args.workload)
+    n_sample = 1024
+    W, X, X2 = make_inputs(0, n=n_sample, workload=args.workload)
+    # each step a bounded sample: about five seconds of host float64 work
+    kw = dict(n_rows=n_sample, w_rows=32, sub_in=2048)
     for _ in range(args.warmup):
-        oracle_sample(W, X, X2, C2.n, n_rows=n_sample)
+        oracle_sample(W, X, X2, spec.n, **kw)
     secs = []
     desc = ""
     for _ in range(args.steps):
-        s, desc = oracle_sample(W, X, X2, C2.n, n_rows=n_sample)
+        s, desc = oracle_sample(W, X, X2, spec.n, **kw)
         secs.append(s)
     layer_s = statistics.median(secs)
-    value = C2.out * C2.inp / layer_s / 1e6
-    cfg = workload_config(C2, C2.n)
+    value = spec.out * spec.inp / layer_s / 1e6
+    cfg = workload_config(spec, spec.n, args.workload)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": layer_s * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -256,53 +330,40 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ ours
-def run_ours(args):
-    import torch
-    import post_int4_weight_gptq_b200 as piq
-    from workloads import C2
-
-    rank, world, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    peaks, peak_src = load_peaks()
-
-    W, X, X2 = make_inputs(rank, n=args.samples)
-    out_rows, inp = W.shape
-    n = X.shape[0]
-    Wg, Xg, X2g = to_gpu_w(W, dev), to_gpu_x(X, dev), to_gpu_x(X2, dev)
-    ws = torch.empty(piq.gptq_workspace_bytes(out_rows, inp, n), dtype=torch.uint8, device=dev)
-    ws_err = torch.empty(piq.output_error_workspace_bytes(out_rows, inp, n), dtype=torch.uint8,
-                         device=dev)
-    res = piq.GPTQOutput(torch.empty(out_rows, inp // 8, dtype=torch.int32, device=dev),
-                         torch.empty(out_rows, inp // C2.g, dtype=torch.float16, device=dev),
-                         torch.empty(inp, dtype=torch.int32, device=dev),
-                         torch.empty(inp, dtype=torch.int32, device=dev), None)
+def time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps, warmup, world, local,
+               sample_clocks=True):
+    """Device-timed steps of one layer (inputs resident in HBM): (ms per step,
+    mean phase times, launches per step, clocks, last output, last shifted error)."""
     stream = torch.cuda.current_stream()
 
-    def step(Wd, Xd, X2d):
-        o = piq.gptq_quantize_layer(Wd, Xd, bits=C2.bits, g=C2.g, damp=C2.damp, workspace=ws,
-                                    out=res)
-        e2 = piq.layer_output_error(Wd, o.qweight, o.scales, X2d, C2.bits, C2.g, g_idx=o.g_idx,
-                                    workspace=ws_err)
+    def step():
+        o = piq.gptq_quantize_layer(Wg, Xg, bits=spec.bits, g=spec.g, damp=spec.damp,
+                                    workspace=ws, out=res)
+        e2 = None
+        if X2g is not None:
+            e2 = piq.layer_output_error(Wg, o.qweight, o.scales, X2g, spec.bits, spec.g,
+                                        g_idx=o.g_idx, workspace=ws_err)
         return o, e2
 
-    for _ in range(args.warmup):
-        step(Wg, Xg, X2g)
+    for _ in range(warmup):
+        step()
     torch.cuda.synchronize()
-
-    # ---- device-timed region (inputs resident in HBM)
-    sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
-    sampler.start()
-    time.sleep(0.3)
+    sampler = None
+    if sample_clocks:
+        sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
+        sampler.start()
+        time.sleep(0.3)
     piq.set_timing(True)
     phases = {}
     l0 = piq.kernel_launches()
+    f0 = piq.simt_gemm_fallbacks()
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
     ev0.record(stream)
-    for _ in range(args.steps):
-        o, e2 = step(Wg, Xg, X2g)
+    for _ in range(steps):
+        o, e2 = step()
         for k, v in piq.last_phase_times().items():
             phases.setdefault(k, []).append(v)
     ev1.record(stream)
@@ -310,25 +371,67 @@ def run_ours(args):
     barrier(world)
     t_wall1 = time.time()
     launches = piq.kernel_launches() - l0
+    fallbacks = piq.simt_gemm_fallbacks() - f0
     piq.set_timing(False)
     ms = ev0.elapsed_time(ev1)
-    time.sleep(0.2)
-    sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
+    clocks = None
+    if sampler is not None:
+        time.sleep(0.2)
+        sampler.stop()
+        clocks = sampler.summary(t_wall0, t_wall1)
     ms = max_over_ranks(ms, world)
-    ms_step = ms / args.steps
+    ph = {k: statistics.mean(v) for k, v in phases.items()}
+    return ms / steps, ph, launches, fallbacks, clocks, o, e2
+
+
+def alloc_layer(piq, torch, spec, n, dev, with_shift):
+    out_rows, inp = spec.out, spec.inp
+    ws = torch.empty(piq.gptq_workspace_bytes(out_rows, inp, n, g=spec.g), dtype=torch.uint8,
+                     device=dev)
+    ws_err = None
+    if with_shift:
+        ws_err = torch.empty(piq.output_error_workspace_bytes(out_rows, inp, n),
+                             dtype=torch.uint8, device=dev)
+    res = piq.GPTQOutput(torch.empty(out_rows, inp // 8, dtype=torch.int32, device=dev),
+                         torch.empty(out_rows, -(-inp // spec.g), dtype=torch.float16,
+                                     device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev),
+                         torch.empty(inp, dtype=torch.int32, device=dev), None)
+    return ws, ws_err, res
+
+
+def run_ours(args):
+    import torch
+    import post_int4_weight_gptq_b200 as piq
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    spec = spec_of(args.workload)
+
+    W, X, X2 = make_inputs(rank, n=args.samples, workload=args.workload)
+    out_rows, inp = W.shape
+    n = X.shape[0]
+    Wg, Xg = to_gpu_w(W, dev), to_gpu_x(X, dev)
+    X2g = to_gpu_x(X2, dev) if X2 is not None else None
+    ws, ws_err, res = alloc_layer(piq, torch, spec, n, dev, X2 is not None)
+
+    ms_step, ph, launches, fallbacks, clocks, o, e2 = time_layer(
+        piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, args.steps, args.warmup, world, local)
     value = world * out_rows * inp / (ms_step / 1e3) / 1e6
 
     # ---- end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
+        stream = torch.cuda.current_stream()
         Wh = torch.from_numpy(W).pin_memory()
         Xh = torch.from_numpy(X.view(np.int16)).pin_memory()
-        X2h = torch.from_numpy(X2.view(np.int16)).pin_memory()
-        Wd, Xd, X2d = torch.empty_like(Wg), torch.empty_like(Xg), torch.empty_like(X2g)
+        X2h = torch.from_numpy(X2.view(np.int16)).pin_memory() if X2 is not None else None
+        Wd, Xd = torch.empty_like(Wg), torch.empty_like(Xg)
+        X2d = torch.empty_like(X2g) if X2g is not None else None
         host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in res[:4]]
-        h2d = Wh.numel() * 4 + Xh.numel() * 2 + X2h.numel() * 2
-        d2h = sum(t.numel() * t.element_size() for t in host_out) + 16
+        h2d = Wh.numel() * 4 + Xh.numel() * 2 + (X2h.numel() * 2 if X2h is not None else 0)
+        d2h = sum(t.numel() * t.element_size() for t in host_out) + 8 * (2 if X2 is not None else 1)
         k_e2e = max(1, min(args.steps, 5))
         barrier(world)
         torch.cuda.synchronize()
@@ -337,10 +440,15 @@ def run_ours(args):
         for _ in range(k_e2e):
             Wd.copy_(Wh, non_blocking=True)
             Xd.copy_(Xh.view(torch.bfloat16), non_blocking=True)
-            X2d.copy_(X2h.view(torch.bfloat16), non_blocking=True)
-            o, e2 = step(Wd, Xd, X2d)
-            for h, d in zip(host_out, o[:4]):
-                h.copy_(d, non_blocking=True)
+            if X2d is not None:
+                X2d.copy_(X2h.view(torch.bfloat16), non_blocking=True)
+            oo = piq.gptq_quantize_layer(Wd, Xd, bits=spec.bits, g=spec.g, damp=spec.damp,
+                                         workspace=ws, out=res)
+            if X2d is not None:
+                piq.layer_output_error(Wd, oo.qweight, oo.scales, X2d, spec.bits, spec.g,
+                                       g_idx=oo.g_idx, workspace=ws_err)
+            for hbuf, d in zip(host_out, oo[:4]):
+                hbuf.copy_(d, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -348,54 +456,110 @@ def run_ours(args):
         e2e = {"value": world * out_rows * inp / (ms_e2e / 1e3) / 1e6, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ms_e2e, "steps": k_e2e}
+        del Wd, Xd, X2d, Wh, Xh, X2h
 
-    # ---- roofline of the dominant kernel, the X^T X build (per-phase CUDA
-    # events on the launching stream, averaged over the timed steps).  The
-    # denominator is the measured burst bf16 peak unless the clock samples of
-    # the timed region show the power cap, then the sustained one.
-    ph = {k: statistics.mean(v) for k, v in phases.items()}
-    t_h = ph.get("hessian", float("nan"))
-    flops_h = float(n) * inp * (inp + 1)
+    # ---- rooflines: burst peaks unless the timed region's clocks show the power cap
     capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
     peak_key = "bf16_tflops_sustained" if capped else "bf16_tflops"
-    peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
-    ach_h = flops_h / (t_h / 1e3) / 1e12
-    roof = {"kernel": "syrk_xtx (tcgen05 H = X^T X, 1024-sample chunks summed in registers)",
-            "bound": "tensor", "achieved": ach_h, "peak": peak, "unit": "TFLOP/s",
-            "frac": ach_h / peak,
-            "traffic": args.traffic if args.traffic is not None else (
-                SYRK_TRAFFIC_BYTES if args.samples is None else None),
-            "flops_per_launch": flops_h,
-            "flops_formula": "n*in*(in+1) (upper triangle)", "ms_per_launch": t_h,
-            "peak_source": f"{peak_src} {peak_key}"}
+    bf16_peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    phase_roof = phase_rooflines(ph, out_rows, inp, n, bf16_peak, hbm_peak)
+    dom = max(phase_roof, key=lambda k: phase_roof[k]["ms"])
+    d = phase_roof[dom]
+    roof = {"kernel": {"hessian": "syrk64 (tcgen05 bf16 H = X^T X, FP64 chunk sums)",
+                       "factor": "FP64-grade Cholesky (chol64 diagonal blocks + ozaki_gemm "
+                                 "INT8 tensor-core panel products)",
+                       "sweep": "FP64 sweep (sweep64) + ozaki_gemm block updates",
+                       "pack": "pack", "error": "err_dot (bf16x3 through H)"}[dom],
+            "phase": dom, "bound": "hbm" if d["unit"] == "GB/s" else "tensor",
+            "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+            "traffic": args.traffic, "ms_per_launch": d["ms"],
+            "peak_source": f"{peak_src} {peak_key}" + (
+                "; FP64-grade products: nominal INT8 = 2 x bf16, over the digit products"
+                if "FP64" in d["unit"] else "")}
+    ph_h = ph.get("hessian", float("nan"))
+    xtx = float(n) * inp * (inp + 1) / (ph_h / 1e3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, desc = oracle_sample(W, X, X2, n)
         cpu = {"value": out_rows * inp / secs / 1e6, "unit": UNIT, "cores": cpu_cores(),
                "kind": "oracle", "sample": desc}
+        t_tiny = oracle_tiny_exact()
+        cpu["tiny_exact"] = {"workload": "tiny 256x512, X 2048x512, 4-bit g128 (whole layer, "
+                                         "literal loop, nothing scaled)",
+                             "seconds": t_tiny, "mweights_per_s": 256 * 512 / t_tiny / 1e6}
+    del Wg, Xg, X2g, ws, ws_err
+    torch.cuda.empty_cache()
 
     awq = None
-    if args.awq and rank == 0:
-        awq = run_awq(dev)
-    variants = None
-    if args.variants and rank == 0:
-        variants = run_variants(dev, Wg, Xg)
+    if not args.no_awq and rank == 0:
+        awq = run_awq(dev, peaks)
+    second = None
+    if not args.no_second and rank == 0 and args.samples is None:
+        other = "q_proj_7b" if args.workload == "down_proj_70b" else "down_proj_70b"
+        second = run_second(piq, torch, dev, other)
+    tiny = None
+    if rank == 0 and cpu is not None:
+        tiny = run_tiny(piq, torch, dev)
+        tiny["oracle_seconds"] = cpu["tiny_exact"]["seconds"]
+        tiny["speedup_vs_oracle"] = tiny["oracle_seconds"] / (tiny["ms_per_layer"] / 1e3)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "sec_per_layer": ms_step / 1e3, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16/f32", "data": "synthetic",
-                "config": workload_config(C2, n), "xtx_tflops": ach_h,
-                "phases_ms": ph, "roofline": roof,
+                "vs_baseline": None, "dtype": "bf16 in, f64-grade factor/sweep", "data": "synthetic",
+                "config": workload_config(spec, n, args.workload), "xtx_tflops": xtx,
+                "awq_ms_per_layer": awq["ms_per_layer"] if awq else None,
+                "phases_ms": ph, "phase_roofline": phase_roof, "roofline": roof,
                 "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
-                "awq": awq, "variants": variants, "shift_error": e2, "calib_error": o.err}
+                "simt_gemm_fallbacks": fallbacks, "awq": awq, "second_workload": second,
+                "tiny_exact": tiny, "calib_error": o.err}
+        if e2 is not None:
+            line["shift_error"] = e2
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def run_second(piq, torch, dev, workload, steps=10, warmup=3):
+    """A second GPTQ layer, device-timed like the headline one."""
+    spec = spec_of(workload)
+    W, X, X2 = make_inputs(0, workload=workload)
+    Wg, Xg = to_gpu_w(W, dev), to_gpu_x(X, dev)
+    X2g = to_gpu_x(X2, dev) if X2 is not None else None
+    ws, ws_err, res = alloc_layer(piq, torch, spec, X.shape[0], dev, X2 is not None)
+    ms, ph, _, _, _, o, e2 = time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps,
+                                        warmup, 1, 0, sample_clocks=False)
+    r = {"workload": workload_config(spec, X.shape[0], workload)["workload"],
+         "ms_per_layer": ms, "mweights_per_s": spec.out * spec.inp / (ms / 1e3) / 1e6,
+         "xtx_tflops": float(X.shape[0]) * spec.inp * (spec.inp + 1) / (ph["hessian"] / 1e3) / 1e12,
+         "phases_ms": ph, "calib_error": o.err}
+    if e2 is not None:
+        r["shift_error"] = e2
+    del Wg, Xg, X2g, ws, ws_err
+    torch.cuda.empty_cache()
+    return r
+
+
+def run_tiny(piq, torch, dev, steps=20, warmup=3):
+    """The tiny layer on the GPU (device-timed), beside the oracle's exact time."""
+    from workloads import C1, make_weight, make_x_bits
+    Wg, Xg = to_gpu_w(make_weight(C1), dev), to_gpu_x(make_x_bits(C1), dev)
+    for _ in range(warmup):
+        piq.gptq_quantize_layer(Wg, Xg, bits=4, g=128)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        piq.gptq_quantize_layer(Wg, Xg, bits=4, g=128)
+    e1.record()
+    torch.cuda.synchronize()
+    return {"workload": "tiny 256x512, X 2048x512, 4-bit g128",
+            "ms_per_layer": e0.elapsed_time(e1) / steps}
 
 
 def hbm_phase_rates(phases_ms, n, inp, out, n_alpha, hbm_peak_gbs):
@@ -414,7 +578,7 @@ def hbm_phase_rates(phases_ms, n, inp, out, n_alpha, hbm_peak_gbs):
     return res
 
 
-def run_awq(dev, steps=3, warmup=1):
+def run_awq(dev, peaks, steps=5, warmup=3):
     """AWQ alpha search (20-point grid) on the 8192x8192 layer: ms per layer."""
     import torch
     import post_int4_weight_gptq_b200 as piq
@@ -425,6 +589,7 @@ def run_awq(dev, steps=3, warmup=1):
                      dtype=torch.uint8, device=dev)
     for _ in range(warmup):
         piq.awq_search_layer(Wg, Xg, C5.bits, C5.g, AWQ_GRID, workspace=ws)
+    torch.cuda.synchronize()
     piq.set_timing(True)
     times, ph = [], {}
     for _ in range(steps):
@@ -439,55 +604,15 @@ def run_awq(dev, steps=3, warmup=1):
     piq.set_timing(False)
     ph = {k: statistics.mean(v) for k, v in ph.items()}
     flops = 2.0 * C5.n * C5.inp * C5.out * len(AWQ_GRID)
-    peaks, src = load_peaks()
-    return {"workload": "AWQ 20-point alpha search: W 8192x8192, X 16384x8192",
+    bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tf = flops / (ph["error_gemm"] / 1e3) / 1e12
+    del Wg, Xg, ws
+    torch.cuda.empty_cache()
+    return {"workload": "AWQ 20-point alpha search: W 8192x8192, X 16384x8192, 4-bit g128",
             "ms_per_layer": statistics.median(times), "best_alpha": r.best_alpha,
-            "phases_ms": ph, "error_gemm_tflops": flops / (ph["error_gemm"] / 1e3) / 1e12,
-            "hbm": hbm_phase_rates(ph, C5.n, C5.inp, C5.out, len(AWQ_GRID), peaks["hbm_gbs"]),
-            "hbm_peak_source": f"{src} hbm_gbs"}
-
-
-def run_variants(dev, Wg, Xg, steps=5, warmup=3):
-    """The q_proj layer through plain GPTQ, AWQ-scaled GPTQ (s from AWQ's
-    20-point search, run once untimed) and GPTQ with asymmetric groups, timed
-    interleaved step by step so that all three see the same clocks: ms per layer
-    (median) and each one's output error."""
-    import torch
-    import post_int4_weight_gptq_b200 as piq
-    from workloads import AWQ_GRID, C2
-    out_rows, inp = Wg.shape
-    n = Xg.shape[0]
-    a = piq.awq_search_layer(Wg, Xg, C2.bits, C2.g, AWQ_GRID)
-    ws = torch.empty(piq.gptq_workspace_bytes(out_rows, inp, n), dtype=torch.uint8, device=dev)
-    calls = {
-        "gptq": lambda: piq.gptq_quantize_layer(Wg, Xg, C2.bits, C2.g, C2.damp, workspace=ws),
-        "awq_then_gptq": lambda: piq.awq_gptq_quantize_layer(Wg, Xg, a.s, C2.bits, C2.g,
-                                                             C2.damp, workspace=ws),
-        "gptq_asym": lambda: piq.gptq_quantize_layer(Wg, Xg, C2.bits, C2.g, C2.damp,
-                                                     workspace=ws, sym=False),
-    }
-    for _ in range(warmup):
-        for f in calls.values():
-            f()
-    times = {k: [] for k in calls}
-    errs = {}
-    for _ in range(steps):
-        for k, f in calls.items():
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            r = f()
-            e1.record()
-            torch.cuda.synchronize()
-            times[k].append(e0.elapsed_time(e1))
-            errs[k] = r.err
-    res = {"workload": "q_proj 4096x4096, X 131072x4096, 4-bit g128: three GPTQ variants "
-                       "timed interleaved", "awq_alpha": a.best_alpha,
-           "awq_error": a.err_per_alpha[int(np.argmin([abs(x - a.best_alpha) for x in AWQ_GRID]))]}
-    for k in calls:
-        ms = statistics.median(times[k])
-        res[k] = {"ms_per_layer": ms, "mweights_per_s": out_rows * inp / (ms / 1e3) / 1e6,
-                  "error": errs[k]}
-    return res
+            "phases_ms": ph, "error_gemm_tflops": tf, "error_gemm_frac": tf / bf16,
+            "hbm": hbm_phase_rates(ph, C5.n, C5.inp, C5.out, len(AWQ_GRID),
+                                   peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))}
 
 
 def main(argv=None):
@@ -496,18 +621,17 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=WORKLOADS, default="down_proj_70b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--awq", action="store_true", help="also time the AWQ search (8192^2 layer)")
-    ap.add_argument("--variants", action="store_true",
-                    help="also time plain, AWQ-scaled and asymmetric-group GPTQ on the same "
-                         "layer, interleaved")
+    ap.add_argument("--no-awq", action="store_true", help="skip the AWQ search record")
+    ap.add_argument("--no-second", action="store_true", help="skip the second GPTQ layer record")
     ap.add_argument("--samples", type=int, default=None,
-                    help="calibration rows per layer (default: the workload's 131072); a smaller "
+                    help="calibration rows per layer (default: the workload's); a smaller "
                          "value is for profiler captures, not for reported numbers")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per syrk_xtx launch from an ncu capture of the current "
-                         "kernel (overrides the recorded figure)")
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture of "
+                         "the current kernel (reported as the roofline's traffic)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -127,10 +127,19 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
  *            What = code * fp16(scale) (the layer a user reconstructs),
  *            evaluated as sum_r D_r H D_r^T (D = W - What in fp32) from the H
  *            of the first step: the same quantity, without a second pass over X.
- * Runs every step on the GPU: H (tensor cores), act-order, damping, blocked
- * Cholesky and triangular inverse, per-block sweep + trailing GEMM, packing,
- * output error.  Synchronizes `stream` once at the end. */
-int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int act_order, size_t* bytes);
+ * Runs every step on the GPU: H (tensor cores), act-order, damping, the
+ * blocked Cholesky factor R of the damped H (H_d = R R^T, so U = inv(R); FP64,
+ * its products on the INT8 tensor cores with FP64 accumulation), the per-block
+ * sweep in FP64 with the block updates on the same tensor-core path, packing,
+ * output error.  The sweep uses the exact identity W0 - Q = U^T err (W0 the
+ * weights before any update, Q = code * scale): it carries
+ * acc = (W0 - Q) R to later columns and reads the current weights of a block
+ * G as W0_G + acc_G inv(R_GG), the listing's arithmetic without forming U.
+ * Synchronizes `stream` once at the end.
+ * Workspace: piq_gptq_workspace_bytes with the same out, in, n, g and
+ * act_order (the column blocks of the sweep depend on g). */
+int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int g, int act_order,
+                             size_t* bytes);
 int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
                         int bits, int g, float damp, int act_order, uint32_t* qweight,
                         uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,

@@ -238,24 +238,30 @@ def block_partition_ref(inp: int, g: int, block: int = 128):
     return blocks
 
 
-def _sweep_blocked(Wp, U, bits, g, block, sym):
+def _sweep_blocked(Wp, U, bits, g, block, sym, force=None, force_zero=None):
     W = np.array(Wp, dtype=np.float64, copy=True)
     out, inp = W.shape
     codes = np.zeros((out, inp), dtype=np.int16)
     scales = np.zeros((out, -(-inp // g)), dtype=np.float64)
     zeros = np.zeros((out, -(-inp // g)), dtype=np.int16)
+    zvlog = np.zeros((out, -(-inp // g)))
     vlog = np.zeros((out, inp))
     scale = cmin = cmax = None
     for b, e in block_partition_ref(inp, g, block):
         Err = np.zeros((out, e - b))
         for j in range(b, e):
             if j % g == 0:
-                scale, zero, _, cmin, cmax = group_quantizer_ref(W[:, j:j + g], bits, sym)
+                fz = None if force_zero is None else force_zero[:, j // g]
+                scale, zero, zv, cmin, cmax = group_quantizer_ref(W[:, j:j + g], bits, sym,
+                                                                  force_zero=fz)
                 scales[:, j // g] = scale
                 zeros[:, j // g] = zero.astype(np.int16)
+                zvlog[:, j // g] = zv
             live = scale > 0
             v = np.where(live, W[:, j] / np.where(live, scale, 1.0), 0.0)
             c = np.clip(np.round(v), cmin, cmax)
+            if force is not None:
+                c = np.where(force[:, j] != NO_FORCE, force[:, j], c)
             err = (W[:, j] - c * scale) / U[j, j]
             W[:, j + 1:e] -= np.outer(err, U[j, j + 1:e])
             Err[:, j - b] = err
@@ -263,22 +269,24 @@ def _sweep_blocked(Wp, U, bits, g, block, sym):
             vlog[:, j] = v
         if e < inp:
             W[:, e:] -= Err @ U[b:e, e:]
-    return codes, scales, zeros, vlog
+    return codes, scales, zeros, vlog, zvlog
 
 
 def gptq_sweep_blocked_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
-                           block: int = 128):
+                           block: int = 128, force: np.ndarray | None = None):
     """The same loop with updates deferred per column block: inside a block the
     error goes to the block's later columns; after the block one product
-    Err[:, b:e] @ U[b:e, e:] updates every column past it.  (codes, scales, v)."""
-    codes, scales, _, vlog = _sweep_blocked(Wp, U, bits, g, block, True)
+    Err[:, b:e] @ U[b:e, e:] updates every column past it.  (codes, scales, v).
+    ``force`` is the teacher-forcing hook of ``gptq_sweep_ref``."""
+    codes, scales, _, vlog, _ = _sweep_blocked(Wp, U, bits, g, block, True, force)
     return codes, scales, vlog
 
 
 def gptq_sweep_blocked_asym_ref(Wp: np.ndarray, U: np.ndarray, bits: int = 4, g: int = 128,
-                                block: int = 128):
-    """Blocked sweep with asymmetric groups: (codes, scales, zeros, v)."""
-    return _sweep_blocked(Wp, U, bits, g, block, False)
+                                block: int = 128, force: np.ndarray | None = None,
+                                force_zero: np.ndarray | None = None):
+    """Blocked sweep with asymmetric groups: (codes, scales, zeros, v, zv)."""
+    return _sweep_blocked(Wp, U, bits, g, block, False, force, force_zero)
 
 
 def gptq_ref_blocked(W, X=None, *, H=None, bits: int = 4, g: int = 128, damp: float = 0.01,
@@ -288,7 +296,7 @@ def gptq_ref_blocked(W, X=None, *, H=None, bits: int = 4, g: int = 128, damp: fl
         H = hessian_ref(X)
     perm, U, lam = gptq_prepare_ref(H, damp, act_order)
     Wp = np.asarray(W, dtype=np.float64)[:, perm]
-    codes, scales, zeros, v = _sweep_blocked(Wp, U, bits, g, block, sym)
+    codes, scales, zeros, v, _ = _sweep_blocked(Wp, U, bits, g, block, sym)
     return GPTQResult(codes, scales, perm, g_idx_from_perm(perm, g), v, None, U, lam, bits, g,
                       None if sym else zeros)
 

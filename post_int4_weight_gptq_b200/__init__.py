@@ -54,7 +54,7 @@ SIGNATURES = {
     "piq_gptq_sweep_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_size_p]),
     "piq_gptq_sweep": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_int, _c_int, _vp, _vp, _vp,
                                 ctypes.c_size_t, _vp]),
-    "piq_gptq_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_size_p]),
+    "piq_gptq_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_int, _c_size_p]),
     "gptq_quantize_layer": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int, _c_float,
                                      _c_int, _vp, _vp, _vp, _vp,
                                      ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
@@ -215,8 +215,9 @@ GPTQOutput = collections.namedtuple("GPTQOutput", "qweight scales perm g_idx err
 AWQOutput = collections.namedtuple("AWQOutput", "best_alpha s qweight scales err_per_alpha")
 
 
-def gptq_workspace_bytes(out, inp, n, act_order=False) -> int:
-    return _query(load_library().piq_gptq_workspace_bytes, out, inp, n, int(bool(act_order)))
+def gptq_workspace_bytes(out, inp, n, act_order=False, g=128) -> int:
+    return _query(load_library().piq_gptq_workspace_bytes, out, inp, n, int(g),
+                  int(bool(act_order)))
 
 
 def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_error=True,
@@ -239,7 +240,7 @@ def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_er
                          torch.empty(inp, dtype=torch.int32, device=dev),
                          torch.empty(inp, dtype=torch.int32, device=dev), None,
                          None if sym else torch.empty(rows, ng, dtype=torch.uint8, device=dev))
-    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order), dev, workspace)
+    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order, g), dev, workspace)
     err = ctypes.c_double(0.0)
     eptr = ctypes.byref(err) if with_error else None
     if sym:
@@ -304,7 +305,7 @@ def awq_gptq_quantize_layer(W, X, s, bits=4, g=128, damp=0.01, act_order=False,
                          torch.empty(rows, -(-inp // g), dtype=torch.float16, device=dev),
                          torch.empty(inp, dtype=torch.int32, device=dev),
                          torch.empty(inp, dtype=torch.int32, device=dev), None)
-    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order), dev, workspace)
+    ws = _workspace(gptq_workspace_bytes(rows, inp, n, act_order, g), dev, workspace)
     err = ctypes.c_double(0.0)
     _check(lib.awq_gptq_quantize_layer(_ptr(W), rows, inp, _ptr(X), n, _ptr(s), bits, g,
                                        float(damp), int(bool(act_order)), _ptr(out.qweight),

@@ -190,28 +190,26 @@ SweepWs carve_sweep(Carver& c, int64_t out, int64_t in) {
 
 struct GptqWs {
   DeviceStatus* st;
-  float* H;      // X^T X, kept for the output error
-  float* fwork;  // factor scratch; U is written over its first in * in floats, then
-                 // the error's bf16 split of H goes after it
-  float* Wq;     // sweep copy of W; later the error's bf16 split of D
-  float* Err;
+  double* H;       // X^T X (fp64 sums), kept for the output error
+  void* fwork;     // FP64 factor (L first); later the error's bf16 split of H
+  float* Wq;       // W in quantization order (read by the sweep); later the bf16 split of D
   int8_t* codes;
   float* qscale;
-  float* dW;     // W - What (fp32, memory order)
+  float* dW;       // W - What (fp32, memory order)
   int32_t* perm;
   int32_t* invperm;
   double* colpart;
   double* sumsq;
   double* partials;
   double* err;
+  Sweep64Ws sw;
 };
-GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int act_order) {
+GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int g, int act_order) {
   GptqWs w;
   w.st = c.take<DeviceStatus>(1);
-  w.H = c.take<float>(in * in);
-  w.fwork = c.take<float>(factor_workspace_floats(in));
+  w.H = c.take<double>(in * in);
+  w.fwork = c.take<uint8_t>(factor64_workspace_bytes(in));
   w.Wq = c.take<float>(out * in);
-  w.Err = c.take<float>(out * kSweepB);
   w.codes = c.take<int8_t>(out * in);
   w.qscale = c.take<float>(out * ceil_div(in, 1));  // sized for g >= 1
   w.dW = c.take<float>(out * in);
@@ -221,6 +219,8 @@ GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int act_order) 
   w.sumsq = c.take<double>(in);
   w.partials = c.take<double>(err_via_h_partials(out, in));
   w.err = c.take<double>(1);
+  uint8_t* sb = c.take<uint8_t>(sweep64_workspace_bytes(out, in, g));
+  carve_sweep64(sb, out, in, g, &w.sw);
   return w;
 }
 
@@ -307,9 +307,9 @@ int check_ws(void* ws, size_t have, size_t need) {
   return have >= need ? PIQ_OK : PIQ_ERR_WORKSPACE_TOO_SMALL;
 }
 
-size_t gptq_ws_bytes(int64_t out, int64_t in, int64_t n, int act_order) {
+size_t gptq_ws_bytes(int64_t out, int64_t in, int64_t n, int g, int act_order) {
   Carver c(nullptr);
-  carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  carve_gptq(c, out, in, n, g, act_order ? 1 : 0);
   return c.bytes();
 }
 
@@ -330,14 +330,14 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
   PIQ_TRY(injected_fault());
   DeviceInfo info;
   PIQ_TRY(device_info(&info));
-  PIQ_TRY(check_ws(workspace, ws_bytes, gptq_ws_bytes(out, in, n, act_order)));
+  PIQ_TRY(check_ws(workspace, ws_bytes, gptq_ws_bytes(out, in, n, g, act_order)));
   Carver c(workspace);
-  GptqWs w = carve_gptq(c, out, in, n, act_order ? 1 : 0);
+  GptqWs w = carve_gptq(c, out, in, n, g, act_order ? 1 : 0);
   PhaseClock clk(0, s);
 
   PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
   // 1. H = X^T X on the tensor cores (scaled to H' for the AWQ-scaled layer)
-  PIQ_TRY(launch_syrk_xtx(X, n, in, w.H, 0, w.st, s));
+  PIQ_TRY(launch_syrk64(X, n, in, w.H, w.st, s));
   if (s_ch) PIQ_TRY(launch_scale_upper(w.H, in, s_ch, w.st, s));
   clk.mark();
   // 2. quantization order
@@ -357,13 +357,13 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
       PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
   }
   clk.mark();
-  // 3. damping + U (H is kept; U goes over the factor's own scratch)
-  float* U = w.fwork;
-  PIQ_TRY(run_upper_factor(w.H, in, damp, qperm, U, w.fwork, w.st, s));
+  // 3. damping + the FP64 factor L of J H_d J (H is kept for the error)
+  double* L = nullptr;
+  PIQ_TRY(run_factor64(w.H, in, damp, qperm, w.fwork, &L, w.st, s));
   clk.mark();
-  // 4. blocked sweep on the permuted (and scaled) copy
+  // 4. the sweep on R = J L J over the permuted (and scaled) copy of W
   PIQ_TRY(launch_gather_columns(W, out, in, qperm, s_ch, w.Wq, s));
-  PIQ_TRY(run_gptq_sweep(w.Wq, out, in, U, bits, g, w.codes, w.qscale, zeros, w.Err, w.st, s));
+  PIQ_TRY(run_gptq_sweep64(w.Wq, out, in, L, bits, g, w.codes, w.qscale, zeros, w.sw, w.st, s));
   clk.mark();
   // 5. pack (+ D = W diag(s) - What' for the error)
   PIQ_TRY(launch_pack(w.codes, w.qscale, zeros, qinv, out, in, bits, g, W, s_ch, qweight, scales,
@@ -373,8 +373,7 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
   //    (scratch: the sweep copy, and the factor's inverse region after U)
   if (out_err)
     PIQ_TRY(run_error_via_h(w.dW, out, in, w.H, reinterpret_cast<uint16_t*>(w.Wq),
-                            reinterpret_cast<uint16_t*>(w.fwork + in * in), w.partials, w.err,
-                            w.st, s));
+                            reinterpret_cast<uint16_t*>(w.fwork), w.partials, w.err, w.st, s));
   clk.mark();
   double e = 0.0;
   if (out_err)
@@ -478,9 +477,10 @@ int piq_gptq_sweep(const float* Wp, int64_t out, int64_t in, const float* U, int
   return finish_call(w.st, s, nullptr);
 }
 
-int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int act_order, size_t* bytes) {
-  if (bytes == nullptr || out < 1 || in < 1 || n < 1) return PIQ_ERR_INVALID_ARG;
-  *bytes = gptq_ws_bytes(out, in, n, act_order);
+int piq_gptq_workspace_bytes(int64_t out, int64_t in, int64_t n, int g, int act_order,
+                             size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1 || n < 1 || g < 1) return PIQ_ERR_INVALID_ARG;
+  *bytes = gptq_ws_bytes(out, in, n, g, act_order);
   return PIQ_OK;
 }
 

@@ -41,19 +41,37 @@ __global__ void split_vec_kernel(const float4* __restrict__ d, int64_t n4, uint2
   }
 }
 
+// Four consecutive entries of a row of H as floats (H fp32 or fp64).
+__device__ __forceinline__ void load4(const float* row, int64_t t, float (&xs)[4]) {
+  const float4 x = reinterpret_cast<const float4*>(row)[t];
+  xs[0] = x.x;
+  xs[1] = x.y;
+  xs[2] = x.z;
+  xs[3] = x.w;
+}
+__device__ __forceinline__ void load4(const double* row, int64_t t, float (&xs)[4]) {
+  const double2 a = reinterpret_cast<const double2*>(row)[2 * t];
+  const double2 b = reinterpret_cast<const double2*>(row)[2 * t + 1];
+  xs[0] = static_cast<float>(a.x);
+  xs[1] = static_cast<float>(a.y);
+  xs[2] = static_cast<float>(b.x);
+  xs[3] = static_cast<float>(b.y);
+}
+
 // Hu[k][j] = H[k][j] (k < j), H[k][k] / 2, 0 (k > j), split; in % 4 == 0.
-__global__ void split_upper_half_kernel(const float* __restrict__ H, int64_t in,
+template <typename T>
+__global__ void split_upper_half_kernel(const T* __restrict__ H, int64_t in,
                                         uint2* __restrict__ hi, uint2* __restrict__ lo) {
   const int64_t in4 = in >> 2;
   for (int64_t k = blockIdx.y; k < in; k += gridDim.y) {
-    const float4* row = reinterpret_cast<const float4*>(H + k * in);
+    const T* row = H + k * in;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < in4;
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
       const int64_t j = 4 * t;
       float v[4] = {0.f, 0.f, 0.f, 0.f};
       if (j + 3 >= k) {  // some column on or above the diagonal
-        const float4 x = row[t];
-        const float xs[4] = {x.x, x.y, x.z, x.w};
+        float xs[4];
+        load4(row, t, xs);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           v[e] = (j + e > k) ? xs[e] : (j + e == k ? 0.5f * xs[e] : 0.f);
@@ -80,9 +98,10 @@ unsigned grid_1d(int64_t work) {
 
 int64_t err_via_h_partials(int64_t out, int64_t in) { return err_dot_partials_count(out, in); }
 
-int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uint16_t* dsplit,
-                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
-                    cudaStream_t stream) {
+template <typename T>
+int error_via_h(const float* D, int64_t out, int64_t in, const T* H, uint16_t* dsplit,
+                uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                cudaStream_t stream) {
   if (out < 1 || in < 8 || in % 8 != 0) return PIQ_ERR_INVALID_ARG;
   uint16_t* d_hi = dsplit;
   uint16_t* d_lo = dsplit + out * in;
@@ -97,13 +116,25 @@ int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uin
     dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in / 4, 256), 16)),
               static_cast<unsigned>(std::min<int64_t>(in, 65535)));
     note_launch();
-    split_upper_half_kernel<<<grid, 256, 0, stream>>>(H, in, reinterpret_cast<uint2*>(h_hi),
-                                                      reinterpret_cast<uint2*>(h_lo));
+    split_upper_half_kernel<T><<<grid, 256, 0, stream>>>(H, in, reinterpret_cast<uint2*>(h_hi),
+                                                         reinterpret_cast<uint2*>(h_lo));
     if (!launch_ok()) return PIQ_ERR_CUDA;
   }
   int rc = launch_err_dot(d_hi, d_lo, h_hi, h_lo, D, out, in, partials, st, stream);
   if (rc != PIQ_OK) return rc;
   return launch_reduce_sum(partials, err_dot_partials_count(out, in), 1, err, stream);
+}
+
+int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uint16_t* dsplit,
+                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                    cudaStream_t stream) {
+  return error_via_h(D, out, in, H, dsplit, hsplit, partials, err, st, stream);
+}
+
+int run_error_via_h(const float* D, int64_t out, int64_t in, const double* H, uint16_t* dsplit,
+                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                    cudaStream_t stream) {
+  return error_via_h(D, out, in, H, dsplit, hsplit, partials, err, st, stream);
 }
 
 }  // namespace piq

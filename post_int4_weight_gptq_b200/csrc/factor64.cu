@@ -1,0 +1,350 @@
+// FP64-grade factor of the damped proxy Hessian for the GPTQ sweep.
+//
+// "GPTQ versus AWQ objectives", section "A strong answer" (listing): H +=
+// damp * mean(diag H) * I, then U = cholesky(inv(H)).T with inv(H_d) = U^T U.
+// Section "What interviewers probe next": the damping keeps the factorization
+// stable; act-order takes columns by decreasing diag(H).
+//
+// Route (exact identities, no inverse of H): with J the index reversal and
+// P = J H_d J = L L^T (lower Cholesky), R = J L J is upper triangular with
+// H_d = R R^T and U = inv(R).  The sweep (sweep64.cu) runs on R and on the
+// inverses of R's diagonal blocks only, so the full triangular inverse is never
+// formed.  Everything here is FP64 or FP64-grade: at a 28672-column layer the
+// decisions of the rounding loop need U to about 1e-9 of U_jj, which an FP32
+// factorization does not reach.
+//
+//   1. lambda = damp * mean(diag H), P = J H_p J + lambda I (lower, fp64)
+//   2. right-looking blocked Cholesky, 128-wide panels: the diagonal block is
+//      factored and inverted in FP64 on one SM (chol64_block_kernel); the panel
+//      below is L21 = A21 inv(L11)^T and the trailing matrix A22 -= L21 L21^T,
+//      both on the INT8 tensor cores with FP64 accumulation (ozaki.cu)
+//   3. inverses of R's diagonal blocks for the sweep (block_inverse_kernel)
+// A non-positive pivot sets PIQ_ERR_NOT_PD.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace piq {
+
+namespace {
+
+constexpr int NB = 128;
+constexpr int LDS = NB + 1;  // fp64 shared-memory row stride
+constexpr int CT = 512;      // threads of the diagonal-block kernel
+// Columns per superpanel: inside one, each 128-wide panel updates only the
+// superpanel's own later columns; the rest of the trailing matrix gets the
+// whole superpanel's product at once (K = 1024), which cuts the fp64
+// read-modify-write traffic of the trailing matrix by eight.
+constexpr int kSuperPanel = 1024;
+
+__global__ void diag_mean64_kernel(const double* H, int64_t in, float damp, DeviceStatus* st,
+                                   double* lambda) {
+  __shared__ double sh[256];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < in; i += 256) acc += H[i * in + i];
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double lam = static_cast<double>(damp) * (sh[0] / static_cast<double>(in));
+    st->lambda = lam;
+    *lambda = lam;
+  }
+}
+
+// P[a][b] (b <= a) = H[s(a)][s(b)] + lambda [a == b], s(a) = perm[in-1-a]; fp64.
+__global__ void build_rev64_kernel(const double* H, int64_t in, const int32_t* perm,
+                                   const double* lambda, double* P) {
+  const int64_t a0 = static_cast<int64_t>(blockIdx.y) * 32;
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * 32;
+  if (b0 > a0 + 31) return;
+  const double lam = *lambda;
+  const int64_t b = b0 + threadIdx.x;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int64_t a = a0 + r;
+    if (a >= in || b >= in || b > a) continue;
+    const int64_t x = perm ? perm[in - 1 - a] : in - 1 - a;
+    const int64_t y = perm ? perm[in - 1 - b] : in - 1 - b;
+    const int64_t lo = x < y ? x : y, hi = x < y ? y : x;
+    double v = H[lo * in + hi];
+    if (a == b) v += lam;
+    P[a * in + b] = v;
+  }
+}
+
+// Factor the nb x nb diagonal block of P at (o, o) in place (lower Cholesky,
+// FP64) and write its inverse to X11 (128 x 128, row-major, zeros above the
+// diagonal and outside nb).  Rows/cols >= nb are padded with the identity.
+// Pivot by pivot: the pivot's square root, the column scaled, then the
+// trailing lower triangle updated by all threads.  The inverse is formed one
+// column per thread by forward substitution, kept transposed in the strictly
+// upper part of the same shared array (the factor occupies the lower part).
+__global__ void __launch_bounds__(CT)
+    chol64_block_kernel(double* P, int64_t ld, int64_t o, int nb, double* X11,
+                        DeviceStatus* st) {
+  extern __shared__ __align__(16) double S[];  // [NB][LDS]
+  __shared__ double xd[NB];                    // diagonal of the inverse
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (status_bad(st)) return;
+  if (tid == 0) bad = 0;
+  for (int idx = tid; idx < NB * NB; idx += CT) {
+    const int i = idx >> 7, j = idx & (NB - 1);
+    double v = 0.0;
+    if (i < nb && j <= i) v = P[(o + i) * ld + (o + j)];
+    else if (i == j) v = 1.0;
+    S[i * LDS + j] = v;
+  }
+  __syncthreads();
+  for (int j = 0; j < NB; ++j) {
+    const double d = S[j * LDS + j];
+    if (!(d > 0.0)) {  // uniform: every thread reads the same value
+      if (tid == 0) {
+        bad = 1;
+        set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + j));
+      }
+      break;
+    }
+    const double ljj = sqrt(d);
+    const double r = 1.0 / ljj;
+    __syncthreads();  // everyone has read S[j][j]
+    if (tid == 0) S[j * LDS + j] = ljj;
+    for (int i = j + 1 + tid; i < NB; i += CT) S[i * LDS + j] *= r;
+    __syncthreads();
+    // A22 -= l l^T on the lower triangle below pivot j: pairs (i, k), j < k <= i
+    const int m = NB - 1 - j;
+    const int npairs = m * (m + 1) / 2;
+    for (int t = tid; t < npairs; t += CT) {
+      // t -> (ii, kk) with 0 <= kk <= ii < m, row-major over the triangle
+      int ii = static_cast<int>((sqrt(8.0 * t + 1.0) - 1.0) * 0.5);
+      while ((ii + 1) * (ii + 2) / 2 <= t) ++ii;
+      while (ii * (ii + 1) / 2 > t) --ii;
+      const int kk = t - ii * (ii + 1) / 2;
+      const int i = j + 1 + ii, k = j + 1 + kk;
+      S[i * LDS + k] = fma(-S[i * LDS + j], S[k * LDS + j], S[i * LDS + k]);
+    }
+    __syncthreads();
+  }
+  __syncthreads();
+  if (bad) return;
+  // inverse: column c by forward substitution, X[i][c] stored at S[c][i] (i > c)
+  if (tid < NB) {
+    const int c = tid;
+    const double xcc = 1.0 / S[c * LDS + c];
+    xd[c] = xcc;
+    for (int i = c + 1; i < NB; ++i) {
+      double acc0 = S[i * LDS + c] * xcc, acc1 = 0.0;
+      int k = c + 1;
+      for (; k + 1 < i; k += 2) {
+        acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
+        acc1 = fma(S[i * LDS + k + 1], S[c * LDS + k + 1], acc1);
+      }
+      if (k < i) acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
+      S[c * LDS + i] = -(acc0 + acc1) / S[i * LDS + i];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < NB * NB; idx += CT) {
+    const int i = idx >> 7, j = idx & (NB - 1);
+    if (i < nb && j <= i) P[(o + i) * ld + (o + j)] = S[i * LDS + j];
+    double x = 0.0;
+    if (i < nb && j < nb) x = (j < i) ? S[j * LDS + i] : (j == i ? xd[i] : 0.0);
+    X11[i * NB + j] = x;
+  }
+}
+
+// Inverse of R's diagonal block [b, e) for every sweep block, R = J L J
+// (R[i][k] = L[in-1-i][in-1-k]).  One CTA per block: U = inv(R_bb) is upper
+// triangular; column c by back substitution, one thread per column.
+// Out: Ub[blk][128][128] row-major, zeros below the diagonal and outside kb.
+__global__ void __launch_bounds__(NB)
+    block_inverse_kernel(const double* L, int64_t in, const int64_t* starts, int nblocks,
+                         double* Ub) {
+  extern __shared__ __align__(16) double S[];  // [NB][LDS]: R block, then U transposed
+  __shared__ double ud[NB];
+  const int blk = blockIdx.x;
+  if (blk >= nblocks) return;
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();  // L and the block starts come from earlier work of the stream
+  const int64_t b = starts[blk], e = starts[blk + 1];
+  const int kb = static_cast<int>(e - b);
+  for (int idx = tid; idx < NB * NB; idx += NB) {
+    const int i = idx >> 7, k = idx & (NB - 1);
+    double v = 0.0;
+    if (i < kb && k < kb && k >= i) v = L[(in - 1 - b - i) * in + (in - 1 - b - k)];
+    else if (i == k) v = 1.0;
+    S[i * LDS + k] = v;
+  }
+  __syncthreads();
+  // U[c][c] = 1 / R_cc; U[i][c] = -(sum_{k=i+1..c} R_ik U_kc) / R_ii, i = c-1 .. 0;
+  // U[i][c] (i < c) is kept at S[c][i] (the strictly lower part, free)
+  {
+    const int c = tid;
+    const double ucc = 1.0 / S[c * LDS + c];
+    ud[c] = ucc;
+    for (int i = c - 1; i >= 0; --i) {
+      double acc0 = S[i * LDS + c] * ucc, acc1 = 0.0;
+      int k = i + 1;
+      for (; k + 1 < c; k += 2) {
+        acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
+        acc1 = fma(S[i * LDS + k + 1], S[c * LDS + k + 1], acc1);
+      }
+      if (k < c) acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
+      S[c * LDS + i] = -(acc0 + acc1) / S[i * LDS + i];
+    }
+  }
+  __syncthreads();
+  double* out = Ub + static_cast<int64_t>(blk) * NB * NB;
+  for (int idx = tid; idx < NB * NB; idx += NB) {
+    const int i = idx >> 7, k = idx & (NB - 1);
+    double u = 0.0;
+    if (i < kb && k < kb) u = (k > i) ? S[k * LDS + i] : (k == i ? ud[i] : 0.0);
+    out[idx] = u;
+  }
+}
+
+constexpr int kBlockSmem = NB * LDS * 8;
+
+}  // namespace
+
+struct Factor64Ws {
+  double* P;
+  double* X11;
+  double* lam;
+  DigitMat dA, dX, dS;
+};
+
+int64_t carve_factor64(void* base, int64_t in, Factor64Ws* w) {
+  uint8_t* p0 = static_cast<uint8_t*>(base);
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) -> uint8_t* {
+    off = (off + 255) / 256 * 256;
+    uint8_t* p = p0 ? p0 + off : nullptr;
+    off += std::max<int64_t>(bytes, 1);
+    return p;
+  };
+  const int64_t kpad = digit_kpad(NB);
+  w->P = reinterpret_cast<double*>(take(in * in * 8));
+  w->X11 = reinterpret_cast<double*>(take(NB * NB * 8));
+  w->lam = reinterpret_cast<double*>(take(64));
+  w->dA.s = kFactorDigits;
+  w->dA.kpad = kpad;
+  w->dA.q = reinterpret_cast<int8_t*>(take(static_cast<int64_t>(kFactorDigits) * in * kpad));
+  w->dA.ex = reinterpret_cast<int*>(take(in * 4));
+  w->dX.s = kFactorDigits;
+  w->dX.kpad = kpad;
+  w->dX.q = reinterpret_cast<int8_t*>(take(static_cast<int64_t>(kFactorDigits) * NB * kpad));
+  w->dX.ex = reinterpret_cast<int*>(take(NB * 4));
+  const int64_t spk = digit_kpad(std::min<int64_t>(kSuperPanel, in));
+  w->dS.s = kFactorDigits;
+  w->dS.kpad = spk;
+  w->dS.q = reinterpret_cast<int8_t*>(take(static_cast<int64_t>(kFactorDigits) * in * spk));
+  w->dS.ex = reinterpret_cast<int*>(take(in * 4));
+  return (off + 255) / 256 * 256;
+}
+
+int64_t factor64_workspace_bytes(int64_t in) {
+  Factor64Ws w;
+  return carve_factor64(nullptr, in, &w);
+}
+
+int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, void* work,
+                 double** L_out, DeviceStatus* st, cudaStream_t stream) {
+  if (in < 1) return PIQ_ERR_INVALID_ARG;
+  Factor64Ws fw;
+  carve_factor64(work, in, &fw);
+  double* P = fw.P;
+  double* X11 = fw.X11;
+  double* lam = fw.lam;
+  DigitMat dA = fw.dA;
+  DigitMat dX = fw.dX;
+  const int64_t ld = in;
+
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(chol64_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kBlockSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kBlockSmem) != cudaSuccess)
+      return PIQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  note_launch();
+  diag_mean64_kernel<<<1, 256, 0, stream>>>(H, in, damp, st, lam);
+  {
+    dim3 grid(static_cast<unsigned>(ceil_div(in, 32)), static_cast<unsigned>(ceil_div(in, 32)));
+    note_launch();
+    build_rev64_kernel<<<grid, dim3(32, 8), 0, stream>>>(H, in, perm, lam, P);
+  }
+  if (!launch_ok()) return PIQ_ERR_CUDA;
+
+  for (int64_t s0 = 0; s0 < in; s0 += kSuperPanel) {
+    const int64_t s1 = std::min<int64_t>(s0 + kSuperPanel, in);
+    for (int64_t k0 = s0; k0 < s1; k0 += NB) {
+      const int nb = static_cast<int>(std::min<int64_t>(NB, in - k0));
+      note_launch();
+      if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kBlockSmem, stream, P, ld, k0, nb,
+                     X11, st) != cudaSuccess)
+        return PIQ_ERR_CUDA;
+      const int64_t rem = in - k0 - nb;
+      if (rem <= 0) continue;
+      double* A21 = P + (k0 + nb) * ld + k0;
+      // L21 = A21 inv(L11)^T: C[r][c] = sum_k A21[r][k] X11[c][k]
+      dA.rows = rem;
+      dX.rows = nb;
+      dA.kpad = dX.kpad = digit_kpad(nb);
+      int rc = launch_slice(A21, ld, 1, rem, nb, kFactorDigits, &dA, stream);
+      if (rc == PIQ_OK) rc = launch_slice(X11, NB, 1, nb, nb, kFactorDigits, &dX, stream);
+      if (rc == PIQ_OK) rc = launch_ozaki_gemm(rem, nb, dA, dX, 1.0, 0, 0, A21, ld, st, stream);
+      // this panel's update of the superpanel's later columns, every row below:
+      // A[k0+nb:, k0+nb:s1] -= L21 L21[:s1-k0-nb]^T (c <= r)
+      const int64_t ncol = s1 - (k0 + nb);
+      if (rc == PIQ_OK) rc = launch_slice(A21, ld, 1, rem, nb, kFactorDigits, &dA, stream);
+      if (rc == PIQ_OK && ncol > 0)
+        rc = launch_ozaki_gemm(rem, ncol, dA, dA, -1.0, 1, 1, P + (k0 + nb) * ld + (k0 + nb), ld,
+                               st, stream);
+      if (rc != PIQ_OK) return rc;
+    }
+    // the superpanel's update of the rest: A[s1:, s1:] -= L[s1:, s0:s1] L[s1:, s0:s1]^T
+    const int64_t rest = in - s1;
+    if (rest > 0) {
+      DigitMat dS = fw.dS;
+      dS.rows = rest;
+      dS.kpad = digit_kpad(s1 - s0);
+      int rc = launch_slice(P + s1 * ld + s0, ld, 1, rest, s1 - s0, kFactorDigits, &dS, stream);
+      if (rc == PIQ_OK)
+        rc = launch_ozaki_gemm(rest, rest, dS, dS, -1.0, 1, 1, P + s1 * ld + s1, ld, st, stream);
+      if (rc != PIQ_OK) return rc;
+    }
+  }
+  *L_out = P;
+  return PIQ_OK;
+}
+
+int launch_block_inverses(const double* L, int64_t in, const int64_t* starts_dev, int nblocks,
+                          double* Ub, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kBlockSmem) != cudaSuccess)
+      return PIQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  note_launch();
+  if (launch_pdl(block_inverse_kernel, dim3(static_cast<unsigned>(nblocks)), dim3(NB), kBlockSmem,
+                 stream, L, in, starts_dev, nblocks, Ub) != cudaSuccess)
+    return PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+}  // namespace piq

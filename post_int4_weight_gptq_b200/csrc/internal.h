@@ -38,6 +38,10 @@ int finish_call(DeviceStatus* st, cudaStream_t stream, DeviceStatus* host_st);
 // H (+)= X^T X: upper-triangle tiles of a [in, in] fp32 matrix (row-major).
 int launch_syrk_xtx(const uint16_t* X, int64_t n, int64_t in, float* H, int accumulate,
                     DeviceStatus* st, cudaStream_t stream);
+// H = X^T X with FP64 sums (128-sample tensor-core chunks added in FP64):
+// upper triangle of a [in, in] fp64 matrix (syrk64.cu).
+int launch_syrk64(const uint16_t* X, int64_t n, int64_t in, double* H, DeviceStatus* st,
+                  cudaStream_t stream);
 // Fused ||X D_b^T||_F^2 for b < batch, D stacked [batch][rows][in] bf16.
 // Writes four doubles per output tile into `partials` (size: sumsq_partials_count).
 int launch_err_sumsq(const uint16_t* X, int64_t n, int64_t in, const uint16_t* D, int64_t rows,
@@ -63,6 +67,9 @@ int64_t err_dot_partials_count(int64_t out, int64_t in);
 // (upper triangle read).  Scratch: dsplit 2 out in, hsplit 2 in in bf16;
 // partials err_via_h_partials(out, in) doubles.
 int run_error_via_h(const float* D, int64_t out, int64_t in, const float* H, uint16_t* dsplit,
+                    uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
+                    cudaStream_t stream);
+int run_error_via_h(const float* D, int64_t out, int64_t in, const double* H, uint16_t* dsplit,
                     uint16_t* hsplit, double* partials, double* err, DeviceStatus* st,
                     cudaStream_t stream);
 int64_t err_via_h_partials(int64_t out, int64_t in);
@@ -112,6 +119,65 @@ int launch_act_order_perm(const double* sumsq, int64_t in, int32_t* perm, int32_
                           cudaStream_t stream);
 int launch_identity_perm(int64_t in, int32_t* perm, int32_t* invperm, cudaStream_t stream);
 
+// ------------------------------------ FP64-grade GEMM on the INT8 tensor cores (ozaki.cu)
+// A matrix as s signed 7-bit digits per entry, scaled per row by 2^ex[row]:
+// q[i][row][kpad] int8 (K-major, zero padded to kpad), ex[row] int32.
+constexpr int kMaxDigits = 7;
+constexpr int kFactorDigits = 6;  // Cholesky panel products: ~1e-12 relative
+constexpr int kSweepDigits = 5;   // GPTQ block updates: ~1e-10 relative
+struct DigitMat {
+  int8_t* q = nullptr;
+  int* ex = nullptr;
+  int64_t rows = 0, kpad = 0;
+  int s = 0;
+};
+int64_t digit_kpad(int64_t K);  // K rounded up to a multiple of 64
+// Digits of the rows x K matrix whose entry (r, k) is src[r * rs + k * ks]
+// (strides may be negative); out->rows, kpad and s must match.
+int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_t K, int s,
+                 DigitMat* out, cudaStream_t stream);
+// C[r][c] (+)= alpha sum_k A(r, k) B(c, k) for r < M, c < N, C fp64 row-major;
+// beta 0 stores, 1 adds; lower != 0 touches only c <= r.
+int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B, double alpha,
+                      int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
+                      cudaStream_t stream);
+
+// ---------------------------------------------- FP64-grade factor (factor64.cu)
+// L = chol(J H_p J + lambda I) in fp64 (lower, row-major [in][in] inside
+// `work`); R = J L J is the upper factor with H_d = R R^T and U = inv(R).
+int64_t factor64_workspace_bytes(int64_t in);
+int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, void* work,
+                 double** L_out, DeviceStatus* st, cudaStream_t stream);
+// Ub[blk] = inv(R[b:e, b:e]) (128 x 128 fp64) for the blocks [starts[blk], starts[blk+1]).
+int launch_block_inverses(const double* L, int64_t in, const int64_t* starts_dev, int nblocks,
+                          double* Ub, cudaStream_t stream);
+
+// ------------------------------------------------ FP64 sweep on R (sweep64.cu)
+struct Sweep64Ws {
+  int nblocks = 0;
+  double* acc = nullptr;     // [out][in] accumulated updates
+  double* Ub = nullptr;      // [nblocks][128][128]
+  int64_t* starts = nullptr; // [nblocks + 1]
+  int8_t* dq = nullptr;      // digits of W0 - Q of one block [s][out][128]
+  int* dex = nullptr;
+  int8_t* rq = nullptr;      // digits of one block row of R [s][in][128]
+  int* rex = nullptr;
+  double* yscr = nullptr;    // group scales wider than a block
+  double* dsb = nullptr;     // W0 - Q of a superblock [out][1024] (fp64)
+  int8_t* sbq = nullptr;     // its digits, and those of R's rows of the superblock
+  int* sbex = nullptr;
+  int8_t* sbrq = nullptr;
+  int* sbrex = nullptr;
+};
+int sweep64_blocks(int64_t in, int g);
+int64_t carve_sweep64(void* base, int64_t out, int64_t in, int g, Sweep64Ws* w);
+int64_t sweep64_workspace_bytes(int64_t out, int64_t in, int g);
+// Codes and scales (and zero-points) of the listing's loop over W0 (quantization
+// order, fp32, not modified) with the factor L of run_factor64.
+int run_gptq_sweep64(const float* W0, int64_t out, int64_t in, const double* L, int bits, int g,
+                     int8_t* codes, float* qscale, uint8_t* qzero, const Sweep64Ws& w,
+                     DeviceStatus* st, cudaStream_t stream);
+
 // ---------------------------------------------------------------- sweep (sweep.cu)
 constexpr int kSweepB = 128;
 // Full blocked sweep over quantization-order weights Wq (updated in place).
@@ -138,6 +204,8 @@ int launch_pack(const int8_t* codes, const float* qscale, const uint8_t* qzero,
 // H = diag(1/s) H diag(1/s) on the upper triangle, in place; a non-finite or
 // non-positive s_k sets PIQ_ERR_INVALID_ARG (where = k) in st.
 int launch_scale_upper(float* H, int64_t in, const float* s, DeviceStatus* st,
+                       cudaStream_t stream);
+int launch_scale_upper(double* H, int64_t in, const float* s, DeviceStatus* st,
                        cudaStream_t stream);
 // sumsq[j] /= s_j^2 (FP64).
 int launch_scale_sumsq(double* sumsq, int64_t in, const float* s, cudaStream_t stream);

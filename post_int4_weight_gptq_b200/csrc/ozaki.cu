@@ -1,0 +1,440 @@
+// FP64-grade GEMM on the INT8 tensor cores (tcgen05 kind::i8), for the steps
+// whose results decide rounding sites: the Cholesky factor of the damped
+// Hessian and the GPTQ block updates.
+//
+// Why: the GPTQ listing of "GPTQ versus AWQ objectives" ("A strong answer")
+// forms U = cholesky(inv(H)) and pushes every rounding error through it; at a
+// 28672-column layer an FP32 factor (or FP32-accumulated updates) moves w/scale
+// by ~1e-5, which flips several thousand rounding decisions against an FP64
+// evaluation of the same loop.  B200 has ~37 TFLOP/s of FP64 but ~2.6 POP/s of
+// INT8, so FP64-grade products are formed from exact integer ones.
+//
+// Method (splitting of floating-point operands into small integers, summed
+// exactly in integer arithmetic; Ozaki et al., "Error-free transformations of
+// matrix multiplication", and its integer-unit variants): every row of an
+// operand is scaled by a power of two 2^e (e from frexp of the row's largest
+// magnitude, so the row lies in (-1, 1)), and then written as
+//     y = 2^-6 (q0 + 2^-7 (q1 + 2^-7 (q2 + ...)))
+// with signed digits q_i in [-64, 64] (each step rounds to nearest, so the
+// remainder stays in [-1/2, 1/2] and the next digit fits in 7 bits plus sign).
+// s digits keep about 6 + 7 (s - 1) bits of every entry relative to its row's
+// largest one.  For C = A B^T the integer products q_i(A) q_j(B) with the same
+// weight 2^(-7 (i + j)) go to one int32 accumulator d = i + j in TMEM (exact:
+// at most 64 * 64 * K * (d + 1) < 2^31 for K (d + 1) < 2^19); pairs with
+// i + j >= s are dropped (their weight is below 2^(-7 s)).  The epilogue turns
+// the s accumulators into one fp64 value by Horner's rule in powers of 2^-7,
+// scales it by 2^(e_A(r) + e_B(c) - 12) and alpha, and adds it to (or stores
+// it into) an fp64 C.  With s = 6 the relative error of each product sum is
+// about 1e-12 of max|A_r| max|B_c| K, far below FP32 (6e-8).
+//
+// Layout: digits are stored K-major, q[i][row][kpad] int8 with kpad a multiple
+// of 64 (zero padded), and the exponents e[row] int32.  Tiles: 128 rows of A x
+// 64 rows of B, K in blocks of 64 bytes (64-byte swizzle); a pipeline stage
+// holds all s digit tiles of A and of B for one k block.  TMEM holds the s
+// accumulators side by side (s * 64 columns), double-buffered when s <= 4.
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 lane 0
+// issues the MMAs; warps 2..5 drain TMEM (warp w reads lanes 32 (w % 4) ..)
+// and own 32 rows of C each.  Every wait is bounded; no multicast loads.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "internal.h"
+
+namespace piq {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 64;
+constexpr int BK = 64;                        // int8 digits = one 64-byte row
+constexpr int A_TILE = BM * BK;               // 8 KB per digit
+constexpr int B_TILE = BN * BK;               // 4 KB per digit
+constexpr int THREADS = 192;
+constexpr int MAX_SMEM = 227 * 1024;
+
+struct OzParams {
+  int M, N, K, s;
+  int m_tiles, n_tiles, num_tiles;
+  int nbuf;             // TMEM accumulator sets (1 or 2)
+  int stages;
+  int stage_bytes;
+  double alpha;
+  int beta;             // 0: C = alpha A B^T; 1: C += alpha A B^T
+  int lower;            // only entries c <= r (tiles touching the lower triangle)
+  double* C;
+  int64_t ldc;
+  const int* ea;
+  const int* eb;
+  DeviceStatus* st;
+};
+
+__device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& nt) {
+  if (p.lower) {
+    // row tile mt holds column tiles 0 .. last(mt) where last = floor((128 mt + 127) / 64)
+    // = 2 mt + 1 (clipped to n_tiles - 1); walk rows (few hundred at most)
+    int acc = 0;
+    for (int m = 0; m < p.m_tiles; ++m) {
+      const int cnt = min(p.n_tiles, 2 * m + 2);
+      if (t < acc + cnt) {
+        mt = m;
+        nt = t - acc;
+        return;
+      }
+      acc += cnt;
+    }
+    mt = nt = 0;
+  } else {
+    mt = t / p.n_tiles;
+    nt = t - mt * p.n_tiles;
+  }
+}
+
+// Instruction descriptor: kind::i8, signed A and B, s32 accumulate, K-major
+// A and B, M = 128, N = 64.
+__host__ __device__ constexpr uint32_t idesc_i8() {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+constexpr uint32_t kLayoutSw64 = 4;  // smem descriptor: 64-byte swizzle
+
+__device__ __forceinline__ void tmem_ld_i32x32(uint32_t taddr, int (&v)[32]) {
+  float f[32];
+  tmem_ld_32x32b_x32(taddr, f);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __float_as_int(f[i]);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    ozaki_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, OzParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * p.stage_bytes);
+  uint64_t* empty = full + p.stages;
+  uint64_t* acc_full = empty + p.stages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (p.K + BK - 1) / BK;
+  pdl_wait();
+  const bool skip = status_bad(p.st);
+  const int S = p.s;
+  const uint32_t set_cols = static_cast<uint32_t>(S * BN);
+
+  if (skip) {
+  } else if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_of(p, t, mt, nt);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int st = it % p.stages;
+          const uint32_t ph = (it / p.stages) & 1u;
+          if (!mbar_wait(&empty[st], ph ^ 1u, p.st, 41)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + st * p.stage_bytes;
+          uint8_t* sb = sa + S * A_TILE;
+          mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(p.stage_bytes));
+          for (int i = 0; i < S; ++i) {
+            tma_load_3d(sa + i * A_TILE, &tmA, &full[st], kb * BK, mt * BM, i);
+            tma_load_3d(sb + i * B_TILE, &tmB, &full[st], kb * BK, nt * BN, i);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_i8();
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++lt) {
+        const int buf = lt % p.nbuf;
+        const uint32_t use = static_cast<uint32_t>(lt / p.nbuf);
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 42)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf) * set_cols;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int st = it % p.stages;
+          const uint32_t ph = (it / p.stages) & 1u;
+          if (!mbar_wait(&full[st], ph, p.st, 43)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + st * p.stage_bytes);
+          const uint32_t b0 = a0 + static_cast<uint32_t>(S * A_TILE);
+          for (int i = 0; i < S; ++i) {
+            for (int j = 0; i + j < S; ++j) {
+              const uint32_t dt = d0 + static_cast<uint32_t>((i + j) * BN);
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk) {
+                const uint64_t ad = smem_desc(a0 + i * A_TILE + kk * 32, 16, 512, kLayoutSw64);
+                const uint64_t bd = smem_desc(b0 + j * B_TILE + kk * 32, 16, 512, kLayoutSw64);
+                // the first product into accumulator d of this tile starts it
+                const bool first = kb == 0 && kk == 0 && i == 0;
+                umma_i8(dt, ad, bd, idesc, first ? 0u : 1u);
+              }
+            }
+          }
+          umma_commit(&empty[st]);
+        }
+        if (ok) umma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    int lt = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
+      int mt, nt;
+      tile_of(p, t, mt, nt);
+      const int buf = lt % p.nbuf;
+      const uint32_t use = static_cast<uint32_t>(lt / p.nbuf);
+      if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 44)) break;
+      tc_fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(buf) * set_cols;
+      const int ear = row < p.M ? __ldg(p.ea + row) : 0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        double v[32];
+        {
+          int a[32];
+          tmem_ld_i32x32(taddr + static_cast<uint32_t>((S - 1) * BN + c * 32), a);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = static_cast<double>(a[i]);
+        }
+        for (int d = S - 2; d >= 0; --d) {
+          int a[32];
+          tmem_ld_i32x32(taddr + static_cast<uint32_t>(d * BN + c * 32), a);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fma(v[i], 0.0078125, static_cast<double>(a[i]));
+        }
+        const int col0 = nt * BN + c * 32;
+        if (row < p.M && col0 < p.N) {
+          double* crow = p.C + static_cast<int64_t>(row) * p.ldc + col0;
+          const int lim = min(32, p.N - col0);
+          const int clim = p.lower ? min(lim, row - col0 + 1) : lim;  // c <= r
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i < clim) {
+              const double sc = ldexp(p.alpha, ear + __ldg(p.eb + col0 + i) - 12);
+              const double val = v[i] * sc;
+              crow[i] = p.beta ? crow[i] + val : val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ----------------------------------------------------------------- digits
+// Row r of the logical rows x K matrix: element (r, k) at src[r * rs + k * ks].
+// One warp per row: pass 1 finds the largest magnitude, pass 2 writes the s
+// digits of every entry (zeros for k in [K, kpad)).
+__global__ void slice_rows_kernel(const double* __restrict__ src, int64_t rs, int64_t ks,
+                                  int64_t rows, int64_t K, int s, int8_t* __restrict__ q,
+                                  int64_t kpad, int* __restrict__ ex) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const double* row = src + r * rs;
+  double m = 0.0;
+  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(row[k * ks]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  int e = 0;
+  if (m > 0.0) frexp(m, &e);  // m = f 2^e with f in [0.5, 1)
+  if (lane == 0) ex[r] = e;
+  const int64_t plane = rows * kpad;
+  // four consecutive k per lane per step: one 32-bit store per digit
+  for (int64_t k0 = 4 * lane; k0 < kpad; k0 += 128) {
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int64_t k = k0 + t;
+      double y = (k < K && m > 0.0) ? ldexp(row[k * ks], 6 - e) : 0.0;  // |y| < 64
+      for (int i = 0; i < s; ++i) {
+        const double di = rint(y);
+        y = (y - di) * 128.0;
+        w[i] |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+      }
+    }
+    for (int i = 0; i < s; ++i)
+      *reinterpret_cast<uint32_t*>(q + i * plane + r * kpad + k0) = w[i];
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_i8() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    tried = true;
+  }
+  return fn;
+}
+
+// int8 digit planes [s][rows][kpad] as a 3-D map {kpad, rows, s}, box {64, box_rows, 1}.
+bool make_digit_map(CUtensorMap* map, const int8_t* q, int64_t rows, int64_t kpad, int s,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn_i8();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kpad), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(s)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kpad),
+                                 static_cast<cuuint64_t>(rows * kpad)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(q), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int64_t digit_kpad(int64_t K) { return (K + BK - 1) / BK * BK; }
+
+int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_t K, int s,
+                 DigitMat* out, cudaStream_t stream) {
+  if (rows < 1 || K < 1 || s < 1 || s > kMaxDigits) return PIQ_ERR_INVALID_ARG;
+  if (out->kpad != digit_kpad(K) || out->s != s || out->rows != rows) return PIQ_ERR_INVALID_ARG;
+  const int64_t threads = rows * 32;
+  note_launch();
+  slice_rows_kernel<<<static_cast<unsigned>(ceil_div(threads, 256)), 256, 0, stream>>>(
+      src, rs, ks, rows, K, s, out->q, out->kpad, out->ex);
+  return launch_ok("digit split launch") ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B, double alpha,
+                      int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
+                      cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return PIQ_OK;
+  if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s > kMaxDigits)
+    return PIQ_ERR_INVALID_ARG;
+  if (A.kpad * (A.s + 1) >= (int64_t)1 << 19) return PIQ_ERR_INVALID_ARG;  // int32 exactness
+  if (M > INT32_MAX || N > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+  DeviceInfo info;
+  int rc = device_info(&info);
+  if (rc != PIQ_OK) return rc;
+  CUtensorMap ma, mb;
+  if (!make_digit_map(&ma, A.q, A.rows, A.kpad, A.s, BM) ||
+      !make_digit_map(&mb, B.q, B.rows, B.kpad, B.s, BN))
+    return PIQ_ERR_INVALID_ARG;
+  OzParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(A.kpad);
+  p.s = A.s;
+  p.m_tiles = static_cast<int>(ceil_div(M, BM));
+  p.n_tiles = static_cast<int>(ceil_div(N, BN));
+  if (lower) {
+    int64_t tot = 0;
+    for (int m = 0; m < p.m_tiles; ++m) tot += std::min<int64_t>(p.n_tiles, 2 * m + 2);
+    if (tot > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tot);
+  } else {
+    const int64_t tot = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    if (tot > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tot);
+  }
+  p.nbuf = (2 * p.s * BN <= 512) ? 2 : 1;
+  p.stage_bytes = p.s * (A_TILE + B_TILE);
+  p.stages = std::min(4, (MAX_SMEM - 1024 - 256) / p.stage_bytes);
+  if (p.stages < 2) return PIQ_ERR_INVALID_ARG;
+  p.alpha = alpha;
+  p.beta = beta ? 1 : 0;
+  p.lower = lower ? 1 : 0;
+  p.C = C;
+  p.ldc = ldc;
+  p.ea = A.ex;
+  p.eb = B.ex;
+  p.st = st;
+  // at least half an SM's shared memory, so that two CTAs that each hold all
+  // 512 TMEM columns never share an SM
+  const int smem = std::max(p.stages * p.stage_bytes + 1024 + 256, 120 * 1024);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(ozaki_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             MAX_SMEM) != cudaSuccess)
+      return PIQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
+  note_launch();
+  if (launch_pdl(ozaki_gemm_kernel, dim3(grid), dim3(THREADS), static_cast<size_t>(smem), stream,
+                 ma, mb, p) != cudaSuccess)
+    return PIQ_ERR_CUDA;
+  return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
+}
+
+}  // namespace piq

@@ -161,6 +161,21 @@ __global__ void scale_upper_kernel(float* __restrict__ H, int64_t in, const floa
   }
 }
 
+// The same on an fp64 H (the upper triangle, rows from their diagonal on).
+__global__ void scale_upper64_kernel(double* __restrict__ H, int64_t in,
+                                     const float* __restrict__ s, DeviceStatus* st) {
+  for (int64_t k = blockIdx.y; k < in; k += gridDim.y) {
+    const float sk = s[k];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && !(sk > 0.f && sk <= 3.4028235e38f))
+      set_status(st, PIQ_ERR_INVALID_ARG, static_cast<int>(k));
+    const double rk = 1.0 / static_cast<double>(sk);
+    double* row = H + k * in;
+    for (int64_t j = k + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < in;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      row[j] = row[j] * rk / static_cast<double>(__ldg(s + j));
+  }
+}
+
 // sumsq[j] /= s_j^2 in FP64 (s_j^2 is exact there): diag of the scaled Hessian,
 // the act-order key of the scaled layer.
 __global__ void scale_sumsq_kernel(double* __restrict__ sumsq, int64_t in,
@@ -619,6 +634,16 @@ int launch_scale_upper(float* H, int64_t in, const float* s, DeviceStatus* st,
             static_cast<unsigned>(std::min<int64_t>(in, 65535)));
   note_launch();
   scale_upper_kernel<<<grid, 256, 0, stream>>>(H, in, s, st);
+  return last_error();
+}
+
+int launch_scale_upper(double* H, int64_t in, const float* s, DeviceStatus* st,
+                       cudaStream_t stream) {
+  if (s == nullptr) return PIQ_ERR_INVALID_ARG;
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(in, 256), 16)),
+            static_cast<unsigned>(std::min<int64_t>(in, 65535)));
+  note_launch();
+  scale_upper64_kernel<<<grid, 256, 0, stream>>>(H, in, s, st);
   return last_error();
 }
 

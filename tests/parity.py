@@ -1,17 +1,16 @@
 """GPU-vs-oracle comparison helpers (used by the gpu tests and smoke()).
 
-Contract: codes are decided identically except where the oracle's w/scale is
-within the tie window of a rounding tie, and such sites are at most 0.1% of the
-codes.  Because GPTQ feeds every rounding error forward, one tie flip changes
-the rest of its row, so the comparison is teacher-forced: the oracle is re-run
-on the affected rows with the GPU's code forced at the first mismatching site
-(which must be a tie), until the rows agree; the forced sites are the
-mismatches.  Scales and output errors then agree within 1e-3 relative.
+Contract (the benchmark spec's): at least 99.9% of the codes are
+identical to the oracle's before anything is forced, and every code decided
+differently lies where the oracle's w/scale is within 1e-4 of a rounding tie.
+Because GPTQ feeds every rounding error forward, one tie flip changes the rest
+of its row, so the comparison is teacher-forced: the oracle is re-run on the
+affected rows with the GPU's code forced at the first mismatching site (which
+must be a tie), until the rows agree; the forced sites are the codes decided
+differently.  Scales and output errors then agree within 1e-3 relative.
 
-The tie window is 1e-4, or twice the drift of the same loop run in float32 (the
-working precision of the GPU sweep and its block updates) when that is larger: over tens of
-thousands of columns float32 arithmetic alone moves w/scale by up to ~2e-4 from
-float64, so closer decisions are not fixed by the method at that precision.
+Large layers (2048 columns and more) are re-run with the oracle's blocked
+sweep, the same arithmetic as the literal loop (pinned by the oracle tests).
 """
 from __future__ import annotations
 
@@ -24,6 +23,7 @@ from oracle.gptq import NO_FORCE
 TIE_TOL = 1e-4
 MAX_MISMATCH_FRAC = 1e-3
 REL_TOL = 1e-3
+BLOCKED_FROM = 2048  # columns from which the forced re-runs use the blocked sweep
 
 
 def to_gpu_w(W: np.ndarray, device="cuda"):
@@ -43,7 +43,9 @@ def tie_distance(v: np.ndarray) -> np.ndarray:
 def fp32_drift(Wp: np.ndarray, U: np.ndarray, bits: int, g: int, ref) -> float:
     """Largest |w/scale| difference between the loop run in float32 and the
     float64 oracle ``ref`` on the same rows, up to each row's first differing
-    code (after it the two runs follow different codes)."""
+    code (after it the two runs follow different codes).  A diagnostic of what
+    FP32 arithmetic alone does to the loop; the contract's tie window does not
+    depend on it."""
     c32, _, v32, _ = O.gptq_sweep_ref(Wp, U, bits, g, dtype=np.float32)
     codes64, _, v64, _ = ref
     drift = 0.0
@@ -56,7 +58,14 @@ def fp32_drift(Wp: np.ndarray, U: np.ndarray, bits: int, g: int, ref) -> float:
 
 
 def _sweep(Wr, U, bits, g, asym, force=None, force_zero=None):
-    """(codes, scales, zeros, zv, v) of the oracle's literal loop."""
+    """(codes, scales, zeros, zv, v) of the oracle's loop (blocked for wide layers)."""
+    if Wr.shape[1] >= BLOCKED_FROM:
+        if asym:
+            c, s, z, v, zv = O.gptq_sweep_blocked_asym_ref(Wr, U, bits, g, force=force,
+                                                           force_zero=force_zero)
+            return c, s, z, zv, v
+        c, s, v = O.gptq_sweep_blocked_ref(Wr, U, bits, g, force=force)
+        return c, s, None, None, v
     if asym:
         c, s, z, zv, v, _ = O.gptq_sweep_asym_ref(Wr, U, bits, g, force=force,
                                                   force_zero=force_zero)
@@ -67,14 +76,19 @@ def _sweep(Wr, U, bits, g, asym, force=None, force_zero=None):
 
 def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray, bits: int,
                            g: int, ref=None, max_iters: int = 64, tie_tol: float = TIE_TOL,
-                           gpu_zeros: np.ndarray | None = None):
+                           gpu_zeros: np.ndarray | None = None, bound: str = "raw"):
     """gpu_codes (signed), Wp in quantization order.  Returns (stats, codes,
     scales) of the forced oracle run on all rows, plus its zero-points when
     ``gpu_zeros`` ([out, ngroups], asymmetric groups) is given; raises
-    AssertionError on a contract violation.  A zero-point is a rounded value
-    too (-lo / scale): where the GPU's differs, the oracle's unrounded value
-    must be within the tie window of a half-integer, and it is forced like a
-    code."""
+    AssertionError on a contract violation.  ``ref`` = (codes, scales, v) of
+    the oracle's unforced run, when the caller has it.  A zero-point is a
+    rounded value too (-lo / scale): where the GPU's differs, the oracle's
+    unrounded value must be within the tie window of a half-integer, and it is
+    forced like a code.
+
+    bound="raw": mismatches before forcing (codes and zero-points) at most 0.1%
+    of the codes; bound="forced": the forced sites at most 0.1% (for the FP32
+    step entry, whose rows may diverge after a legitimate tie flip)."""
     asym = gpu_zeros is not None
     if asym and ref is not None:
         raise ValueError("a precomputed ref carries no zero-points; pass ref=None")
@@ -88,8 +102,8 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
     zmism0 = (gpu_zeros != zeros0) if asym else np.zeros((Wp.shape[0], 1), dtype=bool)
     n0 = int(mism0.sum())
     total = gpu_codes.size
-    stats = {"mismatches": n0, "total": total, "frac": n0 / total, "forced": 0, "iters": 0,
-             "forced_zeros": 0}
+    stats = {"mismatches": n0, "zero_mismatches": int(zmism0.sum()), "total": total,
+             "frac": n0 / total, "forced": 0, "iters": 0, "forced_zeros": 0, "max_tie": 0.0}
     codes, scales = codes0.copy(), scales0.copy()
     zeros = zeros0.copy() if asym else None
     rows = np.unique(np.concatenate([np.nonzero(mism0)[0], np.nonzero(zmism0)[0]]))
@@ -117,6 +131,7 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
                         f"oracle {z[k, jz]} at -lo/scale = {zv[k, jz]!r} (tie distance {td:.3g})")
                     fz[k, jz] = gpu_zeros[rows[k], jz]
                     stats["forced_zeros"] += 1
+                    stats["max_tie"] = max(stats["max_tie"], td)
                     continue
                 td = float(tie_distance(v[k, j]))
                 assert td < tie_tol, (
@@ -124,10 +139,16 @@ def teacher_forced_compare(gpu_codes: np.ndarray, Wp: np.ndarray, U: np.ndarray,
                     f"{c[k, j]} at w/scale = {v[k, j]!r} (tie distance {td:.3g})")
                 force[k, j] = gpu_codes[rows[k], j]
                 stats["forced"] += 1
+                stats["max_tie"] = max(stats["max_tie"], td)
         else:
             raise AssertionError("teacher forcing did not converge")
-    assert stats["forced"] + stats["forced_zeros"] <= MAX_MISMATCH_FRAC * total, (
-        f"{stats['forced']} of {total} codes decided differently")
+    if bound == "raw":
+        assert n0 + stats["zero_mismatches"] <= MAX_MISMATCH_FRAC * total, (
+            f"{n0} of {total} codes (and {stats['zero_mismatches']} zero-points) differ before "
+            f"forcing ({stats['forced']} forced tie sites)")
+    else:
+        assert stats["forced"] + stats["forced_zeros"] <= MAX_MISMATCH_FRAC * total, (
+            f"{stats['forced']} of {total} codes decided differently")
     if asym:
         return stats, codes, scales, zeros
     return stats, codes, scales

@@ -122,5 +122,5 @@ def test_empty_and_oversized_layers_rejected(lib):
         rc = lib.awq_search_layer(fake, rows, inp, fake, n, 4, 32, grid, 2, None, fake, fake,
                                   fake, None, fake, 1 << 30, None)
         assert rc == piq.PIQ_ERR_INVALID_ARG, (rows, inp, n)
-    for args in ((0, 64, 64, 0), (16, 0, 64, 0), (16, 64, 0, 0)):
+    for args in ((0, 64, 64, 128, 0), (16, 0, 64, 128, 0), (16, 64, 0, 128, 0), (16, 64, 64, 0, 0)):
         assert lib.piq_gptq_workspace_bytes(*args, ctypes.byref(out)) == piq.PIQ_ERR_INVALID_ARG

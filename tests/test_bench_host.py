@@ -29,15 +29,14 @@ def test_reference_arm_line(monkeypatch, capsys):
     import json
     import numpy as np
     monkeypatch.setattr(bench, "make_inputs",
-                        lambda rank, n=None: (np.zeros((8, 8), np.float32),
-                                              np.zeros((4, 8), np.uint16),
-                                              np.zeros((4, 8), np.uint16)))
+                        lambda rank, n=None, workload="down_proj_70b": (
+                            np.zeros((8, 8), np.float32), np.zeros((4, 8), np.uint16), None))
     monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: (2.0, "stub sample"))
     assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference"
     assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
-    assert line["value"] == pytest.approx(4096 * 4096 / 2.0 / 1e6)
+    assert line["value"] == pytest.approx(8192 * 28672 / 2.0 / 1e6)  # the 70B down_proj layer
     assert line["higher_is_better"] is True and line["steps"] == 2 and line["warmup"] == 3
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["cpu_baseline"]["sample"] == "stub sample"
@@ -49,3 +48,19 @@ def test_reference_arm_line(monkeypatch, capsys):
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_phase_rooflines():
+    # q_proj 4096^2, 131072 samples; 1 ms per phase
+    ph = {k: 1.0 for k in ("hessian", "factor", "sweep", "pack", "error")}
+    r = bench.phase_rooflines(ph, 4096, 4096, 131072, 1600.0, 6500.0)
+    assert r["hessian"]["achieved"] == pytest.approx(131072 * 4096 * 4097 / 1e-3 / 1e12)
+    assert r["hessian"]["frac"] == pytest.approx(r["hessian"]["achieved"] / 1600.0)
+    # FP64-grade products: INT8 = 2 x bf16, 21 (factor) and 15 (sweep) digit products
+    assert r["factor"]["peak"] == pytest.approx(3200.0 / 21)
+    assert r["factor"]["achieved"] == pytest.approx(4096 ** 3 / 3 / 1e-3 / 1e12)
+    assert r["sweep"]["peak"] == pytest.approx(3200.0 / 15)
+    assert r["sweep"]["achieved"] == pytest.approx(4096 ** 3 / 1e-3 / 1e12)
+    assert r["pack"]["achieved"] == pytest.approx(4096 * 4096 * 9.5 / 1e-3 / 1e9)
+    assert r["pack"]["unit"] == "GB/s"
+    assert bench.phase_rooflines({}, 8, 8, 8, 1.0, 1.0) == {}

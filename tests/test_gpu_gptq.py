@@ -113,3 +113,53 @@ def test_shifted_inputs_error_entry():
     codes = unpack_gpu(out.qweight, 4)
     What = codes * np.repeat(out.scales.cpu().numpy().astype(np.float64), 128, axis=1)
     assert rel(e2, O.output_error_ref(W, What, X2)) < REL_TOL
+
+
+def test_clip_example_step_entry(golden):
+    # the hand-worked sweep where the clip binds at +qmax and -qmax-1, through
+    # the sweep step entry with the example's U
+    d = golden("sweep_clip_example.json")
+    U = torch.tensor(d["U"], dtype=torch.float32, device="cuda")
+    w = torch.tensor([d["w"]], dtype=torch.float32, device="cuda")
+    codes, qscale = piq.gptq_sweep(w, U, d["bits"], d["g"])
+    assert codes.cpu().numpy()[0].tolist() == d["codes"]
+    assert qscale.cpu().numpy()[0].tolist() == d["scales"]
+
+
+@pytest.mark.parametrize("bits,act", [(2, False), (3, True), (2, True)])
+def test_clip_binds(bits, act):
+    # at 2 and 3 bits the error feedback pushes many weights past the code
+    # range; the oracle clips them and the GPU must decide the same codes
+    spec = small_spec(96, 520, 2000, seed=40 + bits, sigma_ln=1.0, n_outlier=5,
+                      outlier_gain=30.0)
+    W, X = make_weight(spec), make_x_bits(spec)
+    Hx = O.hessian_ref(X)
+    perm, U, _ = O.gptq_prepare_ref(Hx, 0.01, act)
+    _, _, v, _ = O.gptq_sweep_ref(W.astype(np.float64)[:, perm], U, bits, 128)
+    qmax = 2 ** (bits - 1) - 1
+    assert (np.round(v) > qmax).sum() > 0 and (np.round(v) < -qmax - 1).sum() > 0
+    _check_layer(W, X, bits, 128, act)
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_dead_input_channel(act):
+    # an input channel that is zero in every sample: H_jj = 0 and its row and
+    # column vanish; damping keeps H_d positive definite (page 1, damping)
+    spec = small_spec(64, 264, 1000, seed=51, sigma_ln=0.8)
+    W, X = make_weight(spec), make_x_bits(spec).copy()
+    X[:, 17] = 0
+    X[:, 200] = 0
+    assert O.hessian_ref(X)[17, 17] == 0.0
+    _check_layer(W, X, 4, 128, act)
+
+
+def test_zero_weight_rows():
+    # an all-zero row and a row with an all-zero group: scale 0, codes 0
+    spec = small_spec(40, 384, 1200, seed=52, sigma_ln=0.8)
+    W, X = make_weight(spec).copy(), make_x_bits(spec)
+    W[5] = 0.0
+    W[9, 128:256] = 0.0
+    stats, out, _ = _check_layer(W, X, 4, 128, False)
+    codes = unpack_gpu(out.qweight, 4)
+    sc = out.scales.cpu().numpy()
+    assert (codes[5] == 0).all() and (sc[5] == 0).all()

@@ -51,9 +51,14 @@ def test_upper_factor_matches_oracle(inp, act):
     assert rel(lam, lam_x) < 1e-5
     assert np.count_nonzero(np.tril(U, -1)) == 0
     scale = np.abs(Ux).max(axis=1, keepdims=True)
-    assert (np.abs(U - Ux) / scale).max() < 2e-3
+    e_u = (np.abs(U - Ux) / scale).max()
     Hd, _ = O.damped_ref(Hx[np.ix_(perm, perm)], 0.01)
-    assert np.abs(U.T @ U @ Hd - np.eye(inp)).max() < 5e-3
+    e_inv = np.abs(U.T @ U @ Hd - np.eye(inp)).max()
+    print(f"upper factor in={inp} act={act}: max |dU|/rowmax {e_u:.3g}, |U^T U H_d - I| {e_inv:.3g}")
+    # an FP32 factorization (this step entry's precision): errors of a few
+    # units of float32 rounding times the conditioning of these layers
+    assert e_u < 2e-5
+    assert e_inv < 1e-4
 
 
 def test_not_positive_definite_reports_status():
@@ -73,8 +78,11 @@ def test_sweep_given_u(out, inp, g, bits):
     _, Ux, _ = O.gptq_prepare_ref(Hx, 0.01, False)
     U32 = np.ascontiguousarray(Ux, dtype=np.float32)
     codes, qscale = piq.gptq_sweep(to_gpu_w(W), torch.from_numpy(U32).cuda(), bits, g)
+    # the step entry runs the sweep in FP32: a tie flip may change the rest of
+    # its row, so the forced sites (not the raw differences) are bounded
     stats, c_ref, s_ref = teacher_forced_compare(codes.cpu().numpy(), W.astype(np.float64),
-                                                 U32.astype(np.float64), bits, g)
+                                                 U32.astype(np.float64), bits, g,
+                                                 bound="forced")
     qs = qscale.cpu().numpy().astype(np.float64)
     assert (np.abs(qs - s_ref) / np.maximum(s_ref, 1e-30)).max() < REL_TOL, stats
 

@@ -168,7 +168,7 @@ def test_asym_blocked_equals_literal(inp, g):
     perm, U, _ = O.gptq_prepare_ref(H, 0.01, False)
     Wp = W.astype(np.float64)
     c1, s1, z1, _, _, _ = gptq_sweep_asym_ref(Wp, U, 4, g)
-    c2, s2, z2, _ = gptq_sweep_blocked_asym_ref(Wp, U, 4, g)
+    c2, s2, z2, _, _ = gptq_sweep_blocked_asym_ref(Wp, U, 4, g)
     assert np.array_equal(c1, c2) and np.array_equal(z1, z2)
     assert np.allclose(s1, s2, rtol=1e-12, atol=0)
 

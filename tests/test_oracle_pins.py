@@ -77,6 +77,23 @@ def test_sweep_worked_example(golden):
     assert e[0].tolist() == d["err"]
 
 
+def test_sweep_clip_example(golden):
+    # both ends of the code range bind: an update pushes one code past qmax and
+    # another past -qmax-1
+    d = golden("sweep_clip_example.json")
+    U = np.array(d["U"], dtype=np.float64)
+    w = np.array([d["w"]], dtype=np.float64)
+    for sweep in (lambda: O.gptq_sweep_ref(w, U, d["bits"], d["g"]),
+                  lambda: O.gptq_sweep_ref(w, U, d["bits"], d["g"], dtype=np.float32)):
+        codes, scales, v, e = sweep()
+        assert codes[0].tolist() == d["codes"]
+        assert scales[0].tolist() == d["scales"]
+        assert v[0].tolist() == d["v"]
+        assert e[0].tolist() == d["err"]
+    codes, scales, v = O.gptq_sweep_blocked_ref(w, U, d["bits"], d["g"], block=4)
+    assert codes[0].tolist() == d["codes"] and v[0].tolist() == d["v"]
+
+
 def _random_layer(seed, out, inp, n, corr=0.6):
     rng = np.random.default_rng(seed)
     Z = rng.standard_normal((n, inp))

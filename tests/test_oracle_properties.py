@@ -65,7 +65,7 @@ def test_blocked_equals_literal(p):
         z1 = z2 = None
     else:
         c1, s1, z1, _, _, _ = gptq_sweep_asym_ref(Wp, U, bits, g)
-        c2, s2, z2, _ = gptq_sweep_blocked_asym_ref(Wp, U, bits, g, block=16)
+        c2, s2, z2, _, _ = gptq_sweep_blocked_asym_ref(Wp, U, bits, g, block=16)
     assert np.array_equal(c1, c2)
     assert np.allclose(s1, s2, rtol=1e-12, atol=0)
     if z1 is not None:

@@ -64,6 +64,23 @@ def test_calls_in_a_row_match_the_workspace_entry():
             _assert_close(U, first)  # the same input again, after a different size
 
 
+def test_matches_the_oracle():
+    # the same U the float64 oracle forms from the listing (cholesky(inv(H_d)).T),
+    # to the accuracy of the workspace entry's FP32 factorization
+    for inp, act, seed in ((512, False, 3), (264, True, 4)):
+        spec = small_spec(8, inp, 4 * inp, seed=seed, sigma_ln=0.8)
+        Hx = O.hessian_ref(make_x_bits(spec))
+        perm, Ux, lam_x = O.gptq_prepare_ref(Hx, 0.01, act)
+        H = torch.from_numpy(Hx.astype(np.float32)).cuda()
+        pg = torch.from_numpy(perm.astype(np.int32)).cuda() if act else None
+        rc, U, lam = _noalloc(H, 0.01, pg)
+        assert rc == piq.PIQ_OK, piq.status_string(rc)
+        U = U.cpu().numpy().astype(np.float64)
+        assert abs(lam - lam_x) <= 1e-5 * lam_x
+        assert np.count_nonzero(np.tril(U, -1)) == 0
+        assert (np.abs(U - Ux) / np.abs(Ux).max(axis=1, keepdims=True)).max() < 2e-5
+
+
 def test_larger_than_the_region_is_rejected():
     H = torch.zeros(piq.NOALLOC_MAX_IN + 8, piq.NOALLOC_MAX_IN + 8, device="cuda")
     rc, _, _ = _noalloc(H, 0.01, None)
