@@ -145,6 +145,43 @@ int gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t*
                         uint16_t* scales, int32_t* perm, int32_t* g_idx, double* out_err,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* One layer split over several GPUs, in two calls around one exchange.
+ * ("GPTQ versus AWQ objectives", sizing block under "A strong answer": H is an
+ * in x in FP32 sum over the calibration samples, and one layer at a time fits
+ * one GPU.  The sum splits over the samples; given H, the rows of W are
+ * independent problems: the listing's updates never mix rows.)
+ *
+ * piq_layer_statistics: the statistics of one shard of the calibration samples.
+ *   X      device bf16 [n, in] row-major (this shard's samples), read-only.
+ *   H      device fp64 [in, in] row-major: on and above the diagonal, X^T X of
+ *          this shard with FP64-grade sums (the same kernel as the layer call);
+ *          below it, unspecified.  Summing the shards' H (an all-reduce of
+ *          in * in doubles) gives the layer's H.
+ *   sumsq  device fp64 [in] or NULL: sum_n x_nj^2 in exact FP64 sums, the
+ *          act-order key; shards add up like H.
+ *   Workspace: piq_layer_statistics_workspace_bytes.  Synchronizes once.
+ *
+ * gptq_quantize_rows_from_h: GPTQ of some rows of W given the layer's H.
+ *   W      device fp32 [out, in]: these rows (any subset of the layer's rows).
+ *   H      device fp64 [in, in], read-only: the upper triangle of the layer's
+ *          X^T X (e.g. the all-reduced piq_layer_statistics outputs).
+ *   sumsq  device fp64 [in]: the act-order key; required when act_order != 0.
+ *   zeros  device uint8 [out, ceil(in/g)] or NULL: with it, a scale and a
+ *          zero-point per group as in gptq_quantize_layer_asym.
+ *   The other arguments and outputs are gptq_quantize_layer's, for these rows;
+ *   out_err is these rows' share of ||X W^T - X What^T||^2 (the shares add up
+ *   to the layer's).  Every rank computes the same damping, factor and perm.
+ *   Workspace: piq_gptq_from_h_workspace_bytes.  Synchronizes once. */
+int piq_layer_statistics_workspace_bytes(int64_t n, int64_t in, size_t* bytes);
+int piq_layer_statistics(const uint16_t* X, int64_t n, int64_t in, double* H, double* sumsq,
+                         void* workspace, size_t ws_bytes, void* stream);
+int piq_gptq_from_h_workspace_bytes(int64_t out, int64_t in, int g, size_t* bytes);
+int gptq_quantize_rows_from_h(const float* W, int64_t out, int64_t in, const double* H,
+                              const double* sumsq, int bits, int g, float damp, int act_order,
+                              uint32_t* qweight, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                              int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                              void* stream);
+
 /* GPTQ with a scale and a zero-point per group (the uplatz.com report, GPTQ's
  * key parameters, Group Size).  The pages give no formula; the quantizer is
  * min/max affine rounding of the group's current weights over a range widened

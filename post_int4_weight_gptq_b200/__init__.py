@@ -59,6 +59,13 @@ SIGNATURES = {
                                      _c_int, _vp, _vp, _vp, _vp,
                                      ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
                                      _vp]),
+    "piq_layer_statistics_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_size_p]),
+    "piq_layer_statistics": (_c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "piq_gptq_from_h_workspace_bytes": (_c_int, [_c_i64, _c_i64, _c_int, _c_size_p]),
+    "gptq_quantize_rows_from_h": (_c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _c_int, _c_int,
+                                           _c_float, _c_int, _vp, _vp, _vp, _vp, _vp,
+                                           ctypes.POINTER(ctypes.c_double), _vp,
+                                           ctypes.c_size_t, _vp]),
     "gptq_quantize_layer_asym": (_c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _c_int, _c_int,
                                           _c_float, _c_int, _vp, _vp, _vp, _vp, _vp,
                                           ctypes.POINTER(ctypes.c_double), _vp, ctypes.c_size_t,
@@ -257,6 +264,52 @@ def gptq_quantize_layer(W, X, bits=4, g=128, damp=0.01, act_order=False, with_er
                                           _ptr(out.g_idx), eptr, _ptr(ws), ws.numel(),
                                           _stream(stream))
         _check(rc, "gptq_quantize_layer_asym")
+    return out._replace(err=err.value if with_error else None)
+
+
+def layer_statistics(X, want_sumsq=True, stream=None, workspace=None):
+    """(H, sumsq) of one shard of calibration samples X [n, in] (bf16): H fp64
+    [in, in] (upper triangle = X^T X), sumsq fp64 [in] (the act-order key) or
+    None.  Shards add up: the layer's statistics are their sums."""
+    lib = load_library()
+    _need(X, torch.bfloat16, "X")
+    n, inp = X.shape
+    H = torch.empty(inp, inp, dtype=torch.float64, device=X.device)
+    sq = torch.empty(inp, dtype=torch.float64, device=X.device) if want_sumsq else None
+    ws = _workspace(_query(lib.piq_layer_statistics_workspace_bytes, n, inp), X.device, workspace)
+    _check(lib.piq_layer_statistics(_ptr(X), n, inp, _ptr(H), _ptr(sq), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "piq_layer_statistics")
+    return H, sq
+
+
+def gptq_rows_from_h(W, H, sumsq=None, bits=4, g=128, damp=0.01, act_order=False, sym=True,
+                     with_error=True, stream=None, workspace=None):
+    """GPTQ of the rows W [rows, in] (fp32) of a layer whose statistics H (fp64,
+    upper triangle of X^T X) and sumsq (fp64 act-order key) are given.  Returns
+    a GPTQOutput; err is these rows' share of the layer's output error."""
+    lib = load_library()
+    _need(W, torch.float32, "W")
+    _need(H, torch.float64, "H")
+    if sumsq is not None:
+        _need(sumsq, torch.float64, "sumsq")
+    rows, inp = W.shape
+    dev = W.device
+    ng = -(-inp // g)
+    out = GPTQOutput(torch.empty(rows, inp // 8, dtype=torch.int32, device=dev),
+                     torch.empty(rows, ng, dtype=torch.float16, device=dev),
+                     torch.empty(inp, dtype=torch.int32, device=dev),
+                     torch.empty(inp, dtype=torch.int32, device=dev), None,
+                     None if sym else torch.empty(rows, ng, dtype=torch.uint8, device=dev))
+    ws = _workspace(_query(lib.piq_gptq_from_h_workspace_bytes, rows, inp, int(g)), dev,
+                    workspace)
+    err = ctypes.c_double(0.0)
+    eptr = ctypes.byref(err) if with_error else None
+    rc = lib.gptq_quantize_rows_from_h(_ptr(W), rows, inp, _ptr(H), _ptr(sumsq), bits, g,
+                                       float(damp), int(bool(act_order)), _ptr(out.qweight),
+                                       _ptr(out.scales), _ptr(out.zeros), _ptr(out.perm),
+                                       _ptr(out.g_idx), eptr, _ptr(ws), ws.numel(),
+                                       _stream(stream))
+    _check(rc, "gptq_quantize_rows_from_h")
     return out._replace(err=err.value if with_error else None)
 
 

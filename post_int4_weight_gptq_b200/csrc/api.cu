@@ -188,9 +188,9 @@ SweepWs carve_sweep(Carver& c, int64_t out, int64_t in) {
   return w;
 }
 
-struct GptqWs {
+// Everything of a GPTQ call after H (and the act-order key) exist.
+struct FromHWs {
   DeviceStatus* st;
-  double* H;       // X^T X (fp64 sums), kept for the output error
   void* fwork;     // FP64 factor (L first); later the error's bf16 split of H
   float* Wq;       // W in quantization order (read by the sweep); later the bf16 split of D
   int8_t* codes;
@@ -198,16 +198,13 @@ struct GptqWs {
   float* dW;       // W - What (fp32, memory order)
   int32_t* perm;
   int32_t* invperm;
-  double* colpart;
-  double* sumsq;
   double* partials;
   double* err;
   Sweep64Ws sw;
 };
-GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int g, int act_order) {
-  GptqWs w;
+FromHWs carve_from_h(Carver& c, int64_t out, int64_t in, int g) {
+  FromHWs w;
   w.st = c.take<DeviceStatus>(1);
-  w.H = c.take<double>(in * in);
   w.fwork = c.take<uint8_t>(factor64_workspace_bytes(in));
   w.Wq = c.take<float>(out * in);
   w.codes = c.take<int8_t>(out * in);
@@ -215,12 +212,37 @@ GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int g, int act_
   w.dW = c.take<float>(out * in);
   w.perm = c.take<int32_t>(in);
   w.invperm = c.take<int32_t>(in);
-  w.colpart = c.take<double>(act_order ? static_cast<int64_t>(colstats_splits(n, in)) * in * 2 : 1);
-  w.sumsq = c.take<double>(in);
   w.partials = c.take<double>(err_via_h_partials(out, in));
   w.err = c.take<double>(1);
   uint8_t* sb = c.take<uint8_t>(sweep64_workspace_bytes(out, in, g));
   carve_sweep64(sb, out, in, g, &w.sw);
+  return w;
+}
+
+struct StatsWs {
+  double* colpart;
+};
+StatsWs carve_stats(Carver& c, int64_t n, int64_t in) {
+  StatsWs w;
+  w.colpart = c.take<double>(static_cast<int64_t>(colstats_splits(n, in)) * in * 2);
+  return w;
+}
+
+struct GptqWs {
+  double* H;       // X^T X (FP64-grade sums), kept for the output error
+  double* sumsq;   // act-order key
+  StatsWs stats;
+  FromHWs fh;
+};
+GptqWs carve_gptq(Carver& c, int64_t out, int64_t in, int64_t n, int g, int act_order) {
+  GptqWs w;
+  w.H = c.take<double>(in * in);
+  w.sumsq = c.take<double>(in);
+  if (act_order)
+    w.stats = carve_stats(c, n, in);
+  else
+    w.stats.colpart = c.take<double>(1);
+  w.fh = carve_from_h(c, out, in, g);
   return w;
 }
 
@@ -319,6 +341,55 @@ size_t gptq_ws_bytes(int64_t out, int64_t in, int64_t n, int g, int act_order) {
 // D' = W diag(s) - code * fp16(scale), since X' D'^T = X (W - What)^T.
 // With zeros, every group gets a scale and a zero-point (asymmetric groups):
 // the sweep writes the zero-points there and the pack stores code + zero.
+// Steps 2-6 of GPTQ from a given H (upper triangle, fp64) and, for act-order,
+// its key sumsq (diag(H) in exact FP64 sums).  H is read only, except that
+// with s_ch it was scaled in place by the caller.
+int gptq_core(const float* W, int64_t out, int64_t in, const double* H, const double* sumsq,
+              const float* s_ch, int bits, int g, float damp, int act_order, uint32_t* qweight,
+              uint16_t* scales, uint8_t* zeros, int32_t* perm, int32_t* g_idx, double* out_err,
+              const FromHWs& w, PhaseClock& clk, cudaStream_t s) {
+  // 2. quantization order
+  const int32_t* qperm = nullptr;
+  const int32_t* qinv = nullptr;
+  if (act_order) {
+    PIQ_TRY(launch_act_order_perm(sumsq, in, w.perm, w.invperm, s));
+    qperm = w.perm;
+    qinv = w.invperm;
+  }
+  if (perm) {
+    if (act_order)
+      PIQ_TRY(cuda_rc(cudaMemcpyAsync(perm, w.perm, sizeof(int32_t) * in, cudaMemcpyDeviceToDevice, s)));
+    else
+      PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
+  }
+  clk.mark();
+  // 3. damping + the FP64 factor L of J H_d J (H is kept for the error)
+  double* L = nullptr;
+  PIQ_TRY(run_factor64(H, in, damp, qperm, w.fwork, &L, w.st, s));
+  clk.mark();
+  // 4. the sweep on R = J L J over the permuted (and scaled) copy of W
+  PIQ_TRY(launch_gather_columns(W, out, in, qperm, s_ch, w.Wq, s));
+  PIQ_TRY(run_gptq_sweep64(w.Wq, out, in, L, bits, g, w.codes, w.qscale, zeros, w.sw, w.st, s));
+  clk.mark();
+  // 5. pack (+ D = W diag(s) - What' for the error)
+  PIQ_TRY(launch_pack(w.codes, w.qscale, zeros, qinv, out, in, bits, g, W, s_ch, qweight, scales,
+                      nullptr, out_err ? w.dW : nullptr, g_idx, s));
+  clk.mark();
+  // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from H
+  //    (scratch: the sweep copy, and the factor's region)
+  if (out_err)
+    PIQ_TRY(run_error_via_h(w.dW, out, in, H, reinterpret_cast<uint16_t*>(w.Wq),
+                            reinterpret_cast<uint16_t*>(w.fwork), w.partials, w.err, w.st, s));
+  clk.mark();
+  double e = 0.0;
+  if (out_err)
+    PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
+  const int rc = finish_call(w.st, s, nullptr);
+  clk.finish();
+  if (out_err) *out_err = e;
+  return rc;
+}
+
 int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64_t n,
                const float* s_ch, int bits, int g, float damp, int act_order, uint32_t* qweight,
                uint16_t* scales, uint8_t* zeros, int32_t* perm, int32_t* g_idx, double* out_err,
@@ -335,53 +406,19 @@ int gptq_layer(const float* W, int64_t out, int64_t in, const uint16_t* X, int64
   GptqWs w = carve_gptq(c, out, in, n, g, act_order ? 1 : 0);
   PhaseClock clk(0, s);
 
-  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
-  // 1. H = X^T X on the tensor cores (scaled to H' for the AWQ-scaled layer)
-  PIQ_TRY(launch_syrk64(X, n, in, w.H, w.st, s));
-  if (s_ch) PIQ_TRY(launch_scale_upper(w.H, in, s_ch, w.st, s));
-  clk.mark();
-  // 2. quantization order
-  const int32_t* qperm = nullptr;
-  const int32_t* qinv = nullptr;
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.fh.st, 0, sizeof(DeviceStatus), s)));
+  // 1. H = X^T X on the tensor cores (scaled to H' for the AWQ-scaled layer), and
+  //    the act-order key: exact FP64 column sums of squares (scaled alike)
+  PIQ_TRY(launch_syrk64(X, n, in, w.H, w.fh.st, s));
+  if (s_ch) PIQ_TRY(launch_scale_upper(w.H, in, s_ch, w.fh.st, s));
   if (act_order) {
-    PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), nullptr, w.sumsq, s));
+    PIQ_TRY(launch_colstats(X, n, in, w.stats.colpart, colstats_splits(n, in), nullptr, w.sumsq,
+                            s));
     if (s_ch) PIQ_TRY(launch_scale_sumsq(w.sumsq, in, s_ch, s));
-    PIQ_TRY(launch_act_order_perm(w.sumsq, in, w.perm, w.invperm, s));
-    qperm = w.perm;
-    qinv = w.invperm;
-  }
-  if (perm) {
-    if (act_order)
-      PIQ_TRY(cuda_rc(cudaMemcpyAsync(perm, w.perm, sizeof(int32_t) * in, cudaMemcpyDeviceToDevice, s)));
-    else
-      PIQ_TRY(launch_identity_perm(in, perm, nullptr, s));
   }
   clk.mark();
-  // 3. damping + the FP64 factor L of J H_d J (H is kept for the error)
-  double* L = nullptr;
-  PIQ_TRY(run_factor64(w.H, in, damp, qperm, w.fwork, &L, w.st, s));
-  clk.mark();
-  // 4. the sweep on R = J L J over the permuted (and scaled) copy of W
-  PIQ_TRY(launch_gather_columns(W, out, in, qperm, s_ch, w.Wq, s));
-  PIQ_TRY(run_gptq_sweep64(w.Wq, out, in, L, bits, g, w.codes, w.qscale, zeros, w.sw, w.st, s));
-  clk.mark();
-  // 5. pack (+ D = W diag(s) - What' for the error)
-  PIQ_TRY(launch_pack(w.codes, w.qscale, zeros, qinv, out, in, bits, g, W, s_ch, qweight, scales,
-                      nullptr, out_err ? w.dW : nullptr, g_idx, s));
-  clk.mark();
-  // 6. output error ||X D^T||^2 = 2 sum_r D_r Hu D_r^T, from the H built in step 1
-  //    (scratch: the sweep copy, and the factor's inverse region after U)
-  if (out_err)
-    PIQ_TRY(run_error_via_h(w.dW, out, in, w.H, reinterpret_cast<uint16_t*>(w.Wq),
-                            reinterpret_cast<uint16_t*>(w.fwork), w.partials, w.err, w.st, s));
-  clk.mark();
-  double e = 0.0;
-  if (out_err)
-    PIQ_TRY(cuda_rc(cudaMemcpyAsync(&e, w.err, sizeof(double), cudaMemcpyDeviceToHost, s)));
-  const int rc = finish_call(w.st, s, nullptr);
-  clk.finish();
-  if (out_err) *out_err = e;
-  return rc;
+  return gptq_core(W, out, in, w.H, w.sumsq, s_ch, bits, g, damp, act_order, qweight, scales,
+                   zeros, perm, g_idx, out_err, w.fh, clk, s);
 }
 
 }  // namespace
@@ -500,6 +537,70 @@ int gptq_quantize_layer_asym(const float* W, int64_t out, int64_t in, const uint
   if (zeros == nullptr) return PIQ_ERR_INVALID_ARG;
   return gptq_layer(W, out, in, X, n, nullptr, bits, g, damp, act_order, qweight, scales, zeros,
                     perm, g_idx, out_err, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int piq_layer_statistics_workspace_bytes(int64_t n, int64_t in, size_t* bytes) {
+  if (bytes == nullptr || n < 1 || in < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  c.take<DeviceStatus>(1);
+  carve_stats(c, n, in);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int piq_layer_statistics(const uint16_t* X, int64_t n, int64_t in, double* H, double* sumsq,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  if (X == nullptr || H == nullptr || n < 1 || in < 8 || in % 8 != 0 || !aligned16(X) ||
+      !aligned16(H) || in > (int64_t)1 << 20)
+    return PIQ_ERR_INVALID_ARG;
+  PIQ_TRY(injected_fault());
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_layer_statistics_workspace_bytes(n, in, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  DeviceStatus* st = c.take<DeviceStatus>(1);
+  StatsWs w = carve_stats(c, n, in);
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(st, 0, sizeof(DeviceStatus), s)));
+  PIQ_TRY(launch_syrk64(X, n, in, H, st, s));
+  if (sumsq) PIQ_TRY(launch_colstats(X, n, in, w.colpart, colstats_splits(n, in), nullptr, sumsq, s));
+  return finish_call(st, s, nullptr);
+}
+
+int piq_gptq_from_h_workspace_bytes(int64_t out, int64_t in, int g, size_t* bytes) {
+  if (bytes == nullptr || out < 1 || in < 1 || g < 1) return PIQ_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_from_h(c, out, in, g);
+  *bytes = c.bytes();
+  return PIQ_OK;
+}
+
+int gptq_quantize_rows_from_h(const float* W, int64_t out, int64_t in, const double* H,
+                              const double* sumsq, int bits, int g, float damp, int act_order,
+                              uint32_t* qweight, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                              int32_t* g_idx, double* out_err, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  PIQ_TRY(check_layer(out, in, bits, g));
+  if (W == nullptr || H == nullptr || qweight == nullptr || scales == nullptr ||
+      !(damp >= 0.f) || !aligned16(W) || !aligned16(H) || !aligned16(qweight) ||
+      (act_order && sumsq == nullptr))
+    return PIQ_ERR_INVALID_ARG;
+  PIQ_TRY(injected_fault());
+  DeviceInfo info;
+  PIQ_TRY(device_info(&info));
+  size_t need = 0;
+  piq_gptq_from_h_workspace_bytes(out, in, g, &need);
+  PIQ_TRY(check_ws(workspace, ws_bytes, need));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  FromHWs w = carve_from_h(c, out, in, g);
+  PhaseClock clk(0, s);
+  PIQ_TRY(cuda_rc(cudaMemsetAsync(w.st, 0, sizeof(DeviceStatus), s)));
+  clk.mark();  // no H phase: H is given
+  return gptq_core(W, out, in, H, sumsq, nullptr, bits, g, damp, act_order, qweight, scales,
+                   zeros, perm, g_idx, out_err, w, clk, s);
 }
 
 int awq_gptq_quantize_layer(const float* W, int64_t out, int64_t in, const uint16_t* X,

@@ -18,7 +18,8 @@
 //      factored and inverted in FP64 on one SM (chol64_block_kernel); the panel
 //      below is L21 = A21 inv(L11)^T and the trailing matrix A22 -= L21 L21^T,
 //      both on the INT8 tensor cores with FP64 accumulation (ozaki.cu)
-//   3. inverses of R's diagonal blocks for the sweep (block_inverse_kernel)
+//   3. L mirrored into the upper triangle (column n of L as row n), and the
+//      inverses of R's diagonal blocks for the sweep (block_inverse_kernel)
 // A non-positive pivot sets PIQ_ERR_NOT_PD.
 #include <algorithm>
 
@@ -78,17 +79,35 @@ __global__ void build_rev64_kernel(const double* H, int64_t in, const int32_t* p
 // Factor the nb x nb diagonal block of P at (o, o) in place (lower Cholesky,
 // FP64) and write its inverse to X11 (128 x 128, row-major, zeros above the
 // diagonal and outside nb).  Rows/cols >= nb are padded with the identity.
-// Pivot by pivot: the pivot's square root, the column scaled, then the
-// trailing lower triangle updated by all threads.  The inverse is formed one
-// column per thread by forward substitution, kept transposed in the strictly
-// upper part of the same shared array (the factor occupies the lower part).
+//
+// Right-looking over 16-wide sub-panels: warp 0 factors the 16 x 16 diagonal
+// block in registers (lane i holds row i; each pivot's column reaches the
+// lanes by shuffles); one thread per row below solves that row against it by
+// substitution; the trailing lower triangle gets the rank-16 update in 4 x 4
+// register tiles.  The inverse follows in the same 16-row blocks: for block
+// R, T = L[R, <R] X[<R, :] (register tiles over all threads), then each
+// column's 16 entries by substitution against L[R, R].  Factor and inverse
+// share one shared array: the factor in the lower triangle, the inverse
+// transposed in the strictly upper one, its diagonal apart.
+constexpr int SP16 = 16;
+
+__device__ __forceinline__ void fma4x4d(double (&acc)[4][4], const double (&a)[4],
+                                        const double (&b)[4]) {
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = fma(a[x], b[y], acc[x][y]);
+}
+
 __global__ void __launch_bounds__(CT)
     chol64_block_kernel(double* P, int64_t ld, int64_t o, int nb, double* X11,
                         DeviceStatus* st) {
-  extern __shared__ __align__(16) double S[];  // [NB][LDS]
-  __shared__ double xd[NB];                    // diagonal of the inverse
+  extern __shared__ __align__(16) double sm64[];
+  double* S = sm64;               // [NB][LDS] factor (lower), inverse (upper, transposed)
+  __shared__ double rdiag[NB];    // 1 / L_ii
+  __shared__ double xd[NB];       // diagonal of the inverse
   __shared__ int bad;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
   pdl_wait();
   if (status_bad(st)) return;
@@ -101,54 +120,141 @@ __global__ void __launch_bounds__(CT)
     S[i * LDS + j] = v;
   }
   __syncthreads();
-  for (int j = 0; j < NB; ++j) {
-    const double d = S[j * LDS + j];
-    if (!(d > 0.0)) {  // uniform: every thread reads the same value
-      if (tid == 0) {
+
+  for (int c0 = 0; c0 < NB; c0 += SP16) {
+    // ---- the 16 x 16 diagonal block, warp 0
+    if (warp == 0) {
+      double a[SP16];
+#pragma unroll
+      for (int k = 0; k < SP16; ++k)
+        a[k] = (lane < SP16 && k <= lane) ? S[(c0 + lane) * LDS + c0 + k] : 0.0;
+      bool ok = true;
+#pragma unroll
+      for (int J = 0; J < SP16; ++J) {
+        const double d = __shfl_sync(0xffffffffu, a[J], J);
+        ok = ok && (d > 0.0);
+        const double ljj = sqrt(d > 0.0 ? d : 1.0);
+        const double r = 1.0 / ljj;
+        if (lane == J) {
+          a[J] = ljj;
+          rdiag[c0 + J] = r;
+        } else if (lane > J) {
+          a[J] *= r;
+        }
+        // a[k] -= L[i][J] L[k][J] for J < k <= i
+#pragma unroll
+        for (int k = J + 1; k < SP16; ++k) {
+          const double lk = __shfl_sync(0xffffffffu, a[J], k);
+          if (lane >= k) a[k] = fma(-a[J], lk, a[k]);
+        }
+      }
+      if (!ok && lane == 0) {
         bad = 1;
-        set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + j));
+        set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));
       }
-      break;
+      if (lane < SP16) {
+#pragma unroll
+        for (int k = 0; k < SP16; ++k)
+          if (k <= lane) S[(c0 + lane) * LDS + c0 + k] = a[k];
+      }
     }
-    const double ljj = sqrt(d);
-    const double r = 1.0 / ljj;
-    __syncthreads();  // everyone has read S[j][j]
-    if (tid == 0) S[j * LDS + j] = ljj;
-    for (int i = j + 1 + tid; i < NB; i += CT) S[i * LDS + j] *= r;
     __syncthreads();
-    // A22 -= l l^T on the lower triangle below pivot j: pairs (i, k), j < k <= i
-    const int m = NB - 1 - j;
-    const int npairs = m * (m + 1) / 2;
-    for (int t = tid; t < npairs; t += CT) {
-      // t -> (ii, kk) with 0 <= kk <= ii < m, row-major over the triangle
-      int ii = static_cast<int>((sqrt(8.0 * t + 1.0) - 1.0) * 0.5);
-      while ((ii + 1) * (ii + 2) / 2 <= t) ++ii;
-      while (ii * (ii + 1) / 2 > t) --ii;
-      const int kk = t - ii * (ii + 1) / 2;
-      const int i = j + 1 + ii, k = j + 1 + kk;
-      S[i * LDS + k] = fma(-S[i * LDS + j], S[k * LDS + j], S[i * LDS + k]);
+    if (bad) return;
+    const int r0 = c0 + SP16;
+    if (r0 >= NB) break;
+    // ---- rows below: y = A21 row solved against L11 (L21 = A21 inv(L11)^T)
+    for (int r = r0 + tid; r < NB; r += CT) {
+      double y[SP16];
+#pragma unroll
+      for (int k = 0; k < SP16; ++k) y[k] = S[r * LDS + c0 + k];
+#pragma unroll
+      for (int C = 0; C < SP16; ++C) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) y[C] = fma(-y[c], S[(c0 + C) * LDS + c0 + c], y[C]);
+        y[C] *= rdiag[c0 + C];
+      }
+#pragma unroll
+      for (int k = 0; k < SP16; ++k) S[r * LDS + c0 + k] = y[k];
+    }
+    __syncthreads();
+    // ---- A22 -= L21 L21^T on the lower 4 x 4 tiles
+    {
+      const int mt = (NB - r0) / 4;
+      const int ntile = mt * (mt + 1) / 2;
+      for (int t = tid; t < ntile; t += CT) {
+        int bi = static_cast<int>((sqrtf(8.f * static_cast<float>(t) + 1.f) - 1.f) * 0.5f);
+        while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
+        while (bi * (bi + 1) / 2 > t) --bi;
+        const int bj = t - bi * (bi + 1) / 2;
+        const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
+        double acc[4][4] = {};
+#pragma unroll
+        for (int k = 0; k < SP16; ++k) {
+          double av[4], bv[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            av[x] = S[(i0 + x) * LDS + c0 + k];
+            bv[x] = S[(j0 + x) * LDS + c0 + k];
+          }
+          fma4x4d(acc, av, bv);
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            if (j0 + y <= i0 + x) S[(i0 + x) * LDS + j0 + y] -= acc[x][y];
+      }
     }
     __syncthreads();
   }
-  __syncthreads();
-  if (bad) return;
-  // inverse: column c by forward substitution, X[i][c] stored at S[c][i] (i > c)
-  if (tid < NB) {
-    const int c = tid;
-    const double xcc = 1.0 / S[c * LDS + c];
-    xd[c] = xcc;
-    for (int i = c + 1; i < NB; ++i) {
-      double acc0 = S[i * LDS + c] * xcc, acc1 = 0.0;
-      int k = c + 1;
-      for (; k + 1 < i; k += 2) {
-        acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
-        acc1 = fma(S[i * LDS + k + 1], S[c * LDS + k + 1], acc1);
+
+  // ---- inverse X = inv(L), 16 rows at a time: X[R, :] = inv(L_RR) (E_R - L[R, <R] X[<R, :]).
+  // X[i][j] (i > j) is kept at S[j][i] (the strictly upper part, free), X[i][i] in xd.
+  for (int c0 = 0; c0 < NB; c0 += SP16) {
+    // -L[R, <R] X[<R, 0:c0] on the 16 x c0 block (4 x 4 tiles), kept as X[R][0:c0]
+    if (c0 > 0) {
+      const int ntile = (SP16 / 4) * (c0 / 4);
+      for (int t = tid; t < ntile; t += CT) {
+        const int bi = t / (c0 / 4), bj = t - bi * (c0 / 4);
+        const int i0 = c0 + 4 * bi, j0 = 4 * bj;
+        double acc[4][4] = {};
+        for (int k = j0; k < c0; ++k) {  // X[k][j] = 0 for k < j
+          double av[4], bv[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            av[x] = S[(i0 + x) * LDS + k];
+            const int j = j0 + x;
+            bv[x] = k > j ? S[j * LDS + k] : (k == j ? xd[j] : 0.0);
+          }
+          fma4x4d(acc, av, bv);
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) S[(j0 + y) * LDS + i0 + x] = -acc[x][y];
       }
-      if (k < i) acc0 = fma(S[i * LDS + k], S[c * LDS + k], acc0);
-      S[c * LDS + i] = -(acc0 + acc1) / S[i * LDS + i];
+      __syncthreads();
     }
+    // substitution against L_RR, one thread per column j <= c0 + 15
+    for (int j = tid; j < c0 + SP16; j += CT) {
+      double x[SP16];
+#pragma unroll
+      for (int i = 0; i < SP16; ++i) {
+        double v = (j < c0) ? S[j * LDS + c0 + i] : (j == c0 + i ? 1.0 : 0.0);
+#pragma unroll
+        for (int k = 0; k < i; ++k) v = fma(-S[(c0 + i) * LDS + c0 + k], x[k], v);
+        x[i] = v * rdiag[c0 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < SP16; ++i) {
+        const int r = c0 + i;
+        if (r > j) S[j * LDS + r] = x[i];
+        else if (r == j) xd[j] = x[i];
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
+
   for (int idx = tid; idx < NB * NB; idx += CT) {
     const int i = idx >> 7, j = idx & (NB - 1);
     if (i < nb && j <= i) P[(o + i) * ld + (o + j)] = S[i * LDS + j];
@@ -209,7 +315,31 @@ __global__ void __launch_bounds__(NB)
   }
 }
 
+// Mirror the lower triangle of L into the (unused) upper triangle of the same
+// array: P[i][j] = L[j][i] for j > i, so that row n of the upper part holds
+// column n of L contiguously (the sweep reads R's block rows, i.e. columns of
+// L, through it).  32 x 32 tiles through shared memory; reads touch only the
+// lower triangle, writes only the strictly upper one.
+__global__ void mirror_lower_kernel(double* P, int64_t in) {
+  __shared__ double t[32][33];
+  const int64_t bi = blockIdx.y, bj = blockIdx.x;  // destination tile (bi, bj), bi <= bj
+  if (bj < bi) return;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int r = ty; r < 32; r += blockDim.y) {  // source tile (bj, bi): rows of L
+    const int64_t i = bj * 32 + r, j = bi * 32 + tx;
+    t[r][tx] = (i < in && j < in && j <= i) ? P[i * in + j] : 0.0;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += blockDim.y) {
+    const int64_t i = bi * 32 + r, j = bj * 32 + tx;  // destination P[i][j] = L[j][i]
+    if (i < in && j < in && j > i) P[i * in + j] = t[tx][r];
+  }
+}
+
 constexpr int kBlockSmem = NB * LDS * 8;
+constexpr int kCholSmem64 = NB * LDS * 8;
 
 }  // namespace
 
@@ -271,7 +401,7 @@ int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, v
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   if (dev < 64 && !attr_set[dev]) {
     if (cudaFuncSetAttribute(chol64_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kBlockSmem) != cudaSuccess ||
+                             kCholSmem64) != cudaSuccess ||
         cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kBlockSmem) != cudaSuccess)
       return PIQ_ERR_CUDA;
@@ -291,7 +421,7 @@ int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, v
     for (int64_t k0 = s0; k0 < s1; k0 += NB) {
       const int nb = static_cast<int>(std::min<int64_t>(NB, in - k0));
       note_launch();
-      if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kBlockSmem, stream, P, ld, k0, nb,
+      if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kCholSmem64, stream, P, ld, k0, nb,
                      X11, st) != cudaSuccess)
         return PIQ_ERR_CUDA;
       const int64_t rem = in - k0 - nb;
@@ -324,6 +454,13 @@ int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, v
         rc = launch_ozaki_gemm(rest, rest, dS, dS, -1.0, 1, 1, P + s1 * ld + s1, ld, st, stream);
       if (rc != PIQ_OK) return rc;
     }
+  }
+  {
+    const unsigned nt = static_cast<unsigned>(ceil_div(in, 32));
+    note_launch();
+    if (launch_pdl(mirror_lower_kernel, dim3(nt, nt), dim3(32, 8), 0, stream, P, in) !=
+        cudaSuccess)
+      return PIQ_ERR_CUDA;
   }
   *L_out = P;
   return PIQ_OK;

@@ -261,12 +261,31 @@ __global__ void __launch_bounds__(THREADS, 1)
           double* crow = p.C + static_cast<int64_t>(row) * p.ldc + col0;
           const int lim = min(32, p.N - col0);
           const int clim = p.lower ? min(lim, row - col0 + 1) : lim;  // c <= r
+          // v * alpha * 2^(ea + eb - 12): the power of two built from its
+          // exponent field (the row exponents stay far inside the normal range)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (i < clim) {
-              const double sc = ldexp(p.alpha, ear + __ldg(p.eb + col0 + i) - 12);
-              const double val = v[i] * sc;
-              crow[i] = p.beta ? crow[i] + val : val;
+            const int eb = i < clim ? __ldg(p.eb + col0 + i) : 0;
+            v[i] *= __longlong_as_double(static_cast<long long>(1023 + ear + eb - 12) << 52);
+          }
+          if (clim == 32 && (reinterpret_cast<uintptr_t>(crow) & 15u) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              double2 o = make_double2(p.alpha * v[i], p.alpha * v[i + 1]);
+              if (p.beta) {
+                const double2 old = *reinterpret_cast<const double2*>(crow + i);
+                o.x += old.x;
+                o.y += old.y;
+              }
+              *reinterpret_cast<double2*>(crow + i) = o;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < clim) {
+                const double val = p.alpha * v[i];
+                crow[i] = p.beta ? crow[i] + val : val;
+              }
             }
           }
         }
@@ -303,6 +322,8 @@ __global__ void slice_rows_kernel(const double* __restrict__ src, int64_t rs, in
   int e = 0;
   if (m > 0.0) frexp(m, &e);  // m = f 2^e with f in [0.5, 1)
   if (lane == 0) ex[r] = e;
+  // 2^(6 - e) from its exponent field (row maxima stay far inside the normal range)
+  const double sc6 = __longlong_as_double(static_cast<long long>(1023 + 6 - e) << 52);
   const int64_t plane = rows * kpad;
   // four consecutive k per lane per step: one 32-bit store per digit
   for (int64_t k0 = 4 * lane; k0 < kpad; k0 += 128) {
@@ -310,7 +331,7 @@ __global__ void slice_rows_kernel(const double* __restrict__ src, int64_t rs, in
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const int64_t k = k0 + t;
-      double y = (k < K && m > 0.0) ? ldexp(row[k * ks], 6 - e) : 0.0;  // |y| < 64
+      double y = (k < K && m > 0.0) ? row[k * ks] * sc6 : 0.0;  // |y| < 64
       for (int i = 0; i < s; ++i) {
         const double di = rint(y);
         y = (y - di) * 128.0;

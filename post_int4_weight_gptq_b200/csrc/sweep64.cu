@@ -47,11 +47,30 @@ constexpr int RS = 64;       // rows per CTA
 constexpr int SUB = 32;      // columns per register window
 constexpr int THREADS = 256;
 constexpr int LDW = B + 1;   // fp64 row-state stride
-constexpr int kSmem = B * B * 8 + RS * LDW * 8 + 64;
+constexpr int kSmem = B * B * 8 + RS * LDW * 8 + B * 8 + 64;
+constexpr int kSmemQ = B * B * 8 + RS * LDW * 8 + B * 8 + 6 * 64 * 8 + 64 * 128;
 constexpr int64_t kSuperBlock = 1024;  // columns per superblock of the block updates
 
+// rint(w / scale) for the IEEE quotient, from w * (1 / scale): the product is
+// within a few units in the last place of the quotient, so it can only round
+// differently within ~1e-12 |w / scale| of a half-integer, where the division
+// itself decides (rare, out of line).
+__device__ __noinline__ double code64_by_division(double w, double scale) {
+  return rint(w / scale);
+}
+__device__ __forceinline__ double code64(double w, double scale, double rscale) {
+  const double t = w * rscale;
+  const double q = rint(t);
+  return fabs(fabs(t - q) - 0.5) < 1e-12 * fmax(1.0, fabs(t)) ? code64_by_division(w, scale) : q;
+}
+
+// 2^e for |e| well inside the normal range, from the exponent field.
+__device__ __forceinline__ double pow2(int e) {
+  return __longlong_as_double(static_cast<long long>(1023 + e) << 52);
+}
+
 struct Row64 {
-  double scale, cmin, cmax, fqmax;
+  double scale, rscale, cmin, cmax, fqmax;
   int64_t next_gs, b, in, g, ngroups, row;
   int kb;
   bool valid;
@@ -72,6 +91,7 @@ __device__ __forceinline__ void set_group(double m, double mn, bool asym, Row64&
     st.cmax = st.fqmax - z;
     if (st.valid) qzero[st.row * st.ngroups + grp] = static_cast<uint8_t>(z);
   }
+  st.rscale = st.scale > 0.0 ? 1.0 / st.scale : 0.0;
   if (st.valid) qscale[st.row * st.ngroups + grp] = static_cast<float>(st.scale);
 }
 
@@ -85,6 +105,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(16) double smem64[];
   double* Us = smem64;             // [B][B] U_GG
   double* Wr = Us + B * B;         // [RS][LDW] row state, then W0 - Q of used columns
+  double* inv_u = Wr + RS * LDW;   // [B] 1 / U_jj
   const int tid = threadIdx.x;
   pdl_launch_dependents();
   pdl_wait();
@@ -92,6 +113,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * RS;
   const int rows_here = static_cast<int>(std::min<int64_t>(RS, out - row0));
   for (int idx = tid; idx < B * B; idx += THREADS) Us[idx] = Ub[idx];
+  for (int j = tid; j < B; j += THREADS) inv_u[j] = j < kb ? 1.0 / Ub[j * B + j] : 0.0;
   for (int idx = tid; idx < RS * B; idx += THREADS) {
     const int r = idx >> 7, c = idx & (B - 1);
     Wr[r * LDW + c] = (r < rows_here && c < kb) ? acc[(row0 + r) * in + b + c] : 0.0;
@@ -163,6 +185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
       rs.next_gs = 0;
     }
+    rs.rscale = rs.scale > 0.0 ? 1.0 / rs.scale : 0.0;
     double* wrow = Wr + tid * LDW;
     const float* w0row = W0 + rs.row * in + b;
     int8_t* crow = codes + rs.row * in + b;
@@ -200,8 +223,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           const double wj = ws[jj];
           const double sc = rs.scale;
-          const double qv = sc > 0.0 ? fmin(fmax(rint(wj / sc), rs.cmin), rs.cmax) : 0.0;
-          const double err = (wj - qv * sc) / Us[j * B + j];
+          const double qv = sc > 0.0 ? fmin(fmax(code64(wj, sc, rs.rscale), rs.cmin), rs.cmax)
+                                     : 0.0;
+          const double err = (wj - qv * sc) * inv_u[j];
           e[jj] = err;
           if (rs.valid) crow[j] = static_cast<int8_t>(qv);
           // W0 - Q of this column replaces its slot in the row state
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int c = c4 + t;
-          double y = (c < kb && m > 0.0) ? ldexp(wrow[c], 6 - ex) : 0.0;
+          double y = (c < kb && m > 0.0) ? wrow[c] * pow2(6 - ex) : 0.0;
           for (int i = 0; i < ds; ++i) {
             const double di = rint(y);
             y = (y - di) * 128.0;
@@ -247,6 +271,205 @@ __global__ void __launch_bounds__(THREADS, 1)
           *reinterpret_cast<uint32_t*>(dq + i * plane + rs.row * dkpad + c4) = w[i];
       }
     }
+  }
+}
+
+// The same block for g % 128 == 0 (no group starts inside the block except at
+// its first column): 8 warps, warp w owns rows 32 (w % 2) .. + 31 of the CTA
+// (one per lane) and window q = w / 2 (block columns 32 q .. 32 q + 31) in
+// registers.  Phase p (0..3): the window-p threads apply window p-1's errors
+// to their window and run its serial column loop; the threads of later
+// windows apply the same errors meanwhile.  Errors replace the used columns of
+// the row state; W0 - Q is formed at the write-out from W0, the codes and the
+// row's scale.
+constexpr int QT = 256;
+__global__ void __launch_bounds__(QT, 1)
+    sweep64q_kernel(const float* __restrict__ W0, const double* __restrict__ acc, int64_t out,
+                    int64_t in, const double* __restrict__ Ub, int64_t b, int kb, int bits,
+                    int g, int scale_given, int8_t* __restrict__ codes,
+                    float* __restrict__ qscale, uint8_t* __restrict__ qzero,
+                    int8_t* __restrict__ dq, int* __restrict__ dex, int64_t dkpad, int ds,
+                    double* __restrict__ dsb, int64_t ldsb, DeviceStatus* st) {
+  extern __shared__ __align__(16) double smem64[];
+  double* Us = smem64;                                   // [B][B] U_GG
+  double* Wr = Us + B * B;                               // [RS][LDW] row state / errors
+  double* inv_u = Wr + RS * LDW;                         // [B]
+  double* scale_s = inv_u + B;                           // [RS]
+  double* zero_s = scale_s + RS;                         // [RS]
+  double* maxbuf = zero_s + RS;                          // [4][RS]
+  int8_t* Cs = reinterpret_cast<int8_t*>(maxbuf + 4 * RS);  // [RS][B] codes
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q = warp >> 1;                 // window
+  const int lrow = (warp & 1) * 32 + lane;  // row within the CTA
+  pdl_launch_dependents();
+  pdl_wait();
+  if (status_bad(st)) return;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * RS;
+  const int rows_here = static_cast<int>(std::min<int64_t>(RS, out - row0));
+  for (int idx = tid; idx < B * B; idx += QT) Us[idx] = Ub[idx];
+  for (int j = tid; j < B; j += QT) inv_u[j] = j < kb ? 1.0 / Ub[j * B + j] : 0.0;
+  for (int idx = tid; idx < RS * B; idx += QT) {
+    const int r = idx >> 7, c = idx & (B - 1);
+    Wr[r * LDW + c] = (r < rows_here && c < kb) ? acc[(row0 + r) * in + b + c] : 0.0;
+  }
+  __syncthreads();
+  {  // W_G = W0_G + acc_G U_GG
+    const int ty = tid >> 4, tx = tid & 15;
+    double o[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) o[i][c] = 0.0;
+    for (int k = 0; k < kb; ++k) {
+      double a[4], u[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Wr[(4 * ty + i) * LDW + k];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) u[c] = Us[k * B + tx + 16 * c];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[i][c] = fma(a[i], u[c], o[i][c]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 4 * ty + i;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int col = tx + 16 * c;
+        double w = 0.0;
+        if (r < rows_here && col < kb)
+          w = static_cast<double>(W0[(row0 + r) * in + b + col]) + o[i][c];
+        Wr[r * LDW + col] = w;
+      }
+    }
+  }
+  __syncthreads();
+
+  const bool asym = qzero != nullptr;
+  const int qmax = (1 << (bits - 1)) - 1;
+  const double fqmax = asym ? static_cast<double>((1 << bits) - 1) : static_cast<double>(qmax);
+  const int64_t ngroups = (in + g - 1) / g;
+  const int64_t row = row0 + lrow;
+  const bool valid = lrow < rows_here;
+  double* wrow = Wr + lrow * LDW;
+  if (q == 0) {
+    // the row's scale: a group starts here (its whole width is this block when
+    // g == 128) unless it was taken beforehand or continues from earlier
+    double sc, z = 0.0;
+    if (b % g == 0 && !scale_given) {
+      double m = 0.0, mn = 0.0;
+      for (int c = 0; c < kb; ++c) {
+        const double v = wrow[c];
+        m = fmax(m, asym ? v : fabs(v));
+        mn = fmin(mn, v);
+      }
+      if (!asym) {
+        sc = m / fqmax;
+      } else {
+        sc = (m - mn) / fqmax;
+        z = sc > 0.0 ? rint(-mn / sc) : 0.0;
+        z = fmin(fmax(z, 0.0), fqmax);
+        if (valid) qzero[row * ngroups + b / g] = static_cast<uint8_t>(z);
+      }
+      if (valid) qscale[row * ngroups + b / g] = static_cast<float>(sc);
+    } else {
+      sc = valid ? static_cast<double>(qscale[row * ngroups + b / g]) : 0.0;
+      if (asym && valid) z = static_cast<double>(qzero[row * ngroups + b / g]);
+    }
+    scale_s[lrow] = sc;
+    zero_s[lrow] = z;
+  }
+  const int c0 = SUB * q;
+  double ws[SUB];
+#pragma unroll
+  for (int k = 0; k < SUB; ++k) ws[k] = wrow[c0 + k];
+  __syncthreads();
+  const double sc = scale_s[lrow];
+  const double rsc = sc > 0.0 ? 1.0 / sc : 0.0;
+  const double cmin = asym ? -zero_s[lrow] : -static_cast<double>(qmax) - 1.0;
+  const double cmax = asym ? fqmax - zero_s[lrow] : static_cast<double>(qmax);
+  int8_t* crow = Cs + lrow * B;
+
+  for (int p = 0; p < 4; ++p) {
+    if (q >= p && SUB * p < kb) {
+      if (p > 0) {
+        const int cp = SUB * (p - 1);
+#pragma unroll 4
+        for (int t = 0; t < SUB; ++t) {
+          const double ev = wrow[cp + t];
+          const double* urow = Us + (cp + t) * B + c0;
+#pragma unroll
+          for (int k = 0; k < SUB; ++k) ws[k] = fma(-ev, urow[k], ws[k]);
+        }
+      }
+      if (q == p) {
+#pragma unroll
+        for (int jj = 0; jj < SUB; ++jj) {
+          const int j = c0 + jj;
+          if (j < kb) {
+            const double wj = ws[jj];
+            const double qv = sc > 0.0 ? fmin(fmax(code64(wj, sc, rsc), cmin), cmax) : 0.0;
+            const double err = (wj - qv * sc) * inv_u[j];
+            crow[j] = static_cast<int8_t>(qv);
+            ws[jj] = err;
+#pragma unroll
+            for (int k = jj + 1; k < SUB; ++k) ws[k] = fma(-err, Us[j * B + c0 + k], ws[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < SUB; ++k) wrow[c0 + k] = ws[k];
+      }
+    }
+    __syncthreads();
+  }
+
+  // write-out: codes (this thread's 32 columns), W0 - Q, its digits
+  double d0[SUB];
+  double m = 0.0;
+  const float* w0row = W0 + row * in + b + c0;
+#pragma unroll
+  for (int k = 0; k < SUB; ++k) {
+    const int c = c0 + k;
+    double v = 0.0;
+    if (valid && c < kb) {
+      v = static_cast<double>(w0row[k]) - static_cast<double>(crow[c]) * sc;
+      codes[row * in + b + c] = crow[c];
+    }
+    d0[k] = v;
+    m = fmax(m, fabs(v));
+  }
+  maxbuf[q * RS + lrow] = m;
+  __syncthreads();
+  m = fmax(fmax(maxbuf[lrow], maxbuf[RS + lrow]), fmax(maxbuf[2 * RS + lrow], maxbuf[3 * RS + lrow]));
+  if (!valid) return;
+  int ex = 0;
+  if (m > 0.0) frexp(m, &ex);
+  if (q == 0) dex[row] = ex;
+  if (dsb != nullptr) {
+    double* drow = dsb + row * ldsb + c0;
+#pragma unroll
+    for (int k = 0; k < SUB; ++k)
+      if (c0 + k < kb) drow[k] = d0[k];
+  }
+  if (c0 >= dkpad) return;
+  const double sc6 = m > 0.0 ? pow2(6 - ex) : 0.0;
+  const int64_t plane = out * dkpad;
+#pragma unroll
+  for (int k4 = 0; k4 < SUB; k4 += 4) {
+    uint32_t w[kMaxDigits] = {};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      double y = d0[k4 + t] * sc6;  // zero past kb
+      for (int i = 0; i < ds; ++i) {
+        const double di = rint(y);
+        y = (y - di) * 128.0;
+        w[i] |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+      }
+    }
+    for (int i = 0; i < ds; ++i)
+      *reinterpret_cast<uint32_t*>(dq + i * plane + row * dkpad + c0 + k4) = w[i];
   }
 }
 
@@ -366,7 +589,9 @@ int run_gptq_sweep64(const float* W0, int64_t out, int64_t in, const double* L, 
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
   if (dev < 64 && !attr_set[dev]) {
     if (cudaFuncSetAttribute(sweep64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmem) != cudaSuccess)
+                             kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(sweep64q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemQ) != cudaSuccess)
       return PIQ_ERR_CUDA;
     attr_set[dev] = true;
   }
@@ -414,23 +639,31 @@ int run_gptq_sweep64(const float* W0, int64_t out, int64_t in, const double* L, 
       dA.kpad = digit_kpad(kb);
       dA.s = kSweepDigits;
       note_launch();
-      if (launch_pdl(sweep64_kernel, dim3(grid), dim3(THREADS), kSmem, stream, W0, w.acc, out, in,
-                     w.Ub + static_cast<int64_t>(bk) * B * B, b, kb, bits, g, wide ? 1 : 0, codes,
-                     qscale, qzero, dA.q, dA.ex, dA.kpad, dA.s,
-                     use_sb ? w.dsb + (b - S0) : nullptr, static_cast<int64_t>(kSuperBlock),
-                     st) != cudaSuccess)
-        return PIQ_ERR_CUDA;
+      const cudaError_t le =
+          (g % B == 0)
+              ? launch_pdl(sweep64q_kernel, dim3(grid), dim3(QT), kSmemQ, stream, W0, w.acc, out,
+                           in, w.Ub + static_cast<int64_t>(bk) * B * B, b, kb, bits, g,
+                           wide ? 1 : 0, codes, qscale, qzero, dA.q, dA.ex, dA.kpad, dA.s,
+                           use_sb ? w.dsb + (b - S0) : nullptr,
+                           static_cast<int64_t>(kSuperBlock), st)
+              : launch_pdl(sweep64_kernel, dim3(grid), dim3(THREADS), kSmem, stream, W0, w.acc,
+                           out, in, w.Ub + static_cast<int64_t>(bk) * B * B, b, kb, bits, g,
+                           wide ? 1 : 0, codes, qscale, qzero, dA.q, dA.ex, dA.kpad, dA.s,
+                           use_sb ? w.dsb + (b - S0) : nullptr,
+                           static_cast<int64_t>(kSuperBlock), st);
+      if (le != cudaSuccess) return PIQ_ERR_CUDA;
       const int64_t lim = use_sb ? S1 : in;
       if (e < lim) {
         // acc[:, e:lim] += (W0 - Q)[:, b:e] R[b:e, e:lim];  B operand row n, digit k:
-        // R[b + k][e + n] = L[in-1-b-k][in-1-e-n]
+        // R[b + k][e + n] = L[in-1-b-k][in-1-e-n], read from the mirror of L in
+        // the upper triangle, P[in-1-e-n][in-1-b-k] (contiguous in k)
         DigitMat dB;
         dB.q = w.rq;
         dB.ex = w.rex;
         dB.rows = lim - e;
         dB.kpad = dA.kpad;
         dB.s = kSweepDigits;
-        rc = launch_slice(L + (in - 1 - b) * in + (in - 1 - e), -1, -in, lim - e, kb,
+        rc = launch_slice(L + (in - 1 - e) * in + (in - 1 - b), -in, -1, lim - e, kb,
                           kSweepDigits, &dB, stream);
         if (rc == PIQ_OK)
           rc = launch_ozaki_gemm(out, lim - e, dA, dB, 1.0, 1, 0, w.acc + e, in, st, stream);
@@ -453,7 +686,7 @@ int run_gptq_sweep64(const float* W0, int64_t out, int64_t in, const double* L, 
       dB.s = kSweepDigits;
       rc = launch_slice(w.dsb, kSuperBlock, 1, out, K, kSweepDigits, &dA, stream);
       if (rc == PIQ_OK)
-        rc = launch_slice(L + (in - 1 - S0) * in + (in - 1 - S1), -1, -in, in - S1, K,
+        rc = launch_slice(L + (in - 1 - S1) * in + (in - 1 - S0), -in, -1, in - S1, K,
                           kSweepDigits, &dB, stream);
       if (rc == PIQ_OK)
         rc = launch_ozaki_gemm(out, in - S1, dA, dB, 1.0, 1, 0, w.acc + S1, in, st, stream);

@@ -8,9 +8,14 @@
 // chunks bias diag(H) by -1.9e-6 relative), and an FP32 running sum of chunks
 // adds a random walk on top.  At a 28672-column layer either flips enough GPTQ
 // rounding decisions to break the code parity with an FP64 evaluation of the
-// loop.  Here each 128-sample chunk (8 MMAs) is accumulated in TMEM and then
-// added into FP64 sums held in the epilogue threads' registers, in chunk
-// order: the only FP32 roundings left are those inside a chunk.
+// loop.  Here each 128-sample chunk (8 MMAs) is accumulated in TMEM; two
+// consecutive chunks are added in FP32 (round to nearest) and that sum goes
+// into FP64 sums held in the epilogue threads' registers, in chunk order.  The
+// FP32 roundings left are those inside a chunk and one per chunk pair; the
+// pairing halves the fp32 -> fp64 conversions, which run at a quarter of the
+// FP32 rate and would otherwise set the pace.  Four 128-column TMEM
+// accumulators: the MMA warp fills one pair while the epilogue drains the
+// other.
 //
 // Tiles of 128 x 128 on or above the diagonal (the fp64 sums of a 128 x 256
 // tile would not fit in registers), round-robin over one persistent CTA per
@@ -44,7 +49,8 @@ constexpr int B_BYTES = BN * BK * 2;            // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int NBUF = 4;  // TMEM accumulators (two chunk pairs)
+constexpr int TMEM_COLS = NBUF * BN;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int KC = 128;  // samples per TMEM accumulation
 constexpr int KB_CHUNK = KC / BK;
@@ -72,8 +78,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;  // [2]
-  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* acc_full = empty + STAGES;  // [NBUF]
+  uint64_t* acc_empty = acc_full + NBUF;  // [NBUF]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
     }
@@ -137,8 +143,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         for (int ch = 0; ch < n_chunks && ok; ++ch, ++lt) {
-          const int buf = lt & 1;
-          const uint32_t use = static_cast<uint32_t>(lt >> 1);
+          const int buf = lt % NBUF;
+          const uint32_t use = static_cast<uint32_t>(lt / NBUF);
           if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 52)) {
             ok = false;
             break;
@@ -186,31 +192,47 @@ __global__ void __launch_bounds__(THREADS, 1)
       double sum[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) sum[i] = 0.0;
-      for (int ch = 0; ch < n_chunks; ++ch, ++lt) {
-        const int buf = lt & 1;
-        const uint32_t use = static_cast<uint32_t>(lt >> 1);
-        if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 54)) {
-          ok = false;
-          break;
+      // chunks in pairs (a tile with an odd count ends with a single one);
+      // chunk ch sits in buffer (tile's first chunk index + ch) % NBUF
+      for (int ch = 0; ch < n_chunks; ch += 2) {
+        const int two = (ch + 1 < n_chunks) ? 2 : 1;
+        uint32_t taddr[2];
+        for (int u = 0; u < two; ++u) {
+          const int l = lt + ch + u;
+          const int buf = l % NBUF;
+          const uint32_t use = static_cast<uint32_t>(l / NBUF);
+          if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 54)) {
+            ok = false;
+            break;
+          }
+          taddr[u] = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                     static_cast<uint32_t>(buf * BN + h * 64);
         }
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(buf * BN + h * 64);
         // 16 columns per TMEM load keep the fp64 sums and the loaded values
         // within the register budget of ten warps per SM
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           if (qq < 2 ? live0 : live1) {
             float v[16];
-            tmem_ld_32x32b_x16(taddr + 16 * qq, v);
+            tmem_ld_32x32b_x16(taddr[0] + 16 * qq, v);
+            if (two == 2) {
+              float w[16];
+              tmem_ld_32x32b_x16(taddr[1] + 16 * qq, w);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], w[i]);
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) sum[16 * qq + i] += static_cast<double>(v[i]);
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (lane == 0)
+          for (int u = 0; u < two; ++u) mbar_arrive(&acc_empty[(lt + ch + u) % NBUF]);
       }
+      lt += n_chunks;
       if (!ok) break;
       const int row = row0 + lane;
       if (row < p.in) {

@@ -31,7 +31,7 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     bench.barrier(world)
     t = bench.max_over_ranks(10.0 + rank, world)
-    W, X, X2 = bench.make_inputs(rank, n=64)
+    W, X, X2 = bench.make_inputs(rank, n=64, workload="q_proj_7b")
     q.put((rank, t, float(W[0, :4].sum()), int(X[0, :4].astype(np.int64).sum())))
     bench.barrier(world)
     dist.destroy_process_group()

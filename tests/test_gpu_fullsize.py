@@ -47,8 +47,10 @@ def _layer(spec):
 def _gptq_full(spec, bits=None, shift=False):
     bits = spec.bits if bits is None else bits
     W, X, perm, U = _layer(spec)
+    f0 = piq.simt_gemm_fallbacks()
     out = piq.gptq_quantize_layer(to_gpu_w(W), to_gpu_x(X), bits=bits, g=spec.g,
                                   damp=spec.damp, act_order=spec.act_order)
+    assert piq.simt_gemm_fallbacks() == f0  # every product on the tensor cores
     e2_gpu = X2 = None
     if shift:
         X2 = make_x_bits(spec, seed=spec.seed + 1, permute_seed=spec.seed + 1)

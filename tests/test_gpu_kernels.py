@@ -61,6 +61,18 @@ def test_upper_factor_matches_oracle(inp, act):
     assert e_inv < 1e-4
 
 
+@pytest.mark.parametrize("inp", [512, 1032])
+def test_fp32_step_entries_stay_on_the_tensor_cores(inp):
+    # the FP32 factor and sweep step entries: 16-byte aligned operands, so no
+    # product falls back to the SIMT kernel
+    W, X = _layer(16, inp, 3 * inp, seed=inp + 1)
+    Hx = O.hessian_ref(X)
+    f0 = piq.simt_gemm_fallbacks()
+    U, _ = piq.upper_factor(torch.from_numpy(Hx.astype(np.float32)).cuda(), 0.01)
+    piq.gptq_sweep(to_gpu_w(W), U, 4, 128)
+    assert piq.simt_gemm_fallbacks() == f0
+
+
 def test_not_positive_definite_reports_status():
     H = torch.zeros(64, 64, device="cuda")
     with pytest.raises(piq.PiqError) as e:
