@@ -202,9 +202,9 @@ def workload_config(spec, n, workload="down_proj_70b"):
 
 
 # ------------------------------------------------------------ roofline arithmetic
-# Digits per operand of the FP64-grade products (library constants: factor 6,
+# Digits per operand of the FP64-grade products (library constants: factor 5,
 # block updates 5) and the nominal INT8 : BF16 dense tensor ratio.
-FACTOR_PAIRS = 6 * 7 // 2
+FACTOR_PAIRS = 5 * 6 // 2
 SWEEP_PAIRS = 5 * 6 // 2
 INT8_PER_BF16 = 2.0
 
@@ -213,7 +213,7 @@ def phase_rooflines(ph, out, inp, n, bf16_peak, hbm_peak):
     """Per-phase achieved rate and fraction of its roofline, from the phase
     times (ms) of one gptq_quantize_layer call.  Algorithmic work:
     hessian n in (in+1) bf16 flop (upper triangle); factor in^3 / 3 FP64 flop
-    (Cholesky of the damped H), bound by the INT8 tensor rate over the 21 digit
+    (Cholesky of the damped H), bound by the INT8 tensor rate over the 15 digit
     products of each FP64-grade product; sweep out in^2 FP64 flop of block
     updates (15 digit products); pack out in (1 + 4 + 4 + 1/2) bytes (codes and
     W read, D written, nibbles written); error 3 out in (in + 256) bf16 flop."""

@@ -123,7 +123,7 @@ int launch_identity_perm(int64_t in, int32_t* perm, int32_t* invperm, cudaStream
 // A matrix as s signed 7-bit digits per entry, scaled per row by 2^ex[row]:
 // q[i][row][kpad] int8 (K-major, zero padded to kpad), ex[row] int32.
 constexpr int kMaxDigits = 7;
-constexpr int kFactorDigits = 6;  // Cholesky panel products: ~1e-12 relative
+constexpr int kFactorDigits = 5;  // Cholesky panel products: ~1e-10 relative
 constexpr int kSweepDigits = 5;   // GPTQ block updates: ~1e-10 relative
 struct DigitMat {
   int8_t* q = nullptr;

@@ -117,6 +117,11 @@ __device__ __forceinline__ void tmem_ld_i32x32(uint32_t taddr, int (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __float_as_int(f[i]);
 }
 
+// S (digits per operand) is a template parameter so that the MMA issue loop
+// (S (S + 1) / 2 digit pairs x 2 MMAs per k block) unrolls into straight-line
+// code with constant descriptor offsets: one thread issues every MMA, and with
+// a runtime loop the issue itself, not the tensor core, set the pace.
+template <int S>
 __global__ void __launch_bounds__(THREADS, 1)
     ozaki_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, OzParams p) {
@@ -156,8 +161,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_kb = (p.K + BK - 1) / BK;
   pdl_wait();
   const bool skip = status_bad(p.st);
-  const int S = p.s;
-  const uint32_t set_cols = static_cast<uint32_t>(S * BN);
+  constexpr uint32_t set_cols = static_cast<uint32_t>(S * BN);
 
   if (skip) {
   } else if (warp == 0) {
@@ -206,18 +210,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
+          // descriptors of digit 0 of A and B in this stage; digit i adds
+          // i * tile bytes / 16 to the address field, a k step of 32 bytes adds 2
           const uint32_t a0 = smem_u32(smem + st * p.stage_bytes);
-          const uint32_t b0 = a0 + static_cast<uint32_t>(S * A_TILE);
+          const uint64_t ad0 = smem_desc(a0, 16, 512, kLayoutSw64);
+          const uint64_t bd0 = smem_desc(a0 + S * A_TILE, 16, 512, kLayoutSw64);
+#pragma unroll
           for (int i = 0; i < S; ++i) {
+#pragma unroll
             for (int j = 0; i + j < S; ++j) {
-              const uint32_t dt = d0 + static_cast<uint32_t>((i + j) * BN);
 #pragma unroll
               for (int kk = 0; kk < BK / 32; ++kk) {
-                const uint64_t ad = smem_desc(a0 + i * A_TILE + kk * 32, 16, 512, kLayoutSw64);
-                const uint64_t bd = smem_desc(b0 + j * B_TILE + kk * 32, 16, 512, kLayoutSw64);
                 // the first product into accumulator d of this tile starts it
-                const bool first = kb == 0 && kk == 0 && i == 0;
-                umma_i8(dt, ad, bd, idesc, first ? 0u : 1u);
+                const uint32_t acc = (kb == 0 && kk == 0 && i == 0) ? 0u : 1u;
+                umma_i8(d0 + static_cast<uint32_t>((i + j) * BN),
+                        ad0 + static_cast<uint64_t>(i * (A_TILE >> 4) + kk * 2),
+                        bd0 + static_cast<uint64_t>(j * (B_TILE >> 4) + kk * 2), idesc, acc);
               }
             }
           }
@@ -398,7 +406,7 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
                       int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
                       cudaStream_t stream) {
   if (M <= 0 || N <= 0) return PIQ_OK;
-  if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s > kMaxDigits)
+  if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s < 3 || A.s > 6)
     return PIQ_ERR_INVALID_ARG;
   if (A.kpad * (A.s + 1) >= (int64_t)1 << 19) return PIQ_ERR_INVALID_ARG;  // int32 exactness
   if (M > INT32_MAX || N > INT32_MAX) return PIQ_ERR_INVALID_ARG;
@@ -441,19 +449,27 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
   // at least half an SM's shared memory, so that two CTAs that each hold all
   // 512 TMEM columns never share an SM
   const int smem = std::max(p.stages * p.stage_bytes + 1024 + 256, 120 * 1024);
-  static bool attr_set[64] = {};
+  void (*kern)(CUtensorMap, CUtensorMap, OzParams) = nullptr;
+  switch (p.s) {
+    case 3: kern = ozaki_gemm_kernel<3>; break;
+    case 4: kern = ozaki_gemm_kernel<4>; break;
+    case 5: kern = ozaki_gemm_kernel<5>; break;
+    case 6: kern = ozaki_gemm_kernel<6>; break;
+    default: return PIQ_ERR_INVALID_ARG;
+  }
+  static bool attr_set[64][8] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PIQ_ERR_CUDA;
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(ozaki_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             MAX_SMEM) != cudaSuccess)
+  if (dev < 64 && !attr_set[dev][p.s]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MAX_SMEM) !=
+        cudaSuccess)
       return PIQ_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev][p.s] = true;
   }
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
   note_launch();
-  if (launch_pdl(ozaki_gemm_kernel, dim3(grid), dim3(THREADS), static_cast<size_t>(smem), stream,
-                 ma, mb, p) != cudaSuccess)
+  if (launch_pdl(kern, dim3(grid), dim3(THREADS), static_cast<size_t>(smem), stream, ma, mb, p) !=
+      cudaSuccess)
     return PIQ_ERR_CUDA;
   return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }

@@ -56,8 +56,8 @@ def test_phase_rooflines():
     r = bench.phase_rooflines(ph, 4096, 4096, 131072, 1600.0, 6500.0)
     assert r["hessian"]["achieved"] == pytest.approx(131072 * 4096 * 4097 / 1e-3 / 1e12)
     assert r["hessian"]["frac"] == pytest.approx(r["hessian"]["achieved"] / 1600.0)
-    # FP64-grade products: INT8 = 2 x bf16, 21 (factor) and 15 (sweep) digit products
-    assert r["factor"]["peak"] == pytest.approx(3200.0 / 21)
+    # FP64-grade products: INT8 = 2 x bf16, 15 digit products (factor and sweep)
+    assert r["factor"]["peak"] == pytest.approx(3200.0 / 15)
     assert r["factor"]["achieved"] == pytest.approx(4096 ** 3 / 3 / 1e-3 / 1e12)
     assert r["sweep"]["peak"] == pytest.approx(3200.0 / 15)
     assert r["sweep"]["achieved"] == pytest.approx(4096 ** 3 / 1e-3 / 1e12)

@@ -129,3 +129,30 @@ def test_awq_search_properties(p):
     c2, sc2 = O.group_rtn_ref(W * (2.0 ** p["k"] * s_best)[None, :], p["bits"], p["g"])
     assert np.array_equal(c1, a.codes) and np.array_equal(c1, c2)
     assert np.array_equal(sc2, 2.0 ** p["k"] * sc1)
+
+
+def test_sweep_identity_on_r():
+    # The identity the GPU sweep is built on: with H_d = R R^T (R upper, the
+    # reversed Cholesky factor) and U = inv(R), the listing's loop satisfies
+    # W0 - Q = err U row by row (W0 the weights before any update, Q = code *
+    # scale, err the pushed errors), so err = (W0 - Q) R and the current weights
+    # at the start of a block G are W0_G + acc_G inv(R_GG) with
+    # acc = sum_{p < b} (W0 - Q)_p R[p, :].
+    from workloads import make_weight, make_x_bits, small_spec
+    spec = small_spec(12, 256, 900, seed=71, sigma_ln=0.9, n_outlier=3, outlier_gain=20.0)
+    W, X = make_weight(spec).astype(np.float64), make_x_bits(spec)
+    H = O.hessian_ref(X)
+    perm, U, lam = O.gptq_prepare_ref(H, 0.01, False)
+    Hd = H + lam * np.eye(H.shape[0])
+    Jr = slice(None, None, -1)
+    R = np.linalg.cholesky(Hd[Jr, Jr])[Jr, Jr]
+    assert np.allclose(R @ R.T, Hd, rtol=0, atol=1e-9 * np.abs(Hd).max())
+    codes, scales, v, err = O.gptq_sweep_ref(W, U, 4, 64)
+    Q = codes * np.repeat(scales, 64, axis=1)
+    assert np.allclose(err, (W - Q) @ R, rtol=0, atol=1e-9 * np.abs(err).max())
+    # block-start weights of the block [128, 192): v * scale there equals
+    # W0 + acc inv(R_GG) before any of the block's own updates, at its first column
+    b = 128
+    acc = (W - Q)[:, :b] @ R[:b, b:]
+    Wb = W[:, b:] + acc @ np.linalg.inv(R[b:, b:])
+    assert np.allclose(v[:, b] * scales[:, b // 64], Wb[:, 0], rtol=0, atol=1e-9)
