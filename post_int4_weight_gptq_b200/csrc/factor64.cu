@@ -80,16 +80,23 @@ __global__ void build_rev64_kernel(const double* H, int64_t in, const int32_t* p
 // FP64) and write its inverse to X11 (128 x 128, row-major, zeros above the
 // diagonal and outside nb).  Rows/cols >= nb are padded with the identity.
 //
-// Right-looking over 16-wide sub-panels: warp 0 factors the 16 x 16 diagonal
-// block in registers (lane i holds row i; each pivot's column reaches the
-// lanes by shuffles); one thread per row below solves that row against it by
-// substitution; the trailing lower triangle gets the rank-16 update in 4 x 4
-// register tiles.  The inverse follows in the same 16-row blocks: for block
-// R, T = L[R, <R] X[<R, :] (register tiles over all threads), then each
-// column's 16 entries by substitution against L[R, R].  Factor and inverse
-// share one shared array: the factor in the lower triangle, the inverse
-// transposed in the strictly upper one, its diagonal apart.
-constexpr int SP16 = 16;
+// Factor: right-looking over 32-wide panels.  Warp 0 factors the 32 x 32
+// diagonal block with lane i holding row i in registers; pivot J takes its
+// diagonal by a shuffle, 1 / L_JJ from rsqrt, and hands the next pivot its
+// updated diagonal through one more shuffle, while the rest of column J
+// reaches the lanes through shared memory off that chain.  One thread per row
+// below solves the row against the block by substitution and also stores it
+// transposed; the trailing lower triangle takes the rank-32 update from the
+// transposed copy in 4 x 4 register tiles.
+//
+// Inverse, by recursive doubling: the four 32 x 32 diagonal blocks are
+// inverted column by column (one warp each, lane j: column j), then pairs and
+// halves are joined with
+//     inv([[A, 0], [B, C]]) = [[inv(A), 0], [-inv(C) B inv(A), inv(C)]],
+// each join two products in shared memory.  The factor sits in the lower
+// triangle of one shared array, the inverse transposed in its strictly upper
+// triangle (X[i][j] at S[j][i]) with its diagonal apart.
+constexpr int PW = 32;
 
 __device__ __forceinline__ void fma4x4d(double (&acc)[4][4], const double (&a)[4],
                                         const double (&b)[4]) {
@@ -99,13 +106,74 @@ __device__ __forceinline__ void fma4x4d(double (&acc)[4][4], const double (&a)[4
     for (int y = 0; y < 4; ++y) acc[x][y] = fma(a[x], b[y], acc[x][y]);
 }
 
-__global__ void __launch_bounds__(CT)
+// X[cA + k][cA + j] (k >= j) from the transposed storage; zero for k < j.
+__device__ __forceinline__ double x_lower(const double* S, const double* xd, int r, int c) {
+  const double s = S[c * LDS + r];
+  return r > c ? s : (r == c ? xd[r] : 0.0);
+}
+
+// Join step 1: T[i][j] = sum_k L[cC + i][cA + k] X[cA + k][cA + j] (k >= j),
+// for the thread's outputs i = ti + 16 x, j = tj + js y; T row-major, stride m.
+template <int MX, int NY>
+__device__ __forceinline__ void join_t(const double* S, const double* xd, double* T, int m,
+                                       int cA, int cC, int ti, int tj, int js) {
+  double acc[MX][NY];
+#pragma unroll
+  for (int x = 0; x < MX; ++x)
+#pragma unroll
+    for (int y = 0; y < NY; ++y) acc[x][y] = 0.0;
+  for (int k = tj & ~1; k < m; ++k) {  // warp-uniform start; X[k][j] = 0 below j
+    double a[MX], bv[NY];
+#pragma unroll
+    for (int x = 0; x < MX; ++x) a[x] = S[(cC + ti + 16 * x) * LDS + cA + k];
+#pragma unroll
+    for (int y = 0; y < NY; ++y) bv[y] = x_lower(S, xd, cA + k, cA + tj + js * y);
+#pragma unroll
+    for (int x = 0; x < MX; ++x)
+#pragma unroll
+      for (int y = 0; y < NY; ++y) acc[x][y] = fma(a[x], bv[y], acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < MX; ++x)
+#pragma unroll
+    for (int y = 0; y < NY; ++y) T[(ti + 16 * x) * m + tj + js * y] = acc[x][y];
+}
+
+// Join step 2: X[cC + i][cA + j] = -sum_k X[cC + i][cC + k] T[k][j] (k <= i),
+// stored transposed at S[cA + j][cC + i].
+template <int MX, int NY>
+__device__ __forceinline__ void join_x(double* S, const double* xd, const double* T, int m,
+                                       int cA, int cC, int ti, int tj, int js) {
+  double acc[MX][NY];
+#pragma unroll
+  for (int x = 0; x < MX; ++x)
+#pragma unroll
+    for (int y = 0; y < NY; ++y) acc[x][y] = 0.0;
+  for (int k = 0; k < m; ++k) {
+    double a[MX], bv[NY];
+#pragma unroll
+    for (int x = 0; x < MX; ++x) a[x] = x_lower(S, xd, cC + ti + 16 * x, cC + k);
+#pragma unroll
+    for (int y = 0; y < NY; ++y) bv[y] = T[k * m + tj + js * y];
+#pragma unroll
+    for (int x = 0; x < MX; ++x)
+#pragma unroll
+      for (int y = 0; y < NY; ++y) acc[x][y] = fma(a[x], bv[y], acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < MX; ++x)
+#pragma unroll
+    for (int y = 0; y < NY; ++y) S[(cA + tj + js * y) * LDS + cC + ti + 16 * x] = -acc[x][y];
+}
+
+__global__ void __launch_bounds__(CT, 1)
     chol64_block_kernel(double* P, int64_t ld, int64_t o, int nb, double* X11,
                         DeviceStatus* st) {
   extern __shared__ __align__(16) double sm64[];
-  double* S = sm64;               // [NB][LDS] factor (lower), inverse (upper, transposed)
-  __shared__ double rdiag[NB];    // 1 / L_ii
-  __shared__ double xd[NB];       // diagonal of the inverse
+  double* S = sm64;             // [NB][LDS] factor (lower), inverse (upper, transposed)
+  double* Tb = S + NB * LDS;    // [PW][NB] panel transposed; [64][64] join product
+  __shared__ double rdiag[NB];  // 1 / L_ii
+  __shared__ double xd[NB];     // diagonal of the inverse
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
@@ -114,67 +182,67 @@ __global__ void __launch_bounds__(CT)
   if (tid == 0) bad = 0;
   for (int idx = tid; idx < NB * NB; idx += CT) {
     const int i = idx >> 7, j = idx & (NB - 1);
-    double v = 0.0;
-    if (i < nb && j <= i) v = P[(o + i) * ld + (o + j)];
-    else if (i == j) v = 1.0;
-    S[i * LDS + j] = v;
+    if (i < nb && j <= i)
+      cp_async8(S + i * LDS + j, P + (o + i) * ld + (o + j));
+    else
+      S[i * LDS + j] = (i == j) ? 1.0 : 0.0;
   }
+  cp_async_wait_all();
   __syncthreads();
 
-  for (int c0 = 0; c0 < NB; c0 += SP16) {
-    // ---- the 16 x 16 diagonal block, warp 0
+  for (int c0 = 0; c0 < NB; c0 += PW) {
+    // ---- the 32 x 32 diagonal block, warp 0 (lane i: row c0 + i)
     if (warp == 0) {
-      double a[SP16];
+      double* srow = S + (c0 + lane) * LDS + c0;
+      double a[PW];
 #pragma unroll
-      for (int k = 0; k < SP16; ++k)
-        a[k] = (lane < SP16 && k <= lane) ? S[(c0 + lane) * LDS + c0 + k] : 0.0;
+      for (int k = 0; k < PW; ++k) a[k] = k <= lane ? srow[k] : 0.0;
       bool ok = true;
 #pragma unroll
-      for (int J = 0; J < SP16; ++J) {
+      for (int J = 0; J < PW; ++J) {
         const double d = __shfl_sync(0xffffffffu, a[J], J);
         ok = ok && (d > 0.0);
-        const double ljj = sqrt(d > 0.0 ? d : 1.0);
-        const double r = 1.0 / ljj;
-        if (lane == J) {
-          a[J] = ljj;
-          rdiag[c0 + J] = r;
-        } else if (lane > J) {
-          a[J] *= r;
-        }
-        // a[k] -= L[i][J] L[k][J] for J < k <= i
+        const double r = rsqrt(d > 0.0 ? d : 1.0);
+        a[J] = (lane == J) ? d * r : a[J] * r;  // L_JJ on lane J, L_iJ below it
+        if (lane >= J) srow[J] = a[J];
+        if (lane == 0) rdiag[c0 + J] = r;
+        if (J + 1 < PW) {
+          // the next pivot's diagonal first, by a shuffle
+          const double l1 = __shfl_sync(0xffffffffu, a[J], J + 1);
+          a[J + 1] = fma(-a[J], l1, a[J + 1]);
+          __syncwarp();
 #pragma unroll
-        for (int k = J + 1; k < SP16; ++k) {
-          const double lk = __shfl_sync(0xffffffffu, a[J], k);
-          if (lane >= k) a[k] = fma(-a[J], lk, a[k]);
+          for (int k = J + 2; k < PW; ++k)
+            a[k] = fma(-a[J], S[(c0 + k) * LDS + c0 + J], a[k]);
         }
       }
       if (!ok && lane == 0) {
         bad = 1;
         set_status(st, PIQ_ERR_NOT_PD, static_cast<int>(o + c0));
       }
-      if (lane < SP16) {
-#pragma unroll
-        for (int k = 0; k < SP16; ++k)
-          if (k <= lane) S[(c0 + lane) * LDS + c0 + k] = a[k];
-      }
     }
     __syncthreads();
     if (bad) return;
-    const int r0 = c0 + SP16;
+    const int r0 = c0 + PW;
     if (r0 >= NB) break;
-    // ---- rows below: y = A21 row solved against L11 (L21 = A21 inv(L11)^T)
+    // ---- rows below: L21 = A21 inv(L11)^T by substitution, kept also transposed in Tb
     for (int r = r0 + tid; r < NB; r += CT) {
-      double y[SP16];
+      double* row = S + r * LDS + c0;
+      double y[PW];
 #pragma unroll
-      for (int k = 0; k < SP16; ++k) y[k] = S[r * LDS + c0 + k];
+      for (int k = 0; k < PW; ++k) y[k] = row[k];
 #pragma unroll
-      for (int C = 0; C < SP16; ++C) {
+      for (int C = 0; C < PW; ++C) {
+        double v = y[C];
 #pragma unroll
-        for (int c = 0; c < C; ++c) y[C] = fma(-y[c], S[(c0 + C) * LDS + c0 + c], y[C]);
-        y[C] *= rdiag[c0 + C];
+        for (int c = 0; c < C; ++c) v = fma(-y[c], S[(c0 + C) * LDS + c0 + c], v);
+        y[C] = v * rdiag[c0 + C];
       }
 #pragma unroll
-      for (int k = 0; k < SP16; ++k) S[r * LDS + c0 + k] = y[k];
+      for (int k = 0; k < PW; ++k) {
+        row[k] = y[k];
+        Tb[k * NB + r] = y[k];
+      }
     }
     __syncthreads();
     // ---- A22 -= L21 L21^T on the lower 4 x 4 tiles
@@ -188,14 +256,14 @@ __global__ void __launch_bounds__(CT)
         const int bj = t - bi * (bi + 1) / 2;
         const int i0 = r0 + 4 * bi, j0 = r0 + 4 * bj;
         double acc[4][4] = {};
-#pragma unroll
-        for (int k = 0; k < SP16; ++k) {
-          double av[4], bv[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            av[x] = S[(i0 + x) * LDS + c0 + k];
-            bv[x] = S[(j0 + x) * LDS + c0 + k];
-          }
+#pragma unroll 8
+        for (int k = 0; k < PW; ++k) {
+          const double2 a01 = *reinterpret_cast<const double2*>(Tb + k * NB + i0);
+          const double2 a23 = *reinterpret_cast<const double2*>(Tb + k * NB + i0 + 2);
+          const double2 b01 = *reinterpret_cast<const double2*>(Tb + k * NB + j0);
+          const double2 b23 = *reinterpret_cast<const double2*>(Tb + k * NB + j0 + 2);
+          const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+          const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
           fma4x4d(acc, av, bv);
         }
 #pragma unroll
@@ -208,52 +276,38 @@ __global__ void __launch_bounds__(CT)
     __syncthreads();
   }
 
-  // ---- inverse X = inv(L), 16 rows at a time: X[R, :] = inv(L_RR) (E_R - L[R, <R] X[<R, :]).
-  // X[i][j] (i > j) is kept at S[j][i] (the strictly upper part, free), X[i][i] in xd.
-  for (int c0 = 0; c0 < NB; c0 += SP16) {
-    // -L[R, <R] X[<R, 0:c0] on the 16 x c0 block (4 x 4 tiles), kept as X[R][0:c0]
-    if (c0 > 0) {
-      const int ntile = (SP16 / 4) * (c0 / 4);
-      for (int t = tid; t < ntile; t += CT) {
-        const int bi = t / (c0 / 4), bj = t - bi * (c0 / 4);
-        const int i0 = c0 + 4 * bi, j0 = 4 * bj;
-        double acc[4][4] = {};
-        for (int k = j0; k < c0; ++k) {  // X[k][j] = 0 for k < j
-          double av[4], bv[4];
+  // ---- inverse: the four 32 x 32 diagonal blocks, warp w block w, lane j column j
+  if (warp < NB / PW) {
+    const int bw = PW * warp;
+    double x[PW];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            av[x] = S[(i0 + x) * LDS + k];
-            const int j = j0 + x;
-            bv[x] = k > j ? S[j * LDS + k] : (k == j ? xd[j] : 0.0);
-          }
-          fma4x4d(acc, av, bv);
-        }
+    for (int i = 0; i < PW; ++i) {
+      double v = (i == lane) ? 1.0 : 0.0;
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) S[(j0 + y) * LDS + i0 + x] = -acc[x][y];
-      }
-      __syncthreads();
+      for (int k = 0; k < i; ++k) v = fma(-S[(bw + i) * LDS + bw + k], x[k], v);
+      x[i] = v * rdiag[bw + i];  // zero above the diagonal (i < lane)
     }
-    // substitution against L_RR, one thread per column j <= c0 + 15
-    for (int j = tid; j < c0 + SP16; j += CT) {
-      double x[SP16];
 #pragma unroll
-      for (int i = 0; i < SP16; ++i) {
-        double v = (j < c0) ? S[j * LDS + c0 + i] : (j == c0 + i ? 1.0 : 0.0);
-#pragma unroll
-        for (int k = 0; k < i; ++k) v = fma(-S[(c0 + i) * LDS + c0 + k], x[k], v);
-        x[i] = v * rdiag[c0 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < SP16; ++i) {
-        const int r = c0 + i;
-        if (r > j) S[j * LDS + r] = x[i];
-        else if (r == j) xd[j] = x[i];
-      }
+    for (int i = 0; i < PW; ++i) {
+      if (i > lane) S[(bw + lane) * LDS + bw + i] = x[i];
+      else if (i == lane) xd[bw + lane] = x[i];
     }
+  }
+  __syncthreads();
+  // ---- join pairs (32 -> 64): blocks (0, 1) on threads 0..255, (2, 3) on 256..511
+  {
+    const int half = tid >> 8, t = tid & 255;
+    const int cA = 64 * half, cC = cA + 32;
+    join_t<2, 2>(S, xd, Tb + half * 32 * 32, 32, cA, cC, t & 15, t >> 4, 16);
+    __syncthreads();
+    join_x<2, 2>(S, xd, Tb + half * 32 * 32, 32, cA, cC, t & 15, t >> 4, 16);
     __syncthreads();
   }
+  // ---- join halves (64 -> 128)
+  join_t<4, 2>(S, xd, Tb, 64, 0, 64, tid & 15, tid >> 4, 32);
+  __syncthreads();
+  join_x<4, 2>(S, xd, Tb, 64, 0, 64, tid & 15, tid >> 4, 32);
+  __syncthreads();
 
   for (int idx = tid; idx < NB * NB; idx += CT) {
     const int i = idx >> 7, j = idx & (NB - 1);
@@ -339,7 +393,7 @@ __global__ void mirror_lower_kernel(double* P, int64_t in) {
 }
 
 constexpr int kBlockSmem = NB * LDS * 8;
-constexpr int kCholSmem64 = NB * LDS * 8;
+constexpr int kCholSmem64 = (NB * LDS + PW * NB) * 8;
 
 }  // namespace
 

@@ -48,7 +48,8 @@ constexpr int SUB = 32;      // columns per register window
 constexpr int THREADS = 256;
 constexpr int LDW = B + 1;   // fp64 row-state stride
 constexpr int kSmem = B * B * 8 + RS * LDW * 8 + B * 8 + 64;
-constexpr int kSmemQ = B * B * 8 + RS * LDW * 8 + B * 8 + 6 * 64 * 8 + 64 * 128;
+constexpr int CST = B + 4;   // code row stride in bytes (rows in distinct banks)
+constexpr int kSmemQ = B * B * 8 + RS * LDW * 8 + B * 8 + 10 * RS * 8 + RS * CST;
 constexpr int64_t kSuperBlock = 1024;  // columns per superblock of the block updates
 
 // rint(w / scale) for the IEEE quotient, from w * (1 / scale): the product is
@@ -256,33 +257,68 @@ __global__ void __launch_bounds__(THREADS, 1)
       dex[rs.row] = ex;
       const int64_t plane = out * dkpad;
       for (int c4 = 0; c4 < dkpad; c4 += 4) {
-        uint32_t w[kMaxDigits] = {};
+        double y[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int c = c4 + t;
-          double y = (c < kb && m > 0.0) ? wrow[c] * pow2(6 - ex) : 0.0;
-          for (int i = 0; i < ds; ++i) {
-            const double di = rint(y);
-            y = (y - di) * 128.0;
-            w[i] |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+          y[t] = (c < kb && m > 0.0) ? wrow[c] * pow2(6 - ex) : 0.0;
+        }
+#pragma unroll
+        for (int i = 0; i < kMaxDigits; ++i) {
+          if (i < ds) {
+            uint32_t w = 0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const double di = rint(y[t]);
+              y[t] = (y[t] - di) * 128.0;
+              w |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+            }
+            *reinterpret_cast<uint32_t*>(dq + i * plane + rs.row * dkpad + c4) = w;
           }
         }
-        for (int i = 0; i < ds; ++i)
-          *reinterpret_cast<uint32_t*>(dq + i * plane + rs.row * dkpad + c4) = w[i];
       }
     }
   }
 }
 
 // The same block for g % 128 == 0 (no group starts inside the block except at
-// its first column): 8 warps, warp w owns rows 32 (w % 2) .. + 31 of the CTA
-// (one per lane) and window q = w / 2 (block columns 32 q .. 32 q + 31) in
-// registers.  Phase p (0..3): the window-p threads apply window p-1's errors
-// to their window and run its serial column loop; the threads of later
-// windows apply the same errors meanwhile.  Errors replace the used columns of
-// the row state; W0 - Q is formed at the write-out from W0, the codes and the
-// row's scale.
+// its first column).  256 threads, 64 rows, in five steps:
+//  1. asynchronous copies: U_GG (128 KB) and the rows' acc_G into shared memory;
+//  2. W_G = W0_G + acc_G U_GG: U_GG is upper triangular, so column c sums over
+//     k <= c; warp w owns the column quads {w, 15-w, 16+w, 31-w} (equal work)
+//     and lane l the rows l and l+32;
+//  3. the row scale from the maxima of the four 32-column windows;
+//  4. the serial column loop: warp w owns rows 32 (w % 2) .. + 31 (one per
+//     lane) and window q = w / 2 (block columns 32 q .. 32 q + 31) in
+//     registers.  Phase p (0..3): the window-p threads apply window p-1's
+//     errors to their window and run its serial loop; the threads of later
+//     windows apply the same errors meanwhile.  The rounding takes w * (1 / s)
+//     and only records whether the product came within 1e-12 of a half
+//     integer; a thread that saw one re-runs its window from the saved state
+//     with the exact quotient there (code64), which gives what the plain loop
+//     gives;
+//  5. write-out, one warp per row at a time (lane l: columns 4l .. 4l+3):
+//     codes, W0 - Q, its digits and exponent.
 constexpr int QT = 256;
+
+// The serial loop of one window in shared memory with code64 rounding (the
+// rare path): wrow holds the window's state at the start of the loop and gets
+// its errors; crow gets its codes.
+__device__ __noinline__ void window_redo64(double* wrow, const double* Us, const double* inv_u,
+                                           int c0, int kb, double sc, double rsc, double cmin,
+                                           double cmax, int8_t* crow) {
+  for (int jj = 0; jj < SUB; ++jj) {
+    const int j = c0 + jj;
+    if (j >= kb) break;
+    const double wj = wrow[j];
+    const double qv = sc > 0.0 ? fmin(fmax(code64(wj, sc, rsc), cmin), cmax) : 0.0;
+    const double err = (wj - qv * sc) * inv_u[j];
+    crow[j] = static_cast<int8_t>(qv);
+    wrow[j] = err;
+    for (int k = jj + 1; k < SUB; ++k) wrow[c0 + k] = fma(-err, Us[j * B + c0 + k], wrow[c0 + k]);
+  }
+}
+
 __global__ void __launch_bounds__(QT, 1)
     sweep64q_kernel(const float* __restrict__ W0, const double* __restrict__ acc, int64_t out,
                     int64_t in, const double* __restrict__ Ub, int64_t b, int kb, int bits,
@@ -296,80 +332,115 @@ __global__ void __launch_bounds__(QT, 1)
   double* inv_u = Wr + RS * LDW;                         // [B]
   double* scale_s = inv_u + B;                           // [RS]
   double* zero_s = scale_s + RS;                         // [RS]
-  double* maxbuf = zero_s + RS;                          // [4][RS]
-  int8_t* Cs = reinterpret_cast<int8_t*>(maxbuf + 4 * RS);  // [RS][B] codes
+  double* mx = zero_s + RS;                              // [4][RS] window maxima
+  double* mn = mx + 4 * RS;                              // [4][RS] window minima
+  int8_t* Cs = reinterpret_cast<int8_t*>(mn + 4 * RS);   // [RS][CST] codes
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q = warp >> 1;                 // window
-  const int lrow = (warp & 1) * 32 + lane;  // row within the CTA
   pdl_launch_dependents();
   pdl_wait();
   if (status_bad(st)) return;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * RS;
   const int rows_here = static_cast<int>(std::min<int64_t>(RS, out - row0));
-  for (int idx = tid; idx < B * B; idx += QT) Us[idx] = Ub[idx];
-  for (int j = tid; j < B; j += QT) inv_u[j] = j < kb ? 1.0 / Ub[j * B + j] : 0.0;
+
+  // ---- 1. loads
+  for (int idx = tid; idx < B * B / 2; idx += QT) cp_async16(Us + 2 * idx, Ub + 2 * idx);
   for (int idx = tid; idx < RS * B; idx += QT) {
     const int r = idx >> 7, c = idx & (B - 1);
-    Wr[r * LDW + c] = (r < rows_here && c < kb) ? acc[(row0 + r) * in + b + c] : 0.0;
+    if (r < rows_here && c < kb)
+      cp_async8(Wr + r * LDW + c, acc + (row0 + r) * in + b + c);
+    else
+      Wr[r * LDW + c] = 0.0;
   }
+  cp_async_wait_all();
   __syncthreads();
-  {  // W_G = W0_G + acc_G U_GG
-    const int ty = tid >> 4, tx = tid & 15;
-    double o[4][8];
+  if (tid < B) inv_u[tid] = tid < kb ? 1.0 / Us[tid * B + tid] : 0.0;
+
+  // ---- 2. W_G = W0_G + acc_G U_GG (k <= c)
+  {
+    const int qd[4] = {warp, 15 - warp, 16 + warp, 31 - warp};  // ascending
+    double o[2][4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) o[i][c] = 0.0;
-    for (int k = 0; k < kb; ++k) {
-      double a[4], u[8];
+      for (int s = 0; s < 4; ++s)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = Wr[(4 * ty + i) * LDW + k];
+        for (int c = 0; c < 4; ++c) o[h][s][c] = 0.0;
+    const double* wa = Wr + lane * LDW;
+    const double* wb = Wr + (lane + 32) * LDW;
+    int k = 0;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) u[c] = Us[k * B + tx + 16 * c];
+    for (int s0 = 0; s0 < 4; ++s0) {  // quads s0..3 still take k
+      const int kend = 4 * qd[s0] + 4;
+      for (; k < kend; ++k) {
+        const double a0 = wa[k], a1 = wb[k];
+        const double* urow = Us + k * B;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int s = s0; s < 4; ++s) {
+          const double2 u01 = *reinterpret_cast<const double2*>(urow + 4 * qd[s]);
+          const double2 u23 = *reinterpret_cast<const double2*>(urow + 4 * qd[s] + 2);
+          const double u[4] = {u01.x, u01.y, u23.x, u23.y};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) o[i][c] = fma(a[i], u[c], o[i][c]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = 4 * ty + i;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int col = tx + 16 * c;
-        double w = 0.0;
-        if (r < rows_here && col < kb)
-          w = static_cast<double>(W0[(row0 + r) * in + b + col]) + o[i][c];
-        Wr[r * LDW + col] = w;
+          for (int c = 0; c < 4; ++c) {
+            o[0][s][c] = fma(a0, u[c], o[0][s][c]);
+            o[1][s][c] = fma(a1, u[c], o[1][s][c]);
+          }
+        }
       }
+    }
+    __syncthreads();  // every read of acc_G is done
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      const bool rv = r < rows_here;
+      const float* w0r = W0 + (row0 + r) * in + b;
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = 4 * qd[s] + c;
+          Wr[r * LDW + col] =
+              (rv && col < kb) ? static_cast<double>(w0r[col]) + o[h][s][c] : 0.0;
+        }
     }
   }
   __syncthreads();
 
+  // ---- 3. the row scale
   const bool asym = qzero != nullptr;
   const int qmax = (1 << (bits - 1)) - 1;
   const double fqmax = asym ? static_cast<double>((1 << bits) - 1) : static_cast<double>(qmax);
   const int64_t ngroups = (in + g - 1) / g;
+  const int q = warp >> 1;                  // window
+  const int lrow = (warp & 1) * 32 + lane;  // row within the CTA
   const int64_t row = row0 + lrow;
   const bool valid = lrow < rows_here;
   double* wrow = Wr + lrow * LDW;
+  const int c0 = SUB * q;
+  double ws[SUB];
+  {
+    double m = 0.0, m2 = 0.0;
+#pragma unroll
+    for (int k = 0; k < SUB; ++k) {
+      ws[k] = wrow[c0 + k];  // zero past kb
+      m = fmax(m, asym ? ws[k] : fabs(ws[k]));
+      m2 = fmin(m2, ws[k]);
+    }
+    mx[q * RS + lrow] = m;
+    mn[q * RS + lrow] = m2;
+  }
+  __syncthreads();
   if (q == 0) {
-    // the row's scale: a group starts here (its whole width is this block when
-    // g == 128) unless it was taken beforehand or continues from earlier
+    // a group starts here (its whole width is this block when g == 128)
+    // unless its scale was taken beforehand, or it continues from earlier
     double sc, z = 0.0;
     if (b % g == 0 && !scale_given) {
-      double m = 0.0, mn = 0.0;
-      for (int c = 0; c < kb; ++c) {
-        const double v = wrow[c];
-        m = fmax(m, asym ? v : fabs(v));
-        mn = fmin(mn, v);
-      }
+      const double m = fmax(fmax(mx[lrow], mx[RS + lrow]), fmax(mx[2 * RS + lrow], mx[3 * RS + lrow]));
+      const double m2 = fmin(fmin(mn[lrow], mn[RS + lrow]), fmin(mn[2 * RS + lrow], mn[3 * RS + lrow]));
       if (!asym) {
         sc = m / fqmax;
       } else {
-        sc = (m - mn) / fqmax;
-        z = sc > 0.0 ? rint(-mn / sc) : 0.0;
+        sc = (m - m2) / fqmax;
+        z = sc > 0.0 ? rint(-m2 / sc) : 0.0;
         z = fmin(fmax(z, 0.0), fqmax);
         if (valid) qzero[row * ngroups + b / g] = static_cast<uint8_t>(z);
       }
@@ -381,95 +452,113 @@ __global__ void __launch_bounds__(QT, 1)
     scale_s[lrow] = sc;
     zero_s[lrow] = z;
   }
-  const int c0 = SUB * q;
-  double ws[SUB];
-#pragma unroll
-  for (int k = 0; k < SUB; ++k) ws[k] = wrow[c0 + k];
   __syncthreads();
-  const double sc = scale_s[lrow];
-  const double rsc = sc > 0.0 ? 1.0 / sc : 0.0;
-  const double cmin = asym ? -zero_s[lrow] : -static_cast<double>(qmax) - 1.0;
-  const double cmax = asym ? fqmax - zero_s[lrow] : static_cast<double>(qmax);
-  int8_t* crow = Cs + lrow * B;
 
-  for (int p = 0; p < 4; ++p) {
-    if (q >= p && SUB * p < kb) {
-      if (p > 0) {
-        const int cp = SUB * (p - 1);
+  // ---- 4. the serial column loop
+  {
+    const double sc = scale_s[lrow];
+    const double rsc = sc > 0.0 ? 1.0 / sc : 0.0;
+    const double cmin = asym ? -zero_s[lrow] : -static_cast<double>(qmax) - 1.0;
+    const double cmax = asym ? fqmax - zero_s[lrow] : static_cast<double>(qmax);
+    int8_t* crow = Cs + lrow * CST;
+    for (int p = 0; p < 4; ++p) {
+      if (q >= p && SUB * p < kb) {
+        if (p > 0) {
+          const int cp = SUB * (p - 1);
 #pragma unroll 4
-        for (int t = 0; t < SUB; ++t) {
-          const double ev = wrow[cp + t];
-          const double* urow = Us + (cp + t) * B + c0;
+          for (int t = 0; t < SUB; ++t) {
+            const double ev = wrow[cp + t];
+            const double* urow = Us + (cp + t) * B + c0;
 #pragma unroll
-          for (int k = 0; k < SUB; ++k) ws[k] = fma(-ev, urow[k], ws[k]);
-        }
-      }
-      if (q == p) {
-#pragma unroll
-        for (int jj = 0; jj < SUB; ++jj) {
-          const int j = c0 + jj;
-          if (j < kb) {
-            const double wj = ws[jj];
-            const double qv = sc > 0.0 ? fmin(fmax(code64(wj, sc, rsc), cmin), cmax) : 0.0;
-            const double err = (wj - qv * sc) * inv_u[j];
-            crow[j] = static_cast<int8_t>(qv);
-            ws[jj] = err;
-#pragma unroll
-            for (int k = jj + 1; k < SUB; ++k) ws[k] = fma(-err, Us[j * B + c0 + k], ws[k]);
+            for (int k = 0; k < SUB; ++k) ws[k] = fma(-ev, urow[k], ws[k]);
           }
         }
+        if (q == p) {
 #pragma unroll
-        for (int k = 0; k < SUB; ++k) wrow[c0 + k] = ws[k];
+          for (int k = 0; k < SUB; ++k) wrow[c0 + k] = ws[k];  // the state, for a redo
+          bool near = false;
+#pragma unroll
+          for (int jj = 0; jj < SUB; ++jj) {
+            const int j = c0 + jj;
+            if (j < kb) {
+              const double wj = ws[jj];
+              const double t = wj * rsc;
+              const double r = rint(t);
+              near |= fabs(fabs(t - r) - 0.5) < 1e-12 * fmax(1.0, fabs(t));
+              const double qv = sc > 0.0 ? fmin(fmax(r, cmin), cmax) : 0.0;
+              const double err = (wj - qv * sc) * inv_u[j];
+              crow[j] = static_cast<int8_t>(qv);
+              ws[jj] = err;
+#pragma unroll
+              for (int k = jj + 1; k < SUB; ++k) ws[k] = fma(-err, Us[j * B + c0 + k], ws[k]);
+            }
+          }
+          if (near) {
+            window_redo64(wrow, Us, inv_u, c0, kb, sc, rsc, cmin, cmax, crow);
+          } else {
+#pragma unroll
+            for (int k = 0; k < SUB; ++k) wrow[c0 + k] = ws[k];
+          }
+        }
       }
+      __syncthreads();
     }
-    __syncthreads();
   }
 
-  // write-out: codes (this thread's 32 columns), W0 - Q, its digits
-  double d0[SUB];
-  double m = 0.0;
-  const float* w0row = W0 + row * in + b + c0;
-#pragma unroll
-  for (int k = 0; k < SUB; ++k) {
-    const int c = c0 + k;
-    double v = 0.0;
-    if (valid && c < kb) {
-      v = static_cast<double>(w0row[k]) - static_cast<double>(crow[c]) * sc;
-      codes[row * in + b + c] = crow[c];
-    }
-    d0[k] = v;
-    m = fmax(m, fabs(v));
-  }
-  maxbuf[q * RS + lrow] = m;
-  __syncthreads();
-  m = fmax(fmax(maxbuf[lrow], maxbuf[RS + lrow]), fmax(maxbuf[2 * RS + lrow], maxbuf[3 * RS + lrow]));
-  if (!valid) return;
-  int ex = 0;
-  if (m > 0.0) frexp(m, &ex);
-  if (q == 0) dex[row] = ex;
-  if (dsb != nullptr) {
-    double* drow = dsb + row * ldsb + c0;
-#pragma unroll
-    for (int k = 0; k < SUB; ++k)
-      if (c0 + k < kb) drow[k] = d0[k];
-  }
-  if (c0 >= dkpad) return;
-  const double sc6 = m > 0.0 ? pow2(6 - ex) : 0.0;
+  // ---- 5. write-out: warp w takes rows w, w+8, ...; lane l columns 4l .. 4l+3
   const int64_t plane = out * dkpad;
-#pragma unroll
-  for (int k4 = 0; k4 < SUB; k4 += 4) {
-    uint32_t w[kMaxDigits] = {};
+  const bool c4_aligned = ((in | b) & 3) == 0 && (reinterpret_cast<uintptr_t>(codes) & 3) == 0;
+  for (int r = warp; r < rows_here; r += QT / 32) {
+    const int64_t grow = row0 + r;
+    const double sc = scale_s[r];
+    const float* w0r = W0 + grow * in + b;
+    const int8_t* cr = Cs + r * CST;
+    double d[4];
+    double m = 0.0;
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      double y = d0[k4 + t] * sc6;  // zero past kb
-      for (int i = 0; i < ds; ++i) {
-        const double di = rint(y);
-        y = (y - di) * 128.0;
-        w[i] |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+      const int c = 4 * lane + t;
+      d[t] = c < kb ? static_cast<double>(w0r[c]) - static_cast<double>(cr[c]) * sc : 0.0;
+      m = fmax(m, fabs(d[t]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    int8_t* cg = codes + grow * in + b;
+    if (c4_aligned && 4 * lane + 3 < kb) {
+      *reinterpret_cast<uint32_t*>(cg + 4 * lane) = *reinterpret_cast<const uint32_t*>(cr + 4 * lane);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (4 * lane + t < kb) cg[4 * lane + t] = cr[4 * lane + t];
+    }
+    if (dsb != nullptr) {
+      double* drow = dsb + grow * ldsb;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (4 * lane + t < kb) drow[4 * lane + t] = d[t];
+    }
+    int ex = 0;
+    if (m > 0.0) frexp(m, &ex);
+    if (lane == 0) dex[grow] = ex;
+    if (4 * lane < dkpad) {
+      const double sc6 = m > 0.0 ? pow2(6 - ex) : 0.0;
+      double y[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) y[t] = d[t] * sc6;
+#pragma unroll
+      for (int i = 0; i < kMaxDigits; ++i) {
+        if (i < ds) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const double di = rint(y[t]);
+            y[t] = (y[t] - di) * 128.0;
+            w |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+          }
+          *reinterpret_cast<uint32_t*>(dq + i * plane + grow * dkpad + 4 * lane) = w;
+        }
       }
     }
-    for (int i = 0; i < ds; ++i)
-      *reinterpret_cast<uint32_t*>(dq + i * plane + row * dkpad + c0 + k4) = w[i];
   }
 }
 
