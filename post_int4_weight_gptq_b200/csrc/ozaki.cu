@@ -47,17 +47,19 @@ namespace piq {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 64;
+constexpr int BN = 48;                        // columns of C per tile
 constexpr int BK = 64;                        // int8 digits = one 64-byte row
 constexpr int A_TILE = BM * BK;               // 8 KB per digit
-constexpr int B_TILE = BN * BK;               // 4 KB per digit
+constexpr int B_TILE = BN * BK;               // 3 KB per digit
 constexpr int THREADS = 192;
 constexpr int MAX_SMEM = 227 * 1024;
+constexpr int BUF_COLS = 256;                 // TMEM columns between the two accumulator sets
+constexpr int STG_LD = BN + 2;                // fp64 staging row stride (16-byte rows, 4-way banks)
+constexpr int STG_BYTES = 4 * (32 * STG_LD + BN) * 8;
 
 struct OzParams {
   int M, N, K, s;
   int m_tiles, n_tiles, num_tiles;
-  int nbuf;             // TMEM accumulator sets (1 or 2)
   int stages;
   int stage_bytes;
   double alpha;
@@ -70,13 +72,16 @@ struct OzParams {
   DeviceStatus* st;
 };
 
+// Column tiles of row tile m that reach the lower triangle: n BN <= 128 m + 127.
+__host__ __device__ __forceinline__ int lower_cols(int m, int n_tiles) {
+  return min(n_tiles, (BM * m + BM - 1) / BN + 1);
+}
+
 __device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& nt) {
   if (p.lower) {
-    // row tile mt holds column tiles 0 .. last(mt) where last = floor((128 mt + 127) / 64)
-    // = 2 mt + 1 (clipped to n_tiles - 1); walk rows (few hundred at most)
-    int acc = 0;
+    int acc = 0;  // walk the row tiles (a few hundred at most)
     for (int m = 0; m < p.m_tiles; ++m) {
-      const int cnt = min(p.n_tiles, 2 * m + 2);
+      const int cnt = lower_cols(m, p.n_tiles);
       if (t < acc + cnt) {
         mt = m;
         nt = t - acc;
@@ -92,9 +97,9 @@ __device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& 
 }
 
 // Instruction descriptor: kind::i8, signed A and B, s32 accumulate, K-major
-// A and B, M = 128, N = 64.
-__host__ __device__ constexpr uint32_t idesc_i8() {
-  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+// A and B, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(BM >> 4) << 24);
 }
 
@@ -110,25 +115,23 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_
 
 constexpr uint32_t kLayoutSw64 = 4;  // smem descriptor: 64-byte swizzle
 
-__device__ __forceinline__ void tmem_ld_i32x32(uint32_t taddr, int (&v)[32]) {
-  float f[32];
-  tmem_ld_32x32b_x32(taddr, f);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __float_as_int(f[i]);
+// 2^e for e well inside the normal range, from the exponent field.
+__device__ __forceinline__ double pow2i(int e) {
+  return __longlong_as_double(static_cast<long long>(1023 + e) << 52);
 }
 
 // S (digits per operand) is a template parameter so that the MMA issue loop
-// (S (S + 1) / 2 digit pairs x 2 MMAs per k block) unrolls into straight-line
-// code with constant descriptor offsets: one thread issues every MMA, and with
-// a runtime loop the issue itself, not the tensor core, set the pace.
+// unrolls into straight-line code with constant descriptors.
 template <int S>
 __global__ void __launch_bounds__(THREADS, 1)
     ozaki_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, OzParams p) {
+  static_assert(S * BN <= 256 && S * BN <= BUF_COLS, "stacked digits exceed one MMA");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * p.stage_bytes);
+  double* stg_all = reinterpret_cast<double*>(smem + p.stages * p.stage_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * p.stage_bytes + STG_BYTES);
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;  // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
@@ -161,7 +164,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_kb = (p.K + BK - 1) / BK;
   pdl_wait();
   const bool skip = status_bad(p.st);
-  constexpr uint32_t set_cols = static_cast<uint32_t>(S * BN);
 
   if (skip) {
   } else if (warp == 0) {
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           uint8_t* sa = smem + st * p.stage_bytes;
-          uint8_t* sb = sa + S * A_TILE;
+          uint8_t* sb = sa + S * A_TILE;  // B digits stacked: one S*BN-row K-major matrix
           mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(p.stage_bytes));
           for (int i = 0; i < S; ++i) {
             tma_load_3d(sa + i * A_TILE, &tmA, &full[st], kb * BK, mt * BM, i);
@@ -192,16 +194,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // --------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = idesc_i8();
+      // Digit i of A against B digits 0 .. S-1-i stacked (N = (S - i) BN) lands
+      // in accumulators i .. S-1, i.e. pair (i, j) in accumulator i + j: one
+      // MMA per A digit and 32-byte k step.
       uint32_t it = 0;
       int lt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++lt) {
-        const int buf = lt % p.nbuf;
-        const uint32_t use = static_cast<uint32_t>(lt / p.nbuf);
+        const int buf = lt & 1;
+        const uint32_t use = static_cast<uint32_t>(lt >> 1);
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, p.st, 42)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf) * set_cols;
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * BUF_COLS);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int st = it % p.stages;
           const uint32_t ph = (it / p.stages) & 1u;
@@ -210,23 +214,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          // descriptors of digit 0 of A and B in this stage; digit i adds
-          // i * tile bytes / 16 to the address field, a k step of 32 bytes adds 2
           const uint32_t a0 = smem_u32(smem + st * p.stage_bytes);
           const uint64_t ad0 = smem_desc(a0, 16, 512, kLayoutSw64);
           const uint64_t bd0 = smem_desc(a0 + S * A_TILE, 16, 512, kLayoutSw64);
 #pragma unroll
-          for (int i = 0; i < S; ++i) {
+          for (int kk = 0; kk < BK / 32; ++kk) {
 #pragma unroll
-            for (int j = 0; i + j < S; ++j) {
-#pragma unroll
-              for (int kk = 0; kk < BK / 32; ++kk) {
-                // the first product into accumulator d of this tile starts it
-                const uint32_t acc = (kb == 0 && kk == 0 && i == 0) ? 0u : 1u;
-                umma_i8(d0 + static_cast<uint32_t>((i + j) * BN),
-                        ad0 + static_cast<uint64_t>(i * (A_TILE >> 4) + kk * 2),
-                        bd0 + static_cast<uint64_t>(j * (B_TILE >> 4) + kk * 2), idesc, acc);
-              }
+            for (int i = 0; i < S; ++i) {
+              // digit 0 of A covers every accumulator: it starts the tile
+              const uint32_t acc = (kb == 0 && kk == 0 && i == 0) ? 0u : 1u;
+              umma_i8(d0 + static_cast<uint32_t>(i * BN),
+                      ad0 + static_cast<uint64_t>(i * (A_TILE >> 4) + kk * 2),
+                      bd0 + static_cast<uint64_t>(kk * 2), idesc_i8((S - i) * BN), acc);
             }
           }
           umma_commit(&empty[st]);
@@ -236,72 +235,76 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each warp: its 32 rows of the tile (lane = row).  TMEM -> registers,
+    // Horner in powers of 2^-7, times 2^e_A(row) alpha 2^(e_B(col) - 12), into
+    // the lane's row of the warp's staging block; the TMEM buffer goes back
+    // to the MMA issuer; then one asynchronous bulk copy per row adds the row
+    // segment into C in global memory (or stores it when beta = 0), so that
+    // the read-modify-write of C happens at L2 without a round trip through
+    // the SM.  A row whose segment is not 16-byte aligned or has an odd
+    // length finishes with plain accesses.
     const int q = warp & 3;
+    double* stg = stg_all + q * 32 * STG_LD;
+    double* cs = stg_all + 4 * 32 * STG_LD + q * BN;
     int lt = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
       int mt, nt;
       tile_of(p, t, mt, nt);
-      const int buf = lt % p.nbuf;
-      const uint32_t use = static_cast<uint32_t>(lt / p.nbuf);
+      const int buf = lt & 1;
+      const uint32_t use = static_cast<uint32_t>(lt >> 1);
+      const int col0 = nt * BN;
+      const int row = mt * BM + q * 32 + lane;
       if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 44)) break;
       tc_fence_after();
-      const int row = mt * BM + q * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(buf) * set_cols;
-      const int ear = row < p.M ? __ldg(p.ea + row) : 0;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        double v[32];
-        {
-          int a[32];
-          tmem_ld_i32x32(taddr + static_cast<uint32_t>((S - 1) * BN + c * 32), a);
+      bulk_wait_read<0>();  // this lane's earlier bulk copies are done reading its row
+      for (int c = lane; c < BN; c += 32) {
+        const int col = col0 + c;
+        cs[c] = col < p.N ? p.alpha * pow2i(__ldg(p.eb + col) - 12) : 0.0;
+      }
+      __syncwarp();
+      const double rsc = pow2i(row < p.M ? __ldg(p.ea + row) : 0);
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BUF_COLS);
+      double* srow = stg + lane * STG_LD;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = static_cast<double>(a[i]);
-        }
+      for (int c = 0; c < BN / 16; ++c) {
+        double v[16];
+        float f[16];
+        tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>((S - 1) * BN + 16 * c), f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = static_cast<double>(__float_as_int(f[i]));
+#pragma unroll
         for (int d = S - 2; d >= 0; --d) {
-          int a[32];
-          tmem_ld_i32x32(taddr + static_cast<uint32_t>(d * BN + c * 32), a);
+          tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(d * BN + 16 * c), f);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fma(v[i], 0.0078125, static_cast<double>(a[i]));
+          for (int i = 0; i < 16; ++i)
+            v[i] = fma(v[i], 0.0078125, static_cast<double>(__float_as_int(f[i])));
         }
-        const int col0 = nt * BN + c * 32;
-        if (row < p.M && col0 < p.N) {
-          double* crow = p.C + static_cast<int64_t>(row) * p.ldc + col0;
-          const int lim = min(32, p.N - col0);
-          const int clim = p.lower ? min(lim, row - col0 + 1) : lim;  // c <= r
-          // v * alpha * 2^(ea + eb - 12): the power of two built from its
-          // exponent field (the row exponents stay far inside the normal range)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int eb = i < clim ? __ldg(p.eb + col0 + i) : 0;
-            v[i] *= __longlong_as_double(static_cast<long long>(1023 + ear + eb - 12) << 52);
-          }
-          if (clim == 32 && (reinterpret_cast<uintptr_t>(crow) & 15u) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              double2 o = make_double2(p.alpha * v[i], p.alpha * v[i + 1]);
-              if (p.beta) {
-                const double2 old = *reinterpret_cast<const double2*>(crow + i);
-                o.x += old.x;
-                o.y += old.y;
-              }
-              *reinterpret_cast<double2*>(crow + i) = o;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i < clim) {
-                const double val = p.alpha * v[i];
-                crow[i] = p.beta ? crow[i] + val : val;
-              }
-            }
-          }
-        }
+        for (int i = 0; i < 16; ++i) srow[16 * c + i] = (v[i] * rsc) * cs[16 * c + i];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (row < p.M) {
+        int ncol = min(BN, p.N - col0);
+        if (p.lower) ncol = min(ncol, row - col0 + 1);  // c <= r
+        if (ncol > 0) {
+          double* crow = p.C + static_cast<int64_t>(row) * p.ldc + col0;
+          const int nbulk = (reinterpret_cast<uintptr_t>(crow) & 15u) == 0 ? (ncol & ~1) : 0;
+          if (nbulk > 0) {
+            fence_proxy_async_smem();
+            if (p.beta)
+              bulk_reduce_add_f64(crow, srow, static_cast<uint32_t>(nbulk * 8));
+            else
+              bulk_store_global(crow, srow, static_cast<uint32_t>(nbulk * 8));
+            bulk_commit();
+          }
+          for (int c = nbulk; c < ncol; ++c) crow[c] = p.beta ? crow[c] + srow[c] : srow[c];
+        }
+      }
     }
+    bulk_wait_all();
   }
 
   tc_fence_before();
@@ -406,7 +409,7 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
                       int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
                       cudaStream_t stream) {
   if (M <= 0 || N <= 0) return PIQ_OK;
-  if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s < 3 || A.s > 6)
+  if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s < 3 || A.s > 5)
     return PIQ_ERR_INVALID_ARG;
   if (A.kpad * (A.s + 1) >= (int64_t)1 << 19) return PIQ_ERR_INVALID_ARG;  // int32 exactness
   if (M > INT32_MAX || N > INT32_MAX) return PIQ_ERR_INVALID_ARG;
@@ -426,7 +429,7 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
   if (lower) {
     int64_t tot = 0;
-    for (int m = 0; m < p.m_tiles; ++m) tot += std::min<int64_t>(p.n_tiles, 2 * m + 2);
+    for (int m = 0; m < p.m_tiles; ++m) tot += lower_cols(m, p.n_tiles);
     if (tot > INT32_MAX) return PIQ_ERR_INVALID_ARG;
     p.num_tiles = static_cast<int>(tot);
   } else {
@@ -434,9 +437,8 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
     if (tot > INT32_MAX) return PIQ_ERR_INVALID_ARG;
     p.num_tiles = static_cast<int>(tot);
   }
-  p.nbuf = (2 * p.s * BN <= 512) ? 2 : 1;
   p.stage_bytes = p.s * (A_TILE + B_TILE);
-  p.stages = std::min(4, (MAX_SMEM - 1024 - 256) / p.stage_bytes);
+  p.stages = std::min(4, (MAX_SMEM - 1024 - 256 - STG_BYTES) / p.stage_bytes);
   if (p.stages < 2) return PIQ_ERR_INVALID_ARG;
   p.alpha = alpha;
   p.beta = beta ? 1 : 0;
@@ -446,15 +448,15 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
   p.ea = A.ex;
   p.eb = B.ex;
   p.st = st;
-  // at least half an SM's shared memory, so that two CTAs that each hold all
-  // 512 TMEM columns never share an SM
-  const int smem = std::max(p.stages * p.stage_bytes + 1024 + 256, 120 * 1024);
+  // the pipeline stages, the epilogue's staging blocks and the barriers; more
+  // than half an SM's shared memory, so that two CTAs that each hold all 512
+  // TMEM columns never share an SM
+  const int smem = std::max(p.stages * p.stage_bytes + STG_BYTES + 1024 + 256, 120 * 1024);
   void (*kern)(CUtensorMap, CUtensorMap, OzParams) = nullptr;
   switch (p.s) {
     case 3: kern = ozaki_gemm_kernel<3>; break;
     case 4: kern = ozaki_gemm_kernel<4>; break;
     case 5: kern = ozaki_gemm_kernel<5>; break;
-    case 6: kern = ozaki_gemm_kernel<6>; break;
     default: return PIQ_ERR_INVALID_ARG;
   }
   static bool attr_set[64][8] = {};
