@@ -29,13 +29,21 @@
 //
 // Layout: digits are stored K-major, q[i][row][kpad] int8 with kpad a multiple
 // of 64 (zero padded), and the exponents e[row] int32.  Tiles: 128 rows of A x
-// 64 rows of B, K in blocks of 64 bytes (64-byte swizzle); a pipeline stage
-// holds all s digit tiles of A and of B for one k block.  TMEM holds the s
-// accumulators side by side (s * 64 columns), double-buffered when s <= 4.
+// 48 rows of B, K in blocks of 64 bytes (64-byte swizzle); a pipeline stage
+// holds all s digit tiles of A and of B for one k block, the B tiles one
+// after another so that they read as a single K-major matrix of s * 48 rows.
+// TMEM holds the s accumulators of a tile side by side (accumulator d at
+// column 48 d), two tiles' worth (double-buffered).  Digit i of A times the
+// stacked B digits 0 .. s-1-i is one MMA of N = 48 (s - i) whose output
+// columns are exactly accumulators i .. s-1, i.e. pair (i, j) lands in
+// accumulator i + j: s MMAs per 32-byte k step instead of s (s + 1) / 2 narrow
+// ones, which halves the shared-memory operand reads that bound the tensor
+// pipe at narrow N.
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 lane 0
-// issues the MMAs; warps 2..5 drain TMEM (warp w reads lanes 32 (w % 4) ..)
-// and own 32 rows of C each.  Every wait is bounded; no multicast loads.
+// issues the MMAs; warps 2..5 drain TMEM (warp w reads lanes 32 (w % 4) ..),
+// own 32 rows of C each, and add them into C with asynchronous bulk
+// reduce-adds from shared memory.  Every wait is bounded; no multicast loads.
 #include <cuda.h>
 
 #include <algorithm>
