@@ -62,13 +62,42 @@ struct S64Params {
   DeviceStatus* st;
 };
 
-// Tile t -> (mt, nt) with mt <= nt, column panel by column panel.
-__device__ __forceinline__ void tile_of(int t, int& mt, int& nt) {
-  int b = static_cast<int>((sqrtf(8.f * static_cast<float>(t) + 1.f) - 1.f) * 0.5f);
-  while ((b + 1) * (b + 2) / 2 <= t) ++b;
-  while (b * (b + 1) / 2 > t) --b;
-  nt = b;
-  mt = t - b * (b + 1) / 2;
+// Tile t -> (mt, nt) with mt <= nt.  The upper triangle of tiles is walked in
+// super-blocks of G x G tiles (super-column by super-column; inside a
+// super-column the blocks above the diagonal, then the diagonal one), row by
+// row inside a block.  One wave of persistent CTAs (148 tiles) then covers
+// about one super-block, i.e. 2 G column blocks of X, each read from HBM once
+// and shared by G tiles through L2; column panel by column panel a wave would
+// touch ~150 column blocks and use each once.
+constexpr int kSuperTile = 12;
+
+__device__ __forceinline__ void tile_of(int t, int T, int& mt, int& nt) {
+  constexpr int G = kSuperTile;
+  int acc = 0;
+  for (int J = 0; J * G < T; ++J) {
+    const int c = min(G, T - J * G);  // tile columns of super-column J
+    const int above = c * G * J;      // tiles of its blocks above the diagonal
+    const int cnt = above + c * (c + 1) / 2;
+    if (t < acc + cnt) {
+      int li = t - acc;
+      if (li < above) {
+        const int I = li / (G * c);
+        const int r = li - I * G * c;
+        mt = I * G + r / c;
+        nt = J * G + r % c;
+      } else {
+        li -= above;
+        int b = static_cast<int>((sqrtf(8.f * static_cast<float>(li) + 1.f) - 1.f) * 0.5f);
+        while ((b + 1) * (b + 2) / 2 <= li) ++b;
+        while (b * (b + 1) / 2 > li) --b;
+        mt = J * G + (li - b * (b + 1) / 2);
+        nt = J * G + b;
+      }
+      return;
+    }
+    acc += cnt;
+  }
+  mt = nt = 0;
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -116,7 +145,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         int mt, nt;
-        tile_of(t, mt, nt);
+        tile_of(t, p.tiles_1d, mt, nt);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -183,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
       int mt, nt;
-      tile_of(t, mt, nt);
+      tile_of(t, p.tiles_1d, mt, nt);
       const int row0 = mt * BM + q * 32;
       const int colh = nt * BN + h * 64;
       // a 32-column slab wholly below the diagonal is never stored
