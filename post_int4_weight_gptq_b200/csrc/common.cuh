@@ -66,14 +66,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One bounded test of the phase: with a suspend-time hint the thread sleeps
+// until the phase completes or about kSuspendNs pass, instead of spinning and
+// taking issue slots from the warps that do the work.
+constexpr uint32_t kSuspendNs = 20000u;  // 20 us
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -89,13 +93,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Device
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   const uint64_t lim = (st != nullptr && st->wait_ns != 0) ? st->wait_ns : kWaitLimitNs;
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (global_timer_ns() - t0 > lim) {
-        set_status(st, PIQ_ERR_TIMEOUT, where);
-        return false;
-      }
+    if (global_timer_ns() - t0 > lim) {
+      set_status(st, PIQ_ERR_TIMEOUT, where);
+      return false;
     }
   }
 }

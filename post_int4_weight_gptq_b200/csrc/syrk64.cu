@@ -25,7 +25,7 @@
 // triangle of H as fp64 (entries below the diagonal inside diagonal tiles are
 // written too; nothing reads them).
 //
-// Warp roles (320 threads): warp 0 lane 0 issues TMA loads into a 6-stage ring;
+// Warp roles (320 threads): warp 0 lane 0 issues TMA loads into a 7-stage ring;
 // warp 1 lane 0 issues the MMAs; warps 2..9 drain one of two 128-column TMEM
 // accumulators (warp w reads lanes 32 (w % 4) .. and columns 64 ((w - 2) / 4) ..)
 // while the MMA warp fills the other.  Every wait is bounded; no multicast loads.
@@ -43,7 +43,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 6;
+constexpr int STAGES = 7;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
@@ -52,6 +52,7 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int NBUF = 4;  // TMEM accumulators (two chunk pairs)
 constexpr int TMEM_COLS = NBUF * BN;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+static_assert(SMEM_BYTES <= 227 * 1024, "pipeline exceeds shared memory");
 constexpr int KC = 128;  // samples per TMEM accumulation
 constexpr int KB_CHUNK = KC / BK;
 
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [NBUF]
   uint64_t* acc_empty = acc_full + NBUF;  // [NBUF]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NBUF);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   pdl_launch_dependents();
