@@ -114,14 +114,15 @@ __device__ __forceinline__ double x_lower(const double* S, const double* xd, int
 
 // Join step 1: T[i][j] = sum_k L[cC + i][cA + k] X[cA + k][cA + j] (k >= j),
 // for the thread's outputs i = ti + 16 x, j = tj + js y; T row-major, stride m.
-template <int MX, int NY>
-__device__ __forceinline__ void join_t(const double* S, const double* xd, double* T, int m,
-                                       int cA, int cC, int ti, int tj, int js) {
+template <int MX, int NY, int m>
+__device__ __forceinline__ void join_t(const double* S, const double* xd, double* T, int cA,
+                                       int cC, int ti, int tj, int js) {
   double acc[MX][NY];
 #pragma unroll
   for (int x = 0; x < MX; ++x)
 #pragma unroll
     for (int y = 0; y < NY; ++y) acc[x][y] = 0.0;
+#pragma unroll 4
   for (int k = tj & ~1; k < m; ++k) {  // warp-uniform start; X[k][j] = 0 below j
     double a[MX], bv[NY];
 #pragma unroll
@@ -141,14 +142,15 @@ __device__ __forceinline__ void join_t(const double* S, const double* xd, double
 
 // Join step 2: X[cC + i][cA + j] = -sum_k X[cC + i][cC + k] T[k][j] (k <= i),
 // stored transposed at S[cA + j][cC + i].
-template <int MX, int NY>
-__device__ __forceinline__ void join_x(double* S, const double* xd, const double* T, int m,
-                                       int cA, int cC, int ti, int tj, int js) {
+template <int MX, int NY, int m>
+__device__ __forceinline__ void join_x(double* S, const double* xd, const double* T, int cA,
+                                       int cC, int ti, int tj, int js) {
   double acc[MX][NY];
 #pragma unroll
   for (int x = 0; x < MX; ++x)
 #pragma unroll
     for (int y = 0; y < NY; ++y) acc[x][y] = 0.0;
+#pragma unroll 4
   for (int k = 0; k < m; ++k) {
     double a[MX], bv[NY];
 #pragma unroll
@@ -298,15 +300,15 @@ __global__ void __launch_bounds__(CT, 1)
   {
     const int half = tid >> 8, t = tid & 255;
     const int cA = 64 * half, cC = cA + 32;
-    join_t<2, 2>(S, xd, Tb + half * 32 * 32, 32, cA, cC, t & 15, t >> 4, 16);
+    join_t<2, 2, 32>(S, xd, Tb + half * 32 * 32, cA, cC, t & 15, t >> 4, 16);
     __syncthreads();
-    join_x<2, 2>(S, xd, Tb + half * 32 * 32, 32, cA, cC, t & 15, t >> 4, 16);
+    join_x<2, 2, 32>(S, xd, Tb + half * 32 * 32, cA, cC, t & 15, t >> 4, 16);
     __syncthreads();
   }
   // ---- join halves (64 -> 128)
-  join_t<4, 2>(S, xd, Tb, 64, 0, 64, tid & 15, tid >> 4, 32);
+  join_t<4, 2, 64>(S, xd, Tb, 0, 64, tid & 15, tid >> 4, 32);
   __syncthreads();
-  join_x<4, 2>(S, xd, Tb, 64, 0, 64, tid & 15, tid >> 4, 32);
+  join_x<4, 2, 64>(S, xd, Tb, 0, 64, tid & 15, tid >> 4, 32);
   __syncthreads();
 
   for (int idx = tid; idx < NB * NB; idx += CT) {

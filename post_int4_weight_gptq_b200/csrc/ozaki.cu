@@ -346,19 +346,26 @@ __global__ void slice_rows_kernel(const double* __restrict__ src, int64_t rs, in
   const int64_t plane = rows * kpad;
   // four consecutive k per lane per step: one 32-bit store per digit
   for (int64_t k0 = 4 * lane; k0 < kpad; k0 += 128) {
-    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    double y[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const int64_t k = k0 + t;
-      double y = (k < K && m > 0.0) ? row[k * ks] * sc6 : 0.0;  // |y| < 64
-      for (int i = 0; i < s; ++i) {
-        const double di = rint(y);
-        y = (y - di) * 128.0;
-        w[i] |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+      y[t] = (k < K && m > 0.0) ? row[k * ks] * sc6 : 0.0;  // |y| < 64
+    }
+    // digit by digit (the digit index is unrolled, so nothing is indexed at run time)
+#pragma unroll
+    for (int i = 0; i < kMaxDigits; ++i) {
+      if (i < s) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const double di = rint(y[t]);
+          y[t] = (y[t] - di) * 128.0;
+          w |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+        }
+        *reinterpret_cast<uint32_t*>(q + i * plane + r * kpad + k0) = w;
       }
     }
-    for (int i = 0; i < s; ++i)
-      *reinterpret_cast<uint32_t*>(q + i * plane + r * kpad + k0) = w[i];
   }
 }
 
@@ -383,17 +390,16 @@ EncodeTiledFn encode_fn_i8() {
 }
 
 // int8 digit planes [s][rows][kpad] as a 3-D map {kpad, rows, s}, box {64, box_rows, 1}.
-bool make_digit_map(CUtensorMap* map, const int8_t* q, int64_t rows, int64_t kpad, int s,
-                    uint32_t box_rows) {
+bool make_digit_map(CUtensorMap* map, const DigitMat& d, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn_i8();
   if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kpad), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(s)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kpad),
-                                 static_cast<cuuint64_t>(rows * kpad)};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.kpad), static_cast<cuuint64_t>(d.rows),
+                              static_cast<cuuint64_t>(d.s)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.kpad),
+                                 static_cast<cuuint64_t>(d.rows * d.kpad)};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(q), dims, strides, box,
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(d.q), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -425,8 +431,7 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
   int rc = device_info(&info);
   if (rc != PIQ_OK) return rc;
   CUtensorMap ma, mb;
-  if (!make_digit_map(&ma, A.q, A.rows, A.kpad, A.s, BM) ||
-      !make_digit_map(&mb, B.q, B.rows, B.kpad, B.s, BN))
+  if (!make_digit_map(&ma, A, BM) || !make_digit_map(&mb, B, BN))
     return PIQ_ERR_INVALID_ARG;
   OzParams p{};
   p.M = static_cast<int>(M);
