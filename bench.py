@@ -333,7 +333,8 @@ def run_reference(args):
 def time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps, warmup, world, local,
                sample_clocks=True):
     """Device-timed steps of one layer (inputs resident in HBM): (ms per step,
-    mean phase times, launches per step, clocks, last output, last shifted error)."""
+    mean phase times, launches per step, fallbacks, clocks, last output, last
+    shifted error, mean digit-GEMM stats per step)."""
     stream = torch.cuda.current_stream()
 
     def step():
@@ -355,6 +356,7 @@ def time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps, warmup, wo
         time.sleep(0.3)
     piq.set_timing(True)
     phases = {}
+    gemm = []
     l0 = piq.kernel_launches()
     f0 = piq.simt_gemm_fallbacks()
     barrier(world)
@@ -366,6 +368,7 @@ def time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps, warmup, wo
         o, e2 = step()
         for k, v in piq.last_phase_times().items():
             phases.setdefault(k, []).append(v)
+        gemm.append(piq.last_gemm_stats())
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -381,7 +384,8 @@ def time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps, warmup, wo
         clocks = sampler.summary(t_wall0, t_wall1)
     ms = max_over_ranks(ms, world)
     ph = {k: statistics.mean(v) for k, v in phases.items()}
-    return ms / steps, ph, launches, fallbacks, clocks, o, e2
+    gs = {k: statistics.mean(g[k] for g in gemm) for k in ("ms", "int8_ops", "launches")}
+    return ms / steps, ph, launches, fallbacks, clocks, o, e2, gs
 
 
 def alloc_layer(piq, torch, spec, n, dev, with_shift):
@@ -416,7 +420,7 @@ def run_ours(args):
     X2g = to_gpu_x(X2, dev) if X2 is not None else None
     ws, ws_err, res = alloc_layer(piq, torch, spec, n, dev, X2 is not None)
 
-    ms_step, ph, launches, fallbacks, clocks, o, e2 = time_layer(
+    ms_step, ph, launches, fallbacks, clocks, o, e2, gs = time_layer(
         piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, args.steps, args.warmup, world, local)
     value = world * out_rows * inp / (ms_step / 1e3) / 1e6
 
@@ -464,19 +468,20 @@ def run_ours(args):
     bf16_peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     phase_roof = phase_rooflines(ph, out_rows, inp, n, bf16_peak, hbm_peak)
-    dom = max(phase_roof, key=lambda k: phase_roof[k]["ms"])
-    d = phase_roof[dom]
-    roof = {"kernel": {"hessian": "syrk64 (tcgen05 bf16 H = X^T X, FP64 chunk sums)",
-                       "factor": "FP64-grade Cholesky (chol64 diagonal blocks + ozaki_gemm "
-                                 "INT8 tensor-core panel products)",
-                       "sweep": "FP64 sweep (sweep64) + ozaki_gemm block updates",
-                       "pack": "pack", "error": "err_dot (bf16x3 through H)"}[dom],
-            "phase": dom, "bound": "hbm" if d["unit"] == "GB/s" else "tensor",
-            "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
-            "traffic": args.traffic, "ms_per_launch": d["ms"],
-            "peak_source": f"{peak_src} {peak_key}" + (
-                "; FP64-grade products: nominal INT8 = 2 x bf16, over the digit products"
-                if "FP64" in d["unit"] else "")}
+    # the dominant kernel: the INT8 digit GEMM (FP64-grade products of the factor
+    # and the sweep), timed per launch with CUDA events inside the timed steps;
+    # its algorithmic work is 2 K per computed entry of C per digit pair
+    int8_peak = INT8_PER_BF16 * bf16_peak
+    g_tops = gs["int8_ops"] / (gs["ms"] / 1e3) / 1e12 if gs["ms"] > 0 else float("nan")
+    roof = {"kernel": "ozaki_gemm_kernel<5> (INT8 digit products of the FP64-grade factor "
+                      "and sweep; 48-wide tiles, stacked digits, tcgen05 kind::i8)",
+            "bound": "tensor", "achieved": g_tops, "peak": int8_peak, "unit": "TOP/s (INT8)",
+            "frac": g_tops / int8_peak, "traffic": args.traffic,
+            "ms_per_step": gs["ms"], "share_of_step": gs["ms"] / ms_step,
+            "launches_per_step": gs["launches"],
+            "ms_per_launch": gs["ms"] / gs["launches"] if gs["launches"] else None,
+            "int8_ops_per_launch": gs["int8_ops"] / gs["launches"] if gs["launches"] else None,
+            "peak_source": f"{peak_src} {peak_key} x {INT8_PER_BF16:g} (nominal INT8 : BF16)"}
     ph_h = ph.get("hessian", float("nan"))
     xtx = float(n) * inp * (inp + 1) / (ph_h / 1e3) / 1e12
 
@@ -532,7 +537,7 @@ def run_second(piq, torch, dev, workload, steps=10, warmup=3):
     Wg, Xg = to_gpu_w(W, dev), to_gpu_x(X, dev)
     X2g = to_gpu_x(X2, dev) if X2 is not None else None
     ws, ws_err, res = alloc_layer(piq, torch, spec, X.shape[0], dev, X2 is not None)
-    ms, ph, _, _, _, o, e2 = time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps,
+    ms, ph, _, _, _, o, e2, _ = time_layer(piq, torch, Wg, Xg, X2g, spec, ws, ws_err, res, steps,
                                         warmup, 1, 0, sample_clocks=False)
     r = {"workload": workload_config(spec, X.shape[0], workload)["workload"],
          "ms_per_layer": ms, "mweights_per_s": spec.out * spec.inp / (ms / 1e3) / 1e6,

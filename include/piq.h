@@ -279,6 +279,12 @@ int piq_layer_output_error(const float* W, int64_t out, int64_t in, const uint32
 int piq_set_timing(int enable);
 int piq_last_phase_times(double* ms, int max_phases, int* n_phases);
 const char* piq_phase_name(int i);
+/* With timing on, the same call also records an event pair around every launch
+ * of the INT8 digit GEMM (the FP64-grade products of the factor and the sweep):
+ * *ms = their summed device time, *int8_ops = their algorithmic INT8 operations
+ * (2 K per computed entry of C per digit pair, K padded to 64), *launches = the
+ * number of launches.  Any pointer may be NULL.  Host-side state, per process. */
+int piq_last_gemm_stats(double* ms, double* int8_ops, int* launches);
 
 /* Number of kernels this library has launched in this process (all devices);
  * a monotone diagnostic counter. */

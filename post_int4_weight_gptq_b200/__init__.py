@@ -90,6 +90,8 @@ SIGNATURES = {
     "piq_last_phase_times": (_c_int, [ctypes.POINTER(ctypes.c_double), _c_int,
                                       ctypes.POINTER(_c_int)]),
     "piq_phase_name": (ctypes.c_char_p, [_c_int]),
+    "piq_last_gemm_stats": (_c_int, [ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
     "piq_kernel_launches": (ctypes.c_uint64, []),
     "piq_simt_gemm_fallbacks": (ctypes.c_uint64, []),
     "piq_last_cuda_error": (ctypes.c_char_p, []),
@@ -423,6 +425,15 @@ def last_phase_times() -> dict:
     n = ctypes.c_int(0)
     lib.piq_last_phase_times(buf, 8, ctypes.byref(n))
     return {lib.piq_phase_name(i).decode(): buf[i] for i in range(min(n.value, 8))}
+
+
+def last_gemm_stats() -> dict:
+    """With timing on: the INT8 digit GEMM launches of the last timed call,
+    {"ms": summed device time, "int8_ops": algorithmic operations, "launches": n}."""
+    lib = load_library()
+    ms, ops, n = ctypes.c_double(0.0), ctypes.c_double(0.0), ctypes.c_int(0)
+    lib.piq_last_gemm_stats(ctypes.byref(ms), ctypes.byref(ops), ctypes.byref(n))
+    return {"ms": ms.value, "int8_ops": ops.value, "launches": n.value}
 
 
 def kernel_launches() -> int:

@@ -120,9 +120,43 @@ struct Timing {
   double last_ms[kMaxPhases] = {};
   int last_n = 0;
   int last_kind = 0;
+  // digit GEMM launches of the current call: event pairs and their work
+  bool in_call = false;
+  std::vector<cudaEvent_t> gev;  // 2 per slot, created on demand
+  std::vector<double> gops;
+  int gn = 0;
+  double last_gemm_ms = 0.0, last_gemm_ops = 0.0;
+  int last_gemm_n = 0;
 };
 Timing g_timing;
 std::mutex g_timing_mu;
+constexpr int kMaxGemmSlots = 8192;
+
+}  // namespace
+
+int gemm_timing_begin(cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (!g_timing.enabled || !g_timing.in_call || g_timing.gn >= kMaxGemmSlots) return -1;
+  const int slot = g_timing.gn;
+  while (static_cast<int>(g_timing.gev.size()) < 2 * (slot + 1)) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    g_timing.gev.push_back(e);
+  }
+  if (static_cast<int>(g_timing.gops.size()) <= slot) g_timing.gops.resize(slot + 1);
+  if (cudaEventRecord(g_timing.gev[2 * slot], stream) != cudaSuccess) return -1;
+  ++g_timing.gn;
+  return slot;
+}
+
+void gemm_timing_end(int slot, cudaStream_t stream, double int8_ops) {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  cudaEventRecord(g_timing.gev[2 * slot + 1], stream);
+  g_timing.gops[slot] = int8_ops;
+}
+
+namespace {
 
 struct PhaseClock {
   bool on;
@@ -137,6 +171,8 @@ struct PhaseClock {
       g_timing.created = true;
     }
     g_timing.kind = kind;
+    g_timing.in_call = true;
+    g_timing.gn = 0;
     on = true;
     cudaEventRecord(g_timing.ev[0], s);
   }
@@ -154,6 +190,18 @@ struct PhaseClock {
     }
     g_timing.last_n = idx;
     g_timing.last_kind = g_timing.kind;
+    double gms = 0.0, gops = 0.0;
+    for (int i = 0; i < g_timing.gn; ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, g_timing.gev[2 * i], g_timing.gev[2 * i + 1]);
+      gms += ms;
+      gops += g_timing.gops[i];
+    }
+    g_timing.last_gemm_ms = gms;
+    g_timing.last_gemm_ops = gops;
+    g_timing.last_gemm_n = g_timing.gn;
+    g_timing.in_call = false;
+    g_timing.gn = 0;
   }
 };
 
@@ -760,6 +808,14 @@ int piq_last_phase_times(double* ms, int max_phases, int* n_phases) {
   const int n = std::min(max_phases, g_timing.last_n);
   for (int i = 0; i < n; ++i) ms[i] = g_timing.last_ms[i];
   if (n_phases) *n_phases = g_timing.last_n;
+  return PIQ_OK;
+}
+
+int piq_last_gemm_stats(double* ms, double* int8_ops, int* launches) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (ms) *ms = g_timing.last_gemm_ms;
+  if (int8_ops) *int8_ops = g_timing.last_gemm_ops;
+  if (launches) *launches = g_timing.last_gemm_n;
   return PIQ_OK;
 }
 

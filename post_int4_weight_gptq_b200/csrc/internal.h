@@ -131,6 +131,11 @@ struct DigitMat {
   int64_t rows = 0, kpad = 0;
   int s = 0;
 };
+// Per-launch timing of the digit GEMM while phase timing is on: begin
+// records an event before the launch and returns a slot (-1 when off), end
+// records one after it with the launch's algorithmic INT8 operations.
+int gemm_timing_begin(cudaStream_t stream);
+void gemm_timing_end(int slot, cudaStream_t stream, double int8_ops);
 int64_t digit_kpad(int64_t K);  // K rounded up to a multiple of 64
 // Digits of the rows x K matrix whose entry (r, k) is src[r * rs + k * ks]
 // (strides may be negative); out->rows, kpad and s must match.

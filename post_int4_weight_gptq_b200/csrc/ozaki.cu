@@ -325,46 +325,78 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ----------------------------------------------------------------- digits
 // Row r of the logical rows x K matrix: element (r, k) at src[r * rs + k * ks].
-// One warp per row: pass 1 finds the largest magnitude, pass 2 writes the s
-// digits of every entry (zeros for k in [K, kpad)).
+// One warp per row, lane l holding entries 4 l .. 4 l + 3 of each 128-entry
+// chunk.  Rows of up to 128 CH entries are read once into registers (every
+// load issued before any is used), their largest magnitude found by a warp
+// reduction, and the s digits of every entry written from the registers
+// (zeros for k in [K, kpad)); longer rows take two passes.
+template <int S>
+__device__ __forceinline__ void write_digits4(const double (&x)[4], double sc6, int8_t* q,
+                                              int64_t plane, int64_t off) {
+  double y[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) y[t] = x[t] * sc6;  // |y| < 64
+#pragma unroll
+  for (int i = 0; i < S; ++i) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const double di = rint(y[t]);
+      y[t] = (y[t] - di) * 128.0;
+      w |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
+    }
+    *reinterpret_cast<uint32_t*>(q + i * plane + off) = w;
+  }
+}
+
+template <int S, int CH>
 __global__ void slice_rows_kernel(const double* __restrict__ src, int64_t rs, int64_t ks,
-                                  int64_t rows, int64_t K, int s, int8_t* __restrict__ q,
-                                  int64_t kpad, int* __restrict__ ex) {
+                                  int64_t rows, int64_t K, int8_t* __restrict__ q, int64_t kpad,
+                                  int* __restrict__ ex) {
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
   const double* row = src + r * rs;
+  const int64_t plane = rows * kpad;
+  const int64_t nch = (kpad + 127) / 128;
   double m = 0.0;
-  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(row[k * ks]));
+  double x[CH][4];
+  if (nch <= CH) {
+#pragma unroll
+    for (int c = 0; c < CH; ++c)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int64_t k = 128 * c + 4 * lane + t;
+        x[c][t] = (c < nch && k < K) ? row[k * ks] : 0.0;
+      }
+#pragma unroll
+    for (int c = 0; c < CH; ++c)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) m = fmax(m, fabs(x[c][t]));
+  } else {
+    for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(row[k * ks]));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
   int e = 0;
   if (m > 0.0) frexp(m, &e);  // m = f 2^e with f in [0.5, 1)
   if (lane == 0) ex[r] = e;
-  // 2^(6 - e) from its exponent field (row maxima stay far inside the normal range)
-  const double sc6 = __longlong_as_double(static_cast<long long>(1023 + 6 - e) << 52);
-  const int64_t plane = rows * kpad;
-  // four consecutive k per lane per step: one 32-bit store per digit
-  for (int64_t k0 = 4 * lane; k0 < kpad; k0 += 128) {
-    double y[4];
+  // 2^(6 - e) from its exponent field (row maxima stay far inside the normal range);
+  // an all-zero row gets zero digits
+  const double sc6 =
+      m > 0.0 ? __longlong_as_double(static_cast<long long>(1023 + 6 - e) << 52) : 0.0;
+  if (nch <= CH) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int64_t k = k0 + t;
-      y[t] = (k < K && m > 0.0) ? row[k * ks] * sc6 : 0.0;  // |y| < 64
+    for (int c = 0; c < CH; ++c) {
+      const int64_t k0 = 128 * c + 4 * lane;
+      if (c < nch && k0 < kpad) write_digits4<S>(x[c], sc6, q, plane, r * kpad + k0);
     }
-    // digit by digit (the digit index is unrolled, so nothing is indexed at run time)
+  } else {
+    for (int64_t k0 = 4 * lane; k0 < kpad; k0 += 128) {
+      double v[4];
 #pragma unroll
-    for (int i = 0; i < kMaxDigits; ++i) {
-      if (i < s) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const double di = rint(y[t]);
-          y[t] = (y[t] - di) * 128.0;
-          w |= (static_cast<uint32_t>(static_cast<int>(di)) & 0xFFu) << (8 * t);
-        }
-        *reinterpret_cast<uint32_t*>(q + i * plane + r * kpad + k0) = w;
-      }
+      for (int t = 0; t < 4; ++t) v[t] = (k0 + t < K) ? row[(k0 + t) * ks] : 0.0;
+      write_digits4<S>(v, sc6, q, plane, r * kpad + k0);
     }
   }
 }
@@ -413,9 +445,22 @@ int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_
   if (rows < 1 || K < 1 || s < 1 || s > kMaxDigits) return PIQ_ERR_INVALID_ARG;
   if (out->kpad != digit_kpad(K) || out->s != s || out->rows != rows) return PIQ_ERR_INVALID_ARG;
   const int64_t threads = rows * 32;
+  const unsigned grid = static_cast<unsigned>(ceil_div(threads, 256));
+  void (*kern)(const double*, int64_t, int64_t, int64_t, int64_t, int8_t*, int64_t, int*) = nullptr;
+  const bool short_row = out->kpad <= 128;
+  switch (s) {
+    case 1: kern = short_row ? slice_rows_kernel<1, 1> : slice_rows_kernel<1, 8>; break;
+    case 2: kern = short_row ? slice_rows_kernel<2, 1> : slice_rows_kernel<2, 8>; break;
+    case 3: kern = short_row ? slice_rows_kernel<3, 1> : slice_rows_kernel<3, 8>; break;
+    case 4: kern = short_row ? slice_rows_kernel<4, 1> : slice_rows_kernel<4, 8>; break;
+    case 5: kern = short_row ? slice_rows_kernel<5, 1> : slice_rows_kernel<5, 8>; break;
+    case 6: kern = short_row ? slice_rows_kernel<6, 1> : slice_rows_kernel<6, 8>; break;
+    case 7: kern = short_row ? slice_rows_kernel<7, 1> : slice_rows_kernel<7, 8>; break;
+    default: break;
+  }
+  if (kern == nullptr) return PIQ_ERR_INVALID_ARG;
   note_launch();
-  slice_rows_kernel<<<static_cast<unsigned>(ceil_div(threads, 256)), 256, 0, stream>>>(
-      src, rs, ks, rows, K, s, out->q, out->kpad, out->ex);
+  kern<<<grid, 256, 0, stream>>>(src, rs, ks, rows, K, out->q, out->kpad, out->ex);
   return launch_ok("digit split launch") ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
@@ -482,10 +527,17 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
     attr_set[dev][p.s] = true;
   }
   const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
+  // algorithmic work: 2 K operations per computed entry of C and digit pair
+  double entries = static_cast<double>(M) * static_cast<double>(N);
+  if (lower)
+    entries = (N <= M) ? static_cast<double>(N) * (N + 1) / 2 + static_cast<double>(M - N) * N
+                       : static_cast<double>(M) * (M + 1) / 2;
+  const int slot = gemm_timing_begin(stream);
   note_launch();
   if (launch_pdl(kern, dim3(grid), dim3(THREADS), static_cast<size_t>(smem), stream, ma, mb, p) !=
       cudaSuccess)
     return PIQ_ERR_CUDA;
+  gemm_timing_end(slot, stream, 2.0 * entries * static_cast<double>(p.K) * p.s * (p.s + 1) / 2);
   return launch_ok() ? PIQ_OK : PIQ_ERR_CUDA;
 }
 
