@@ -26,7 +26,8 @@ stated in the function's docstring.
 from .gptq import (GPTQResult, act_order_perm_ref, block_partition_ref, damped_ref,
                    gptq_prepare_ref, gptq_ref, gptq_ref_blocked, gptq_sweep_asym_ref,
                    gptq_sweep_blocked_asym_ref, gptq_sweep_blocked_ref, gptq_sweep_ref,
-                   group_quantizer_ref, hessian_ref, rtn_asym_ref, rtn_ref, upper_factor_ref)
+                   group_quantizer_ref, hessian_ref, hessian_syrk_ref, rtn_asym_ref, rtn_ref,
+                   upper_factor_r_ref, upper_factor_ref)
 from .awq import AWQResult, awq_ref, awq_scales_ref, channel_mean_abs_ref, group_rtn_ref
 from .pack import dequant_ref, g_idx_ref, pack_asym_ref, pack_ref, unpack_ref
 from .error import output_error_ref, x_to_f64
@@ -36,7 +37,7 @@ __all__ = [
     "GPTQResult", "act_order_perm_ref", "block_partition_ref", "damped_ref",
     "gptq_prepare_ref", "gptq_ref", "gptq_ref_blocked", "gptq_sweep_ref", "hessian_ref",
     "gptq_sweep_blocked_ref", "gptq_sweep_blocked_asym_ref",
-    "rtn_ref", "upper_factor_ref", "gptq_sweep_asym_ref", "group_quantizer_ref", "rtn_asym_ref",
+    "rtn_ref", "upper_factor_ref", "upper_factor_r_ref", "hessian_syrk_ref", "gptq_sweep_asym_ref", "group_quantizer_ref", "rtn_asym_ref",
     "pack_asym_ref", "AWQResult", "awq_ref", "awq_scales_ref",
     "channel_mean_abs_ref", "group_rtn_ref", "dequant_ref", "g_idx_ref", "pack_ref",
     "unpack_ref", "output_error_ref", "x_to_f64", "awq_gptq_dequant_ref", "awq_gptq_ref",

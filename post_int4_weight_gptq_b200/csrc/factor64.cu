@@ -399,6 +399,25 @@ constexpr int kCholSmem64 = (NB * LDS + PW * NB) * 8;
 
 }  // namespace
 
+// A non-blocking stream and two events for one call's look-ahead, released
+// when the call returns (work already enqueued completes first).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t cols = nullptr, diag = nullptr;
+  int open() {
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&cols, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&diag, cudaEventDisableTiming) != cudaSuccess)
+      return cuda_rc(cudaGetLastError());
+    return PIQ_OK;
+  }
+  ~SideStream() {
+    if (diag) cudaEventDestroy(diag);
+    if (cols) cudaEventDestroy(cols);
+    if (s) cudaStreamDestroy(s);
+  }
+};
+
 struct Factor64Ws {
   double* P;
   double* X11;
@@ -472,14 +491,46 @@ int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, v
   }
   if (!launch_ok()) return PIQ_ERR_CUDA;
 
+  // Look-ahead: each trailing update is split into the next panel's columns
+  // and the rest; once the next panel's columns are done, its diagonal block
+  // (one SM) is factored on a side stream while the rest of the update runs
+  // on the caller's stream, one SM short.  Two events carry the order both
+  // ways; the side stream and the events live for this call only.
+  DeviceInfo info;
+  int rc = device_info(&info);
+  if (rc != PIQ_OK) return rc;
+  SideStream side;
+  rc = side.open();
+  if (rc != PIQ_OK) return rc;
+  const int rest_ctas = std::max(1, info.sm_count - 1);
+  bool diag_pending = false;  // the current panel's diagonal block runs on the side stream
+  auto diag_on_side = [&](int64_t k, int nbk) -> int {
+    int r = cuda_rc(cudaEventRecord(side.cols, stream));
+    if (r == PIQ_OK) r = cuda_rc(cudaStreamWaitEvent(side.s, side.cols, 0));
+    if (r != PIQ_OK) return r;
+    note_launch();
+    if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kCholSmem64, side.s, P, ld, k, nbk,
+                   X11, st) != cudaSuccess)
+      return PIQ_ERR_CUDA;
+    r = cuda_rc(cudaEventRecord(side.diag, side.s));
+    if (r == PIQ_OK) diag_pending = true;
+    return r;
+  };
+
   for (int64_t s0 = 0; s0 < in; s0 += kSuperPanel) {
     const int64_t s1 = std::min<int64_t>(s0 + kSuperPanel, in);
     for (int64_t k0 = s0; k0 < s1; k0 += NB) {
       const int nb = static_cast<int>(std::min<int64_t>(NB, in - k0));
-      note_launch();
-      if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kCholSmem64, stream, P, ld, k0, nb,
-                     X11, st) != cudaSuccess)
-        return PIQ_ERR_CUDA;
+      if (diag_pending) {
+        rc = cuda_rc(cudaStreamWaitEvent(stream, side.diag, 0));
+        if (rc != PIQ_OK) return rc;
+        diag_pending = false;
+      } else {
+        note_launch();
+        if (launch_pdl(chol64_block_kernel, dim3(1), dim3(CT), kCholSmem64, stream, P, ld, k0,
+                       nb, X11, st) != cudaSuccess)
+          return PIQ_ERR_CUDA;
+      }
       const int64_t rem = in - k0 - nb;
       if (rem <= 0) continue;
       double* A21 = P + (k0 + nb) * ld + k0;
@@ -487,29 +538,51 @@ int run_factor64(const double* H, int64_t in, float damp, const int32_t* perm, v
       dA.rows = rem;
       dX.rows = nb;
       dA.kpad = dX.kpad = digit_kpad(nb);
-      int rc = launch_slice(A21, ld, 1, rem, nb, kFactorDigits, &dA, stream);
+      rc = launch_slice(A21, ld, 1, rem, nb, kFactorDigits, &dA, stream);
       if (rc == PIQ_OK) rc = launch_slice(X11, NB, 1, nb, nb, kFactorDigits, &dX, stream);
       if (rc == PIQ_OK) rc = launch_ozaki_gemm(rem, nb, dA, dX, 1.0, 0, 0, A21, ld, st, stream);
-      // this panel's update of the superpanel's later columns, every row below:
-      // A[k0+nb:, k0+nb:s1] -= L21 L21[:s1-k0-nb]^T (c <= r)
-      const int64_t ncol = s1 - (k0 + nb);
       if (rc == PIQ_OK) rc = launch_slice(A21, ld, 1, rem, nb, kFactorDigits, &dA, stream);
-      if (rc == PIQ_OK && ncol > 0)
-        rc = launch_ozaki_gemm(rem, ncol, dA, dA, -1.0, 1, 1, P + (k0 + nb) * ld + (k0 + nb), ld,
-                               st, stream);
       if (rc != PIQ_OK) return rc;
+      // this panel's update of the superpanel's later columns, every row below:
+      // A[k0+nb:, k0+nb:s1] -= L21 L21[:s1-k0-nb]^T (c <= r); the next panel's
+      // columns first, then its diagonal block beside the rest
+      const int64_t nx = k0 + nb;
+      const int64_t ncol = s1 - nx;
+      if (ncol > 0) {
+        const int nb2 = static_cast<int>(std::min<int64_t>(NB, ncol));
+        rc = launch_ozaki_gemm(rem, nb2, dA, dA, -1.0, 1, 1, P + nx * ld + nx, ld, st, stream);
+        if (rc == PIQ_OK) rc = diag_on_side(nx, nb2);
+        if (rc == PIQ_OK && ncol > nb2) {
+          const DigitMat v = dA.rows_from(nb2, rem - nb2);
+          rc = launch_ozaki_gemm(rem - nb2, ncol - nb2, v, v, -1.0, 1, 1,
+                                 P + (nx + nb2) * ld + (nx + nb2), ld, st, stream, rest_ctas);
+        }
+        if (rc != PIQ_OK) return rc;
+      }
     }
-    // the superpanel's update of the rest: A[s1:, s1:] -= L[s1:, s0:s1] L[s1:, s0:s1]^T
+    // the superpanel's update of the rest: A[s1:, s1:] -= L[s1:, s0:s1] L[s1:, s0:s1]^T,
+    // the next panel's columns first, then its diagonal block beside the rest
     const int64_t rest = in - s1;
     if (rest > 0) {
       DigitMat dS = fw.dS;
       dS.rows = rest;
       dS.kpad = digit_kpad(s1 - s0);
-      int rc = launch_slice(P + s1 * ld + s0, ld, 1, rest, s1 - s0, kFactorDigits, &dS, stream);
+      rc = launch_slice(P + s1 * ld + s0, ld, 1, rest, s1 - s0, kFactorDigits, &dS, stream);
+      const int nb2 = static_cast<int>(std::min<int64_t>(NB, rest));
       if (rc == PIQ_OK)
-        rc = launch_ozaki_gemm(rest, rest, dS, dS, -1.0, 1, 1, P + s1 * ld + s1, ld, st, stream);
+        rc = launch_ozaki_gemm(rest, nb2, dS, dS, -1.0, 1, 1, P + s1 * ld + s1, ld, st, stream);
+      if (rc == PIQ_OK) rc = diag_on_side(s1, nb2);
+      if (rc == PIQ_OK && rest > nb2) {
+        const DigitMat v = dS.rows_from(nb2, rest - nb2);
+        rc = launch_ozaki_gemm(rest - nb2, rest - nb2, v, v, -1.0, 1, 1,
+                               P + (s1 + nb2) * ld + (s1 + nb2), ld, st, stream, rest_ctas);
+      }
       if (rc != PIQ_OK) return rc;
     }
+  }
+  if (diag_pending) {
+    rc = cuda_rc(cudaStreamWaitEvent(stream, side.diag, 0));
+    if (rc != PIQ_OK) return rc;
   }
   {
     const unsigned nt = static_cast<unsigned>(ceil_div(in, 32));

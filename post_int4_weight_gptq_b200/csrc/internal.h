@@ -130,6 +130,16 @@ struct DigitMat {
   int* ex = nullptr;
   int64_t rows = 0, kpad = 0;
   int s = 0;
+  int64_t plane = 0;  // bytes between digit planes (0: rows * kpad, a matrix of its own)
+  // rows [r0, r0 + n) of this matrix, the planes of the whole one
+  DigitMat rows_from(int64_t r0, int64_t n) const {
+    DigitMat v = *this;
+    v.q = q + r0 * kpad;
+    v.ex = ex + r0;
+    v.rows = n;
+    v.plane = plane ? plane : rows * kpad;
+    return v;
+  }
 };
 // Per-launch timing of the digit GEMM while phase timing is on: begin
 // records an event before the launch and returns a slot (-1 when off), end
@@ -145,7 +155,7 @@ int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_
 // beta 0 stores, 1 adds; lower != 0 touches only c <= r.
 int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B, double alpha,
                       int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
-                      cudaStream_t stream);
+                      cudaStream_t stream, int max_ctas = 0);
 
 // ---------------------------------------------- FP64-grade factor (factor64.cu)
 // L = chol(J H_p J + lambda I) in fp64 (lower, row-major [in][in] inside

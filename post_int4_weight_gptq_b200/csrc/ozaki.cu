@@ -428,7 +428,7 @@ bool make_digit_map(CUtensorMap* map, const DigitMat& d, uint32_t box_rows) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.kpad), static_cast<cuuint64_t>(d.rows),
                               static_cast<cuuint64_t>(d.s)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.kpad),
-                                 static_cast<cuuint64_t>(d.rows * d.kpad)};
+                                 static_cast<cuuint64_t>(d.plane ? d.plane : d.rows * d.kpad)};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(d.q), dims, strides, box,
@@ -444,6 +444,7 @@ int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_
                  DigitMat* out, cudaStream_t stream) {
   if (rows < 1 || K < 1 || s < 1 || s > kMaxDigits) return PIQ_ERR_INVALID_ARG;
   if (out->kpad != digit_kpad(K) || out->s != s || out->rows != rows) return PIQ_ERR_INVALID_ARG;
+  if (out->plane != 0 && out->plane != rows * out->kpad) return PIQ_ERR_INVALID_ARG;  // no views
   const int64_t threads = rows * 32;
   const unsigned grid = static_cast<unsigned>(ceil_div(threads, 256));
   void (*kern)(const double*, int64_t, int64_t, int64_t, int64_t, int8_t*, int64_t, int*) = nullptr;
@@ -466,7 +467,7 @@ int launch_slice(const double* src, int64_t rs, int64_t ks, int64_t rows, int64_
 
 int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B, double alpha,
                       int beta, int lower, double* C, int64_t ldc, DeviceStatus* st,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, int max_ctas) {
   if (M <= 0 || N <= 0) return PIQ_OK;
   if (A.s != B.s || A.kpad != B.kpad || A.rows < M || B.rows < N || A.s < 3 || A.s > 5)
     return PIQ_ERR_INVALID_ARG;
@@ -526,7 +527,9 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
       return PIQ_ERR_CUDA;
     attr_set[dev][p.s] = true;
   }
-  const int grid = std::max(1, std::min(p.num_tiles, info.sm_count));
+  // max_ctas > 0 leaves SMs free for work on another stream
+  const int ctas = max_ctas > 0 ? std::min(max_ctas, info.sm_count) : info.sm_count;
+  const int grid = std::max(1, std::min(p.num_tiles, ctas));
   // algorithmic work: 2 K operations per computed entry of C and digit pair
   double entries = static_cast<double>(M) * static_cast<double>(N);
   if (lower)

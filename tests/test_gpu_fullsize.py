@@ -42,8 +42,11 @@ def _layer(spec):
         _cache.clear()  # one large layer at a time
         W = make_weight(spec)
         X = make_x_bits(spec)
-        H = O.hessian_ref(X)
-        perm, U, _ = O.gptq_prepare_ref(H, spec.damp, spec.act_order)
+        # the symmetric rank-k H and U = inv(R): the same matrices as the
+        # listing's product and cholesky(inv(H_d)).T, in fewer host flops
+        # (pinned in test_oracle_properties)
+        H = O.hessian_syrk_ref(X)
+        perm, U, _ = O.gptq_prepare_ref(H, spec.damp, spec.act_order, via_r=True)
         del H
         _cache[spec.name] = (W, X, perm, U)
     return _cache[spec.name]
@@ -93,7 +96,6 @@ def test_down_proj_7b_act_order_full():
     _gptq_full(C3)
 
 
-@pytest.mark.skipif(not SLOW, reason="minutes of host float64; PIQ_FULLSIZE_SLOW=1")
 @pytest.mark.parametrize("bits", [4, 3])
 def test_down_proj_70b_full(bits):
     # W 8192x28672, X 32768x28672, H 28672^2 (3.29 GB in fp32)

@@ -6,6 +6,7 @@ the factorisation's error identity, blocked = literal, a diagonal Hessian
 reducing to rounding, and s = 1 reducing the composition to plain GPTQ.
 """
 import numpy as np
+import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
 
@@ -156,3 +157,28 @@ def test_sweep_identity_on_r():
     acc = (W - Q)[:, :b] @ R[:b, b:]
     Wb = W[:, b:] + acc @ np.linalg.inv(R[b:, b:])
     assert np.allclose(v[:, b] * scales[:, b // 64], Wb[:, 0], rtol=0, atol=1e-9)
+
+
+def test_syrk_hessian_equals_the_product():
+    # the BLAS symmetric rank-k route to H = X^T X against the plain product,
+    # over a chunk boundary and a ragged width (bf16 bit patterns as inputs)
+    rng = np.random.default_rng(41)
+    X = (rng.standard_normal((2500, 131)) * rng.lognormal(0.0, 1.0, 131)).astype(np.float32)
+    Xb = (X.view(np.uint32) >> 16).astype(np.uint16)
+    H1 = O.hessian_ref(Xb)
+    H2 = O.hessian_syrk_ref(Xb, chunk=1000)
+    assert np.array_equal(H2, H2.T)
+    assert np.abs(H1 - H2).max() <= 1e-13 * np.abs(H1).max()
+
+
+@pytest.mark.parametrize("n", [1, 2, 7, 130])
+def test_r_route_factor_equals_the_listing(n):
+    # U = inv(R) with R = J chol(J H_d J) J is the listing's cholesky(inv(H_d)).T
+    rng = np.random.default_rng(n)
+    A = rng.standard_normal((n + 5, n))
+    Hd, _ = O.damped_ref(A.T @ A, 0.01)
+    U1 = O.upper_factor_ref(Hd)
+    U2 = O.upper_factor_r_ref(Hd)
+    assert np.array_equal(np.tril(U2, -1), np.zeros_like(U2))
+    assert (np.abs(U1 - U2) / np.abs(np.diag(U1))[:, None]).max() < 1e-12
+    assert np.abs(U2.T @ U2 @ Hd - np.eye(n)).max() < 1e-10
