@@ -27,6 +27,7 @@ import oracle as O
 import post_int4_weight_gptq_b200 as piq
 from oracle.gptq import gptq_sweep_blocked_ref
 from oracle.pack import dequant_ref
+from tests.oracle_pool import sweep_rows
 from tests.parity import REL_TOL, rel, teacher_forced_compare, to_gpu_w, to_gpu_x, unpack_gpu
 from workloads import AWQ_GRID, C2, C3, C4, C5, make_weight, make_x_bits
 
@@ -69,7 +70,7 @@ def _gptq_full(spec, bits=None, shift=False):
     assert np.array_equal(out.perm.cpu().numpy(), perm)
     assert np.array_equal(out.g_idx.cpu().numpy(), O.g_idx_ref(perm, spec.g))
     Wp = W.astype(np.float64)[:, perm]
-    ref = gptq_sweep_blocked_ref(Wp, U, bits, spec.g)
+    ref = sweep_rows(Wp, U, bits, spec.g)  # all rows, chunks on the host cores
     stats, c_ref, s_ref = teacher_forced_compare(codes_mem[:, perm], Wp, U, bits, spec.g,
                                                  ref=ref)
     s16 = s_ref.astype(np.float16).astype(np.float64)

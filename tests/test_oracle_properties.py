@@ -182,3 +182,23 @@ def test_r_route_factor_equals_the_listing(n):
     assert np.array_equal(np.tril(U2, -1), np.zeros_like(U2))
     assert (np.abs(U1 - U2) / np.abs(np.diag(U1))[:, None]).max() < 1e-12
     assert np.abs(U2.T @ U2 @ Hd - np.eye(n)).max() < 1e-10
+
+
+def test_row_chunks_sweep_like_one_call():
+    # rows are independent given U: the pooled sweep over chunks of rows
+    # (tests/oracle_pool.py, used at full size) gives one call's codes, and its
+    # scales and quotients up to the rounding order of the block products
+    from oracle.gptq import gptq_sweep_blocked_ref
+    from tests.oracle_pool import sweep_rows
+    rng = np.random.default_rng(8)
+    W = rng.standard_normal((70, 300)) * 0.02
+    A = rng.standard_normal((320, 300))
+    Hd, _ = O.damped_ref(A.T @ A, 0.01)
+    U = O.upper_factor_r_ref(Hd)
+    one = gptq_sweep_blocked_ref(W, U, 4, 128)
+    for workers in (1, 2):
+        codes, scales, v = sweep_rows(W, U, 4, 128, chunk=32, workers=workers)
+        assert np.array_equal(codes, one[0])
+        # the BLAS block products may round in another order for another row count
+        assert np.abs(scales - one[1]).max() <= 1e-12 * np.abs(one[1]).max()
+        assert np.abs(v - one[2]).max() <= 1e-12 * np.abs(one[2]).max()
