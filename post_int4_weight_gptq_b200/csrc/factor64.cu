@@ -22,6 +22,8 @@
 //      inverses of R's diagonal blocks for the sweep (block_inverse_kernel)
 // A non-positive pivot sets PIQ_ERR_NOT_PD.
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -399,12 +401,35 @@ constexpr int kCholSmem64 = (NB * LDS + PW * NB) * 8;
 
 }  // namespace
 
-// A non-blocking stream and two events for one call's look-ahead, released
-// when the call returns (work already enqueued completes first).
+// A non-blocking stream and two events for one call's look-ahead.  They are
+// taken from a per-device pool and returned when the call's work is enqueued
+// (creating and destroying them per call costs host time the GPU then spends
+// idle); a call that reuses them records its own events before waiting on
+// them, and stream order keeps any earlier work on the side stream first.
+struct SideHandles {
+  cudaStream_t s = nullptr;
+  cudaEvent_t cols = nullptr, diag = nullptr;
+};
+std::mutex g_side_mu;
+std::vector<SideHandles> g_side_free[64];
+
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t cols = nullptr, diag = nullptr;
+  int dev = -1;
   int open() {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PIQ_ERR_CUDA;
+    {
+      std::lock_guard<std::mutex> lock(g_side_mu);
+      if (!g_side_free[dev].empty()) {
+        const SideHandles h = g_side_free[dev].back();
+        g_side_free[dev].pop_back();
+        s = h.s;
+        cols = h.cols;
+        diag = h.diag;
+        return PIQ_OK;
+      }
+    }
     if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&cols, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&diag, cudaEventDisableTiming) != cudaSuccess)
@@ -412,9 +437,14 @@ struct SideStream {
     return PIQ_OK;
   }
   ~SideStream() {
-    if (diag) cudaEventDestroy(diag);
-    if (cols) cudaEventDestroy(cols);
-    if (s) cudaStreamDestroy(s);
+    if (s == nullptr || cols == nullptr || diag == nullptr) {
+      if (diag) cudaEventDestroy(diag);
+      if (cols) cudaEventDestroy(cols);
+      if (s) cudaStreamDestroy(s);
+      return;
+    }
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    g_side_free[dev].push_back(SideHandles{s, cols, diag});
   }
 };
 

@@ -26,29 +26,45 @@ namespace {
 
 // ------------------------------------------------------------------- colstats
 // grid (ceil(in/256), splits); 8 warps; lane owns 8 consecutive columns.
+// SQ = 0: sum |x| per column, two rows added in FP32 (round to nearest) before
+// each FP64 addition (relative error below 2^-24 of the sum, for the AWQ
+// channel means); SQ = 1: sum x^2 per column, every square (exact in FP32 for
+// bf16 inputs) added in FP64, so the act-order ranking sees exact sums.
+template <int SQ>
 __global__ void __launch_bounds__(256) colstats_kernel(const uint16_t* __restrict__ X, int64_t n,
                                                        int64_t in, int splits,
                                                        double* __restrict__ part) {
-  __shared__ double sh_abs[8][256];
-  __shared__ double sh_sq[8][256];
+  __shared__ double sh[8][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t col = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
   const int64_t rows_per = (n + splits - 1) / splits;
   const int64_t r0 = blockIdx.y * rows_per;
   const int64_t r1 = std::min<int64_t>(n, r0 + rows_per);
-  double sa[8], sq[8];
+  double acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sa[i] = sq[i] = 0.0;
-  auto add = [&](const uint4 v) {
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  auto term = [](uint16_t b) {
+    const float x = bf16_bits_to_float(b);
+    return SQ ? x * x : fabsf(x);
+  };
+  // one row: every term to FP64
+  auto add1 = [&](const uint4 v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float lo = bf16_bits_to_float(static_cast<uint16_t>(w[i] & 0xFFFFu));
-      const float hi = bf16_bits_to_float(static_cast<uint16_t>(w[i] >> 16));
-      sa[2 * i] += static_cast<double>(fabsf(lo));
-      sa[2 * i + 1] += static_cast<double>(fabsf(hi));
-      sq[2 * i] += static_cast<double>(lo * lo);  // exact: bf16 square fits fp32
-      sq[2 * i + 1] += static_cast<double>(hi * hi);
+      acc[2 * i] += static_cast<double>(term(static_cast<uint16_t>(w[i] & 0xFFFFu)));
+      acc[2 * i + 1] += static_cast<double>(term(static_cast<uint16_t>(w[i] >> 16)));
+    }
+  };
+  // two rows: |x| terms summed in FP32 first (SQ = 0 only)
+  auto add2 = [&](const uint4 va, const uint4 vb) {
+    const uint32_t a[4] = {va.x, va.y, va.z, va.w}, b[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += static_cast<double>(__fadd_rn(term(static_cast<uint16_t>(a[i] & 0xFFFFu)),
+                                                  term(static_cast<uint16_t>(b[i] & 0xFFFFu))));
+      acc[2 * i + 1] += static_cast<double>(
+          __fadd_rn(term(static_cast<uint16_t>(a[i] >> 16)), term(static_cast<uint16_t>(b[i] >> 16))));
     }
   };
   if (col < in) {
@@ -59,44 +75,38 @@ __global__ void __launch_bounds__(256) colstats_kernel(const uint16_t* __restric
       const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(X + (r + 8) * in + col));
       const uint4 v2 = __ldg(reinterpret_cast<const uint4*>(X + (r + 16) * in + col));
       const uint4 v3 = __ldg(reinterpret_cast<const uint4*>(X + (r + 24) * in + col));
-      add(v0);
-      add(v1);
-      add(v2);
-      add(v3);
+      if (SQ) {
+        add1(v0);
+        add1(v1);
+        add1(v2);
+        add1(v3);
+      } else {
+        add2(v0, v1);
+        add2(v2, v3);
+      }
     }
-    for (; r < r1; r += 8) add(__ldg(reinterpret_cast<const uint4*>(X + r * in + col)));
+    for (; r < r1; r += 8) add1(__ldg(reinterpret_cast<const uint4*>(X + r * in + col)));
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sh_abs[warp][lane * 8 + i] = sa[i];
-    sh_sq[warp][lane * 8 + i] = sq[i];
-  }
+  for (int i = 0; i < 8; ++i) sh[warp][lane * 8 + i] = acc[i];
   __syncthreads();
   const int c = threadIdx.x;
   const int64_t gc = static_cast<int64_t>(blockIdx.x) * 256 + c;
   if (gc < in) {
-    double a = 0.0, q = 0.0;
+    double a = 0.0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      a += sh_abs[w][c];
-      q += sh_sq[w][c];
-    }
-    part[(static_cast<int64_t>(blockIdx.y) * in + gc) * 2] = a;
-    part[(static_cast<int64_t>(blockIdx.y) * in + gc) * 2 + 1] = q;
+    for (int w = 0; w < 8; ++w) a += sh[w][c];
+    part[static_cast<int64_t>(blockIdx.y) * in + gc] = a;
   }
 }
 
 __global__ void colstats_finish_kernel(const double* __restrict__ part, int64_t n, int64_t in,
-                                       int splits, double* mean_abs, double* sumsq) {
+                                       int splits, int mean, double* out) {
   const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (c >= in) return;
-  double a = 0.0, q = 0.0;
-  for (int s = 0; s < splits; ++s) {
-    a += part[(static_cast<int64_t>(s) * in + c) * 2];
-    q += part[(static_cast<int64_t>(s) * in + c) * 2 + 1];
-  }
-  if (mean_abs) mean_abs[c] = a / static_cast<double>(n);
-  if (sumsq) sumsq[c] = q;
+  double a = 0.0;
+  for (int s = 0; s < splits; ++s) a += part[static_cast<int64_t>(s) * in + c];
+  out[c] = mean ? a / static_cast<double>(n) : a;
 }
 
 // --------------------------------------------------------------------- gather
@@ -222,16 +232,31 @@ __global__ void pack_kernel(const int8_t* __restrict__ codes, const float* __res
         w0[4] *= sb.x; w0[5] *= sb.y; w0[6] *= sb.z; w0[7] *= sb.w;
       }
     }
+    if (invperm == nullptr && (g & 7) == 0) {
+      // natural order, the word inside one group: one 8-byte load of the codes,
+      // one scale (and zero-point) for the word
+      const uint2 cw = *reinterpret_cast<const uint2*>(crow + wd * 8);
+      const int64_t grp = (wd * 8) / g;
+      const int zp = qzero ? static_cast<int>(qzero[r * ngroups + grp]) : off;
+      const float s16 = delta ? __half2float(__float2half_rn(srow[grp])) : 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int64_t c = wd * 8 + k;
-      const int64_t p = invperm ? invperm[c] : c;
-      const int code = crow[p];
-      const int zp = qzero ? static_cast<int>(qzero[r * ngroups + p / g]) : off;
-      word |= static_cast<uint32_t>(code + zp) << (4 * k);
-      if (delta) {
-        const float s16 = __half2float(__float2half_rn(srow[p / g]));
-        d32[k] = w0[k] - static_cast<float>(code) * s16;
+      for (int k = 0; k < 8; ++k) {
+        const int code = static_cast<int8_t>(((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xFFu);
+        word |= static_cast<uint32_t>(code + zp) << (4 * k);
+        if (delta) d32[k] = w0[k] - static_cast<float>(code) * s16;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int64_t c = wd * 8 + k;
+        const int64_t p = invperm ? invperm[c] : c;
+        const int code = crow[p];
+        const int zp = qzero ? static_cast<int>(qzero[r * ngroups + p / g]) : off;
+        word |= static_cast<uint32_t>(code + zp) << (4 * k);
+        if (delta) {
+          const float s16 = __half2float(__float2half_rn(srow[p / g]));
+          d32[k] = w0[k] - static_cast<float>(code) * s16;
+        }
       }
     }
     qweight[idx] = word;
@@ -604,11 +629,19 @@ int colstats_splits(int64_t n, int64_t in) {
 int launch_colstats(const uint16_t* X, int64_t n, int64_t in, double* partials, int splits,
                     double* mean_abs, double* sumsq, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(ceil_div(in, 256)), static_cast<unsigned>(splits));
-  note_launch();
-  colstats_kernel<<<grid, 256, 0, stream>>>(X, n, in, splits, partials);
-  note_launch();
-  colstats_finish_kernel<<<static_cast<unsigned>(ceil_div(in, 256)), 256, 0, stream>>>(
-      partials, n, in, splits, mean_abs, sumsq);
+  const unsigned fgrid = static_cast<unsigned>(ceil_div(in, 256));
+  if (mean_abs) {
+    note_launch();
+    colstats_kernel<0><<<grid, 256, 0, stream>>>(X, n, in, splits, partials);
+    note_launch();
+    colstats_finish_kernel<<<fgrid, 256, 0, stream>>>(partials, n, in, splits, 1, mean_abs);
+  }
+  if (sumsq) {
+    note_launch();
+    colstats_kernel<1><<<grid, 256, 0, stream>>>(X, n, in, splits, partials);
+    note_launch();
+    colstats_finish_kernel<<<fgrid, 256, 0, stream>>>(partials, n, in, splits, 0, sumsq);
+  }
   return last_error();
 }
 
