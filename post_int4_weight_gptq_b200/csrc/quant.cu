@@ -402,20 +402,13 @@ __global__ void __launch_bounds__(256)
 __device__ __noinline__ float code_by_division(float v, float scale) {
   return rintf(__fdiv_rn(v, scale));
 }
-__device__ __forceinline__ float quant_code_rcp(float v, float scale, float rs, float cmin,
-                                                float cmax) {
-  const float t = v * rs;
-  float q = rintf(t);
-  if (fabsf(fabsf(t - q) - 0.5f) < 1e-5f) q = code_by_division(v, scale);  // rare
-  return scale > 0.f ? fminf(fmaxf(q, cmin), cmax) : 0.f;
-}
 
 // D_a[r][c] = W - code * scale / s for every alpha a, for power-of-two g with
 // 8 <= g <= 256 and in % 8 == 0.  Lane l of a warp holds columns 8l .. 8l+7 of a
 // 256-column slice (g / 8 lanes per group) for kRows rows; per alpha the s and
 // 1 / s of its columns are read once for all kRows rows.
 constexpr int kRows = 4;
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
     awq_delta_rows_kernel(const float* __restrict__ W, int64_t out, int64_t in, int bits, int g,
                           const float* __restrict__ s_table, int n_alpha,
                           uint16_t* __restrict__ dW) {
@@ -473,11 +466,28 @@ __global__ void __launch_bounds__(256)
         for (int o = 1; o < lg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const float scale = __fdiv_rn(m, fqmax);
         const float rs = scale > 0.f ? __frcp_rn(scale) : 0.f;
+        // rint(v / scale) from v * (1 / scale); within 1e-5 of a half-integer the
+        // IEEE quotient decides (code_by_division), on one warp-uniform branch
+        float q[8];
+        bool near = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float t = p[e] * rs;
+          q[e] = rintf(t);
+          near |= fabsf(fabsf(t - q[e]) - 0.5f) < 1e-5f;
+        }
+        if (__any_sync(0xffffffffu, near)) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float t = p[e] * rs;
+            if (fabsf(fabsf(t - rintf(t)) - 0.5f) < 1e-5f) q[e] = code_by_division(p[e], scale);
+          }
+        }
         uint16_t d16[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float q = quant_code_rcp(p[e], scale, rs, cmin, cmax);
-          d16[e] = float_to_bf16_bits(fmaf(-(q * scale), iv[e], w[k][e]));
+          const float qc = scale > 0.f ? fminf(fmaxf(q[e], cmin), cmax) : 0.f;
+          d16[e] = float_to_bf16_bits(fmaf(-(qc * scale), iv[e], w[k][e]));
         }
         if (act && r0 + k < out) {
           uint4 o;
