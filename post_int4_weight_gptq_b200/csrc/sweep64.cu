@@ -371,6 +371,7 @@ __global__ void __launch_bounds__(QT, 1)
 #pragma unroll
     for (int s0 = 0; s0 < 4; ++s0) {  // quads s0..3 still take k
       const int kend = 4 * qd[s0] + 4;
+#pragma unroll 4
       for (; k < kend; ++k) {
         const double a0 = wa[k], a1 = wb[k];
         const double* urow = Us + k * B;
