@@ -40,10 +40,11 @@
 // ones, which halves the shared-memory operand reads that bound the tensor
 // pipe at narrow N.
 //
-// Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 lane 0
-// issues the MMAs; warps 2..5 drain TMEM (warp w reads lanes 32 (w % 4) ..),
-// own 32 rows of C each, and add them into C with asynchronous bulk
-// reduce-adds from shared memory.  Every wait is bounded; no multicast loads.
+// Warp roles (320 threads): warp 0 lane 0 issues TMA loads; warp 1 lane 0
+// issues the MMAs; warps 2..9 drain TMEM (warp w reads lanes 32 (w % 4) ..,
+// two warps per lane quadrant, one per 24-column half of the tile), own 32
+// half rows of C each, and add them into C with asynchronous bulk reduce-adds
+// from shared memory.  Every wait is bounded; no multicast loads.
 #include <cuda.h>
 
 #include <algorithm>
@@ -59,11 +60,14 @@ constexpr int BN = 48;                        // columns of C per tile
 constexpr int BK = 64;                        // int8 digits = one 64-byte row
 constexpr int A_TILE = BM * BK;               // 8 KB per digit
 constexpr int B_TILE = BN * BK;               // 3 KB per digit
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;                  // two per TMEM lane quadrant, one per half tile
+constexpr int HALF = BN / 2;                  // columns of C per epilogue warp
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int MAX_SMEM = 227 * 1024;
 constexpr int BUF_COLS = 256;                 // TMEM columns between the two accumulator sets
-constexpr int STG_LD = BN + 2;                // fp64 staging row stride (16-byte rows, 4-way banks)
-constexpr int STG_BYTES = 4 * (32 * STG_LD + BN) * 8;
+constexpr int STG_LD = HALF + 2;              // fp64 staging row stride (16-byte rows, 4-way banks)
+constexpr int STG_WARP = 32 * STG_LD + HALF;  // doubles per epilogue warp: 32 rows + column scales
+constexpr int STG_BYTES = EPI_WARPS * STG_WARP * 8;
 
 struct OzParams {
   int M, N, K, s;
@@ -85,22 +89,68 @@ __host__ __device__ __forceinline__ int lower_cols(int m, int n_tiles) {
   return min(n_tiles, (BM * m + BM - 1) / BN + 1);
 }
 
+// Tiles in row tiles 0 .. m - 1 of a lower launch, in closed form.  With
+// 128 x 48 tiles, row tile i = 3 a + b reaches column tile 8 a + {2, 5, 7}[b],
+// so three consecutive rows hold 24 a + 17 tiles; rows from the first one whose
+// count reaches n_tiles on hold n_tiles each.
+static_assert(BM == 128 && BN == 48, "lower_prefix assumes 128 x 48 tiles");
+__host__ __device__ __forceinline__ int64_t lower_prefix(int m, int n_tiles) {
+  const int64_t x = static_cast<int64_t>(BN) * (n_tiles - 1) - (BM - 1);
+  const int64_t m_full = x > 0 ? (x + BM - 1) / BM : 0;  // first row with n_tiles tiles
+  const int k = static_cast<int>(m < m_full ? m : m_full);
+  const int64_t a = k / 3;
+  const int b = k - 3 * static_cast<int>(a);
+  const int64_t part = b == 0 ? 0 : (b == 1 ? 8 * a + 3 : 16 * a + 9);
+  return 12 * a * (a - 1) + 17 * a + part +
+         (m > m_full ? m - m_full : 0) * static_cast<int64_t>(n_tiles);
+}
+
+// Tile t of the launch.  Tiles run in groups of RG row tiles: inside a group
+// the column tiles are the outer loop, so that a wave of persistent CTAs works
+// on a few column blocks of B for RG row blocks of A and B's digits are read
+// from DRAM once per group rather than once per row tile (at N = 27648 and
+// K = 1024 they are 141 MB, more than L2 keeps).  A lower launch finds its
+// group by bisection on lower_prefix, walks the group's full columns the same
+// way, then its staircase row by row.
+constexpr int RG = 8;
+
 __device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& nt) {
   if (p.lower) {
-    int acc = 0;  // walk the row tiles (a few hundred at most)
-    for (int m = 0; m < p.m_tiles; ++m) {
-      const int cnt = lower_cols(m, p.n_tiles);
-      if (t < acc + cnt) {
+    int lo = 0, hi = (p.m_tiles + RG - 1) / RG - 1;  // the last group g with prefix <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (lower_prefix(mid * RG, p.n_tiles) <= t)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    const int m0 = lo * RG;
+    const int gs = min(RG, p.m_tiles - m0);
+    int r = t - static_cast<int>(lower_prefix(m0, p.n_tiles));
+    const int c0 = lower_cols(m0, p.n_tiles);  // columns every row of the group has
+    if (r < gs * c0) {
+      nt = r / gs;
+      mt = m0 + r - nt * gs;
+      return;
+    }
+    r -= gs * c0;
+    for (int m = m0; m < m0 + gs; ++m) {
+      const int extra = lower_cols(m, p.n_tiles) - c0;
+      if (r < extra) {
         mt = m;
-        nt = t - acc;
+        nt = c0 + r;
         return;
       }
-      acc += cnt;
+      r -= extra;
     }
     mt = nt = 0;
   } else {
-    mt = t / p.n_tiles;
-    nt = t - mt * p.n_tiles;
+    const int full = RG * p.n_tiles;  // tiles of a complete group
+    const int m0 = (t / full) * RG;
+    const int gs = min(RG, p.m_tiles - m0);
+    const int r = t - m0 * p.n_tiles;
+    nt = r / gs;
+    mt = m0 + r - nt * gs;
   }
 }
 
@@ -155,7 +205,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], EPI_WARPS);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -243,59 +293,60 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Each warp: its 32 rows of the tile (lane = row).  TMEM -> registers,
-    // Horner in powers of 2^-7, times 2^e_A(row) alpha 2^(e_B(col) - 12), into
+    // Each warp: the left or right half of 32 rows of the tile (lane = row).
+    // TMEM -> registers, Horner in powers of 2^-7, times 2^e_A(row) alpha 2^(e_B(col) - 12), into
     // the lane's row of the warp's staging block; the TMEM buffer goes back
     // to the MMA issuer; then one asynchronous bulk copy per row adds the row
     // segment into C in global memory (or stores it when beta = 0), so that
     // the read-modify-write of C happens at L2 without a round trip through
     // the SM.  A row whose segment is not 16-byte aligned or has an odd
     // length finishes with plain accesses.
-    const int q = warp & 3;
-    double* stg = stg_all + q * 32 * STG_LD;
-    double* cs = stg_all + 4 * 32 * STG_LD + q * BN;
+    const int q = warp & 3;         // TMEM lanes 32 q .. 32 q + 31: rows of the tile
+    const int h = (warp - 2) >> 2;  // columns h HALF .. h HALF + HALF - 1 of the tile
+    double* stg = stg_all + (warp - 2) * STG_WARP;
+    double* cs = stg + 32 * STG_LD;
     int lt = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++lt) {
       int mt, nt;
       tile_of(p, t, mt, nt);
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
-      const int col0 = nt * BN;
+      const int col0 = nt * BN + h * HALF;
       const int row = mt * BM + q * 32 + lane;
       if (!mbar_wait(&acc_full[buf], use & 1u, p.st, 44)) break;
       tc_fence_after();
       bulk_wait_read<0>();  // this lane's earlier bulk copies are done reading its row
-      for (int c = lane; c < BN; c += 32) {
-        const int col = col0 + c;
-        cs[c] = col < p.N ? p.alpha * pow2i(__ldg(p.eb + col) - 12) : 0.0;
+      if (lane < HALF) {
+        const int col = col0 + lane;
+        cs[lane] = col < p.N ? p.alpha * pow2i(__ldg(p.eb + col) - 12) : 0.0;
       }
       __syncwarp();
       const double rsc = pow2i(row < p.M ? __ldg(p.ea + row) : 0);
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BUF_COLS);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(buf * BUF_COLS + h * HALF);
       double* srow = stg + lane * STG_LD;
 #pragma unroll
-      for (int c = 0; c < BN / 16; ++c) {
-        double v[16];
-        float f[16];
-        tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>((S - 1) * BN + 16 * c), f);
+      for (int c = 0; c < HALF / 8; ++c) {
+        double v[8];
+        float f[8];
+        tmem_ld_32x32b_x8(taddr + static_cast<uint32_t>((S - 1) * BN + 8 * c), f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = static_cast<double>(__float_as_int(f[i]));
+        for (int i = 0; i < 8; ++i) v[i] = static_cast<double>(__float_as_int(f[i]));
 #pragma unroll
         for (int d = S - 2; d >= 0; --d) {
-          tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(d * BN + 16 * c), f);
+          tmem_ld_32x32b_x8(taddr + static_cast<uint32_t>(d * BN + 8 * c), f);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 8; ++i)
             v[i] = fma(v[i], 0.0078125, static_cast<double>(__float_as_int(f[i])));
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) srow[16 * c + i] = (v[i] * rsc) * cs[16 * c + i];
+        for (int i = 0; i < 8; ++i) srow[8 * c + i] = (v[i] * rsc) * cs[8 * c + i];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       if (row < p.M) {
-        int ncol = min(BN, p.N - col0);
+        int ncol = min(HALF, p.N - col0);
         if (p.lower) ncol = min(ncol, row - col0 + 1);  // c <= r
         if (ncol > 0) {
           double* crow = p.C + static_cast<int64_t>(row) * p.ldc + col0;
@@ -487,8 +538,7 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
   p.m_tiles = static_cast<int>(ceil_div(M, BM));
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
   if (lower) {
-    int64_t tot = 0;
-    for (int m = 0; m < p.m_tiles; ++m) tot += lower_cols(m, p.n_tiles);
+    const int64_t tot = lower_prefix(p.m_tiles, p.n_tiles);
     if (tot > INT32_MAX) return PIQ_ERR_INVALID_ARG;
     p.num_tiles = static_cast<int>(tot);
   } else {
