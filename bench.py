@@ -161,6 +161,12 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------- workload
 WORKLOADS = ("down_proj_70b", "q_proj_7b")
+# DRAM bytes (read + write) per launch of the INT8 digit GEMM, averaged over the
+# 864 launches of one down_proj_70b step in an ncu launch-list capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of this bench's own command.  It
+# describes the kernel as it was captured; a changed kernel needs a new capture
+# (or --traffic).
+GEMM_TRAFFIC_PER_LAUNCH = {"down_proj_70b": 1.929e8}
 
 
 def spec_of(name):
@@ -476,7 +482,10 @@ def run_ours(args):
     roof = {"kernel": "ozaki_gemm_kernel<5> (INT8 digit products of the FP64-grade factor "
                       "and sweep; 48-wide tiles, stacked digits, tcgen05 kind::i8)",
             "bound": "tensor", "achieved": g_tops, "peak": int8_peak, "unit": "TOP/s (INT8)",
-            "frac": g_tops / int8_peak, "traffic": args.traffic,
+            "frac": g_tops / int8_peak,
+            "traffic": (args.traffic if args.traffic is not None
+                        else GEMM_TRAFFIC_PER_LAUNCH.get(args.workload)
+                        if args.samples is None else None),
             "ms_per_step": gs["ms"], "share_of_step": gs["ms"] / ms_step,
             "launches_per_step": gs["launches"],
             "ms_per_launch": gs["ms"] / gs["launches"] if gs["launches"] else None,
