@@ -18,6 +18,13 @@ are independent problems (the listing's error feedback never mixes rows).  So:
 The arithmetic of steps 1 and 3 is the library's; this module only moves
 tensors.  The two compute calls are parameters so that the plumbing can be
 exercised on hosts without the GPU library (its tests inject CPU stand-ins).
+
+AWQ splits over the rows of W instead ("GPTQ versus AWQ objectives", AWQ
+paragraph under "A strong answer": s_j = mean|x_j|^alpha depends on the inputs
+only, and the output error of a candidate alpha is a sum over the rows of W):
+every rank holds all of X and scores every alpha on its own rows, one
+all-reduce of n_alpha doubles sums the scores, and every rank takes the same
+first minimum (awq_layer_split).
 """
 from __future__ import annotations
 
@@ -75,3 +82,60 @@ def _gather_rows(t, out, world, group):
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad, group=group)
     return torch.cat([p[:r1 - r0] for p, (r0, r1) in zip(parts, sizes)], dim=0)
+
+
+def first_minimum(errs) -> int:
+    """Index of the smallest error, the first one on a tie (the library's rule)."""
+    best = 0
+    for i in range(1, len(errs)):
+        if errs[i] < errs[best]:
+            best = i
+    return best
+
+
+def awq_layer_split(W, X, group=None, bits=4, g=128, alpha_grid=None, gather=True,
+                    search_fn=None):
+    """AWQ search of the layer W [out, in] with its rows split over the group.
+    Every rank passes the whole W and the whole calibration input X.
+
+      1. each rank scores every alpha on its block of rows (awq_search_layer on
+         W[r0:r1] and X: s is the same on every rank, the errors are this
+         block's shares of the layer's errors);
+      2. one all-reduce sums the n_alpha shares: the only exchange;
+      3. every rank takes the first minimum of the sums; a rank whose own rows
+         preferred another alpha quantizes them again at the chosen one;
+      4. when asked, the packed rows are gathered.
+
+    Returns (best_alpha, s, qweight, scales, err_per_alpha): qweight and scales
+    hold this rank's rows, or all rows when gather is set; err_per_alpha are
+    the layer's errors."""
+    if alpha_grid is None:
+        alpha_grid = tuple(k / 20.0 for k in range(20))
+    alpha_grid = [float(a) for a in alpha_grid]
+    if search_fn is None:
+        import post_int4_weight_gptq_b200 as piq
+        search_fn = lambda Wr, grid: piq.awq_search_layer(Wr, X, bits=bits, g=g,  # noqa: E731
+                                                          alpha_grid=grid)
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    r0, r1 = row_range(W.shape[0], rank, world)
+    Wr = W[r0:r1].contiguous()
+    res = search_fn(Wr, alpha_grid) if r1 > r0 else None
+    shares = res.err_per_alpha if res is not None else [0.0] * len(alpha_grid)
+    errs = torch.tensor(shares, dtype=torch.float64, device=W.device)
+    dist.all_reduce(errs, op=dist.ReduceOp.SUM, group=group)
+    errs = errs.tolist()
+    k = first_minimum(errs)
+    if res is not None and first_minimum(res.err_per_alpha) != k:
+        res = search_fn(Wr, [alpha_grid[k]])
+    if res is None:  # no rows here: s from a one-row call keeps every rank's s alike
+        one = search_fn(W[:1].contiguous(), [alpha_grid[k]])
+        s = one.s
+        qweight = one.qweight[:0]
+        scales = one.scales[:0]
+    else:
+        s, qweight, scales = res.s, res.qweight, res.scales
+    if gather:
+        qweight = _gather_rows(qweight, W.shape[0], world, group)
+        scales = _gather_rows(scales, W.shape[0], world, group)
+    return alpha_grid[k], s, qweight, scales, errs

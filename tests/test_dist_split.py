@@ -130,3 +130,94 @@ def test_ranges_cover_every_row_once():
             assert all(a[1] == b[0] for a, b in zip(rr, rr[1:]))
             sizes = [b - a for a, b in rr]
             assert max(sizes) - min(sizes) <= 1
+
+
+# ---------------------------------------------------------------- AWQ, rows split
+
+AwqRes = collections.namedtuple("AwqRes", "best_alpha s qweight scales err_per_alpha")
+
+
+def _awq_layer(out):
+    import sys
+    sys.path.insert(0, ROOT)
+    from workloads import make_weight, make_x_bits, small_spec
+    spec = small_spec(out, 256, 700, seed=37, sigma_ln=1.0, n_outlier=4, outlier_gain=30.0)
+    return make_weight(spec), make_x_bits(spec)
+
+
+def _oracle_search(Wr, X, grid, bits, g):
+    """Stand-in for awq_search_layer on a block of rows (the FP64 oracle)."""
+    import oracle as O
+    r = O.awq_ref(Wr.numpy(), X, bits=bits, g=g, grid=grid)
+    return AwqRes(r.best_alpha, torch.from_numpy(r.s.astype(np.float32)),
+                  torch.from_numpy(O.pack_ref(r.codes, bits).view(np.int32)),
+                  torch.from_numpy(r.scales.astype(np.float16)), list(r.err))
+
+
+GRID = [k / 10.0 for k in range(10)]
+
+
+def _awq_worker(rank, world, port, out, q):
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                          WORLD_SIZE=str(world))
+        import sys
+        sys.path.insert(0, ROOT)
+        import datetime
+
+        import torch.distributed as dist
+
+        from post_int4_weight_gptq_b200.split import awq_layer_split
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        W, X = _awq_layer(out)
+        alpha, s, qw, sc, errs = awq_layer_split(
+            torch.from_numpy(W), X, bits=3, g=64, alpha_grid=GRID,
+            search_fn=lambda Wr, grid: _oracle_search(Wr, X, grid, 3, 64))
+        q.put((rank, alpha, s.numpy(), qw.numpy(), sc.numpy(), errs))
+        dist.destroy_process_group()
+    except Exception as e:  # the parent fails fast instead of waiting on the queue
+        q.put((rank, repr(e)))
+        raise
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,out", [(2, 12), (3, 2)])
+def test_awq_rows_split_equals_the_whole_layer(world, out):
+    """Each rank scores every alpha on its rows, one all-reduce sums the scores:
+    the chosen alpha, s, codes and scales are the whole layer's (a rank with no
+    rows, world 3 over 2 rows, still takes part in every collective)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_awq_worker, args=(r, world, port, out, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=240) for _ in procs), key=lambda t: t[0])
+    assert all(len(r) > 2 for r in res), res
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    import sys
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    from post_int4_weight_gptq_b200.split import first_minimum, row_range
+    W, X = _awq_layer(out)
+    ref = O.awq_ref(W, X, bits=3, g=64, grid=GRID)
+    if world == 2:  # rank 0's own rows prefer another alpha: its re-quantization is exercised
+        r0, r1 = row_range(out, 0, world)
+        own = O.awq_ref(W[r0:r1], X, bits=3, g=64, grid=GRID)
+        assert first_minimum(list(own.err)) != ref.best_index
+    for rank, alpha, s, qw, sc, errs in res:
+        assert alpha == ref.best_alpha
+        assert np.array_equal(s, ref.s.astype(np.float32))
+        assert np.array_equal(qw.view(np.uint32), O.pack_ref(ref.codes, 3))
+        assert np.array_equal(sc, ref.scales.astype(np.float16))
+        assert np.allclose(errs, ref.err, rtol=1e-12, atol=0)
+
+
+def test_first_minimum_is_the_first_on_a_tie():
+    from post_int4_weight_gptq_b200.split import first_minimum
+    assert first_minimum([3.0, 1.0, 2.0, 1.0]) == 1
+    assert first_minimum([5.0]) == 0
+    assert first_minimum([2.0, 2.0]) == 0

@@ -124,3 +124,85 @@ def test_two_gpus_give_the_bits_of_the_emulated_split():
     for _, qw_r, sc_r, err_r in res:
         assert np.array_equal(qw_r, qw) and np.array_equal(sc_r, sc)
         assert err_r == pytest.approx(sum(p.err for p in parts), rel=1e-12)
+
+
+# ---------------------------------------------------------------- AWQ, rows split
+
+GRID = tuple(k / 20.0 for k in range(20))
+
+
+def _emulated_awq_split(W, X, world):
+    """awq_layer_split's steps for `world` ranks, one after the other on this GPU."""
+    from post_int4_weight_gptq_b200.split import first_minimum
+    Xg = to_gpu_x(X)
+    blocks = [row_range(W.shape[0], r, world) for r in range(world)]
+    res = [piq.awq_search_layer(to_gpu_w(W[r0:r1]), Xg, bits=4, g=128, alpha_grid=GRID)
+           for r0, r1 in blocks]
+    errs = [sum(r.err_per_alpha[k] for r in res) for k in range(len(GRID))]
+    k = first_minimum(errs)
+    for i, (r0, r1) in enumerate(blocks):
+        if first_minimum(res[i].err_per_alpha) != k:
+            res[i] = piq.awq_search_layer(to_gpu_w(W[r0:r1]), Xg, bits=4, g=128,
+                                          alpha_grid=[GRID[k]])
+    return GRID[k], res, errs
+
+
+def test_awq_row_blocks_equal_one_call_on_all_rows():
+    # s depends on X only and each alpha's error is a sum over rows: blocks of
+    # rows scored apart and summed choose the whole layer's alpha, and give its bits
+    W, X = _layer(63)
+    alpha, parts, errs = _emulated_awq_split(W, X, 3)
+    whole = piq.awq_search_layer(to_gpu_w(W), to_gpu_x(X), bits=4, g=128, alpha_grid=GRID)
+    assert np.float32(alpha) == np.float32(whole.best_alpha)
+    assert np.allclose(errs, whole.err_per_alpha, rtol=1e-12, atol=0)
+    assert all(torch.equal(p.s, whole.s) for p in parts)
+    assert torch.equal(torch.cat([p.qweight for p in parts]), whole.qweight)
+    assert torch.equal(torch.cat([p.scales for p in parts]), whole.scales)
+    ref = O.awq_ref(W, X, bits=4, g=128, grid=list(GRID))
+    e = np.sort(ref.err)
+    if (e[1] - e[0]) / e[0] > 1e-4:  # not tie-ambiguous: the oracle's alpha too
+        assert alpha == ref.best_alpha
+
+
+def _awq_worker(rank, world, port, q):
+    import datetime
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from post_int4_weight_gptq_b200.split import awq_layer_split
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), NCCL_NVLS_ENABLE="0")
+    torch.cuda.set_device(rank)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    W, X = _layer(63)
+    alpha, s, qw, sc, errs = awq_layer_split(to_gpu_w(W, f"cuda:{rank}"),
+                                             to_gpu_x(X, f"cuda:{rank}"), bits=4, g=128,
+                                             alpha_grid=GRID)
+    q.put((rank, alpha, s.cpu().numpy(), qw.cpu().numpy(), sc.cpu().numpy(), errs))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two GPUs")
+@pytest.mark.timeout(600)
+def test_two_gpus_give_the_awq_bits_of_the_emulated_split():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_awq_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=500) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    W, X = _layer(63)
+    alpha, parts, errs = _emulated_awq_split(W, X, 2)
+    qw = torch.cat([p.qweight for p in parts]).cpu().numpy()
+    sc = torch.cat([p.scales for p in parts]).cpu().numpy()
+    for _, alpha_r, s_r, qw_r, sc_r, errs_r in res:
+        assert alpha_r == alpha
+        assert np.array_equal(s_r, parts[0].s.cpu().numpy())
+        assert np.array_equal(qw_r, qw) and np.array_equal(sc_r, sc)
+        assert np.allclose(errs_r, errs, rtol=1e-12, atol=0)
