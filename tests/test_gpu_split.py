@@ -154,7 +154,9 @@ def test_awq_row_blocks_equal_one_call_on_all_rows():
     alpha, parts, errs = _emulated_awq_split(W, X, 3)
     whole = piq.awq_search_layer(to_gpu_w(W), to_gpu_x(X), bits=4, g=128, alpha_grid=GRID)
     assert np.float32(alpha) == np.float32(whole.best_alpha)
-    assert np.allclose(errs, whole.err_per_alpha, rtol=1e-12, atol=0)
+    # the error GEMM sums tiles of rows in FP32 before FP64: blocks of rows round
+    # apart (~1e-9 relative here), far inside the gaps between alphas
+    assert np.allclose(errs, whole.err_per_alpha, rtol=1e-6, atol=0)
     assert all(torch.equal(p.s, whole.s) for p in parts)
     assert torch.equal(torch.cat([p.qweight for p in parts]), whole.qweight)
     assert torch.equal(torch.cat([p.scales for p in parts]), whole.scales)
