@@ -286,6 +286,18 @@ const char* piq_phase_name(int i);
  * number of launches.  Any pointer may be NULL.  Host-side state, per process. */
 int piq_last_gemm_stats(double* ms, double* int8_ops, int* launches);
 
+/* The tile order of the INT8 digit GEMM (host only, no device work): tiles are
+ * 128 rows of C by 48 columns; a launch with m_tiles x n_tiles tiles (only the
+ * tiles that reach the lower triangle when lower != 0: column tile n of row
+ * tile m with 48 n <= 128 m + 127) takes them in groups of eight row tiles,
+ * column tiles outer inside a group, then, for lower launches, each group's
+ * remaining tiles row by row; persistent CTA c takes tiles c, c + grid, ...
+ * Returns the launch's tile count, or a negative status (m_tiles or n_tiles
+ * < 1, more than 2^31 - 1 tiles).  With mt and nt non-NULL (host int arrays of
+ * `count` >= that many entries) tile t's row and column tile are written to
+ * mt[t] and nt[t]; a smaller count is PIQ_ERR_INVALID_ARG. */
+int64_t piq_gemm_tile_order(int m_tiles, int n_tiles, int lower, int64_t count, int* mt, int* nt);
+
 /* Number of kernels this library has launched in this process (all devices);
  * a monotone diagnostic counter. */
 uint64_t piq_kernel_launches(void);

@@ -92,6 +92,7 @@ SIGNATURES = {
     "piq_phase_name": (ctypes.c_char_p, [_c_int]),
     "piq_last_gemm_stats": (_c_int, [ctypes.POINTER(ctypes.c_double),
                                      ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
+    "piq_gemm_tile_order": (_c_i64, [_c_int, _c_int, _c_int, _c_i64, _vp, _vp]),
     "piq_kernel_launches": (ctypes.c_uint64, []),
     "piq_simt_gemm_fallbacks": (ctypes.c_uint64, []),
     "piq_last_cuda_error": (ctypes.c_char_p, []),
@@ -434,6 +435,23 @@ def last_gemm_stats() -> dict:
     ms, ops, n = ctypes.c_double(0.0), ctypes.c_double(0.0), ctypes.c_int(0)
     lib.piq_last_gemm_stats(ctypes.byref(ms), ctypes.byref(ops), ctypes.byref(n))
     return {"ms": ms.value, "int8_ops": ops.value, "launches": n.value}
+
+
+def gemm_tile_order(m_tiles: int, n_tiles: int, lower: bool = False):
+    """(mt, nt): int32 arrays, the row and column tile of each tile of an INT8
+    digit GEMM launch in the order its CTAs take them (host only)."""
+    import numpy as np
+    lib = load_library()
+    total = int(lib.piq_gemm_tile_order(m_tiles, n_tiles, int(bool(lower)), 0, None, None))
+    if total < 0:
+        _check(total, "piq_gemm_tile_order")
+    mt = np.empty(total, dtype=np.int32)
+    nt = np.empty(total, dtype=np.int32)
+    rc = int(lib.piq_gemm_tile_order(m_tiles, n_tiles, int(bool(lower)), total,
+                                     mt.ctypes.data, nt.ctypes.data))
+    if rc < 0:
+        _check(rc, "piq_gemm_tile_order")
+    return mt, nt
 
 
 def kernel_launches() -> int:

@@ -114,7 +114,7 @@ __host__ __device__ __forceinline__ int64_t lower_prefix(int m, int n_tiles) {
 // way, then its staircase row by row.
 constexpr int RG = 8;
 
-__device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& nt) {
+__host__ __device__ __forceinline__ void tile_of(const OzParams& p, int t, int& mt, int& nt) {
   if (p.lower) {
     int lo = 0, hi = (p.m_tiles + RG - 1) / RG - 1;  // the last group g with prefix <= t
     while (lo < hi) {
@@ -595,3 +595,23 @@ int launch_ozaki_gemm(int64_t M, int64_t N, const DigitMat& A, const DigitMat& B
 }
 
 }  // namespace piq
+
+// The order in which the digit GEMM's persistent CTAs take their tiles (tile
+// t of a launch is taken by CTA t mod grid), for tests and tools.
+extern "C" int64_t piq_gemm_tile_order(int m_tiles, int n_tiles, int lower, int64_t count,
+                                       int* mt, int* nt) {
+  using namespace piq;
+  if (m_tiles < 1 || n_tiles < 1) return PIQ_ERR_INVALID_ARG;
+  const int64_t total = lower ? lower_prefix(m_tiles, n_tiles)
+                              : static_cast<int64_t>(m_tiles) * n_tiles;
+  if (total > INT32_MAX) return PIQ_ERR_INVALID_ARG;
+  if (mt == nullptr || nt == nullptr) return total;
+  if (count < total) return PIQ_ERR_INVALID_ARG;
+  OzParams p{};
+  p.m_tiles = m_tiles;
+  p.n_tiles = n_tiles;
+  p.num_tiles = static_cast<int>(total);
+  p.lower = lower ? 1 : 0;
+  for (int t = 0; t < p.num_tiles; ++t) tile_of(p, t, mt[t], nt[t]);
+  return total;
+}

@@ -124,3 +124,38 @@ def test_empty_and_oversized_layers_rejected(lib):
         assert rc == piq.PIQ_ERR_INVALID_ARG, (rows, inp, n)
     for args in ((0, 64, 64, 128, 0), (16, 0, 64, 128, 0), (16, 64, 0, 128, 0), (16, 64, 64, 0, 0)):
         assert lib.piq_gptq_workspace_bytes(*args, ctypes.byref(out)) == piq.PIQ_ERR_INVALID_ARG
+
+
+def _lower_cols(m, n_tiles):
+    # column tiles of row tile m (128 rows) that reach the lower triangle (48 columns each)
+    return min(n_tiles, (128 * m + 127) // 48 + 1)
+
+
+@pytest.mark.parametrize("m_tiles,n_tiles", [(1, 1), (1, 7), (3, 1), (8, 3), (9, 3), (17, 40),
+                                             (64, 171), (215, 574), (224, 3), (23, 598)])
+@pytest.mark.parametrize("lower", [False, True])
+def test_gemm_tile_order_visits_every_tile_once_by_row_groups(lib, m_tiles, n_tiles, lower):
+    import numpy as np
+    mt, nt = piq.gemm_tile_order(m_tiles, n_tiles, lower)
+    cols = [_lower_cols(m, n_tiles) if lower else n_tiles for m in range(m_tiles)]
+    assert len(mt) == sum(cols)
+    assert ((mt >= 0) & (mt < m_tiles)).all() and (nt >= 0).all()
+    assert (nt < np.asarray(cols)[mt]).all()
+    assert len(set(zip(mt.tolist(), nt.tolist()))) == len(mt)    # each tile once
+    # groups of eight row tiles, one after another; column tiles outer inside a
+    # group wherever every row of the group has the column
+    grp = mt // 8
+    assert (np.diff(grp) >= 0).all()
+    for g0 in range(0, m_tiles, 8):
+        sel = grp == g0 // 8
+        full = nt[sel] < cols[g0]
+        assert (np.diff(nt[sel][full]) >= 0).all()
+        assert full[:full.sum()].all()                              # full columns first
+
+
+def test_gemm_tile_order_rejects_bad_sizes(lib):
+    assert lib.piq_gemm_tile_order(0, 3, 0, 0, None, None) < 0
+    assert lib.piq_gemm_tile_order(3, 0, 1, 0, None, None) < 0
+    import numpy as np
+    a = np.empty(2, dtype=np.int32)
+    assert lib.piq_gemm_tile_order(2, 2, 0, 2, a.ctypes.data, a.ctypes.data) < 0  # 4 tiles
